@@ -1,0 +1,748 @@
+// Host side of libspa: argument checks, workspace and handle management,
+// tensor-map encoding and the launch sequence of each C-ABI call.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include <cuda_bf16.h>
+
+#include "../../include/spa.h"
+#include "spa_internal.h"
+
+namespace spa {
+int singular_proxy_host(const float* w_v, int d, int r, float* w_r, int iters);
+}
+
+using namespace spa;
+
+// ---------------------------------------------------------------------------
+// errors
+// ---------------------------------------------------------------------------
+static thread_local char g_last_error[512] = "";
+
+static int fail(int status, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return status;
+}
+
+#define SPA_CK(call)                                                                     \
+  do {                                                                                   \
+    cudaError_t e_ = (call);                                                             \
+    if (e_ != cudaSuccess) return fail(SPA_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+#define SPA_TRY(expr)          \
+  do {                         \
+    int s_ = (expr);           \
+    if (s_ != SPA_OK) return s_; \
+  } while (0)
+
+extern "C" const char* spa_status_string(int status) {
+  switch (status) {
+    case SPA_OK: return "SPA_OK";
+    case SPA_ERR_INVALID: return "SPA_ERR_INVALID";
+    case SPA_ERR_SHAPE: return "SPA_ERR_SHAPE";
+    case SPA_ERR_CUDA: return "SPA_ERR_CUDA";
+    case SPA_ERR_NOMEM: return "SPA_ERR_NOMEM";
+    case SPA_ERR_UNSUPPORTED: return "SPA_ERR_UNSUPPORTED";
+    case SPA_ERR_TIMEOUT: return "SPA_ERR_TIMEOUT";
+    case SPA_ERR_DEVICE: return "SPA_ERR_DEVICE";
+    default: return "SPA_ERR_UNKNOWN";
+  }
+}
+
+extern "C" const char* spa_last_error(void) { return g_last_error; }
+extern "C" int spa_version(void) { return 100; }
+
+// ---------------------------------------------------------------------------
+// budget
+// ---------------------------------------------------------------------------
+extern "C" double spa_rho(int l, int L, double rho_p, int l_p, double rho_1, double rho_L) {
+  if (L < 1 || l < 1 || l > L || l_p < 1 || l_p > L || !(rho_p > 0) || !(rho_1 > 0) ||
+      !(rho_L > 0) || !std::isfinite(rho_p) || !std::isfinite(rho_1) || !std::isfinite(rho_L))
+    return NAN;
+  if (l <= l_p) {
+    if (l_p == 1) return rho_p;
+    const double t = (double)(l - l_p) / (double)(l_p - 1);
+    return rho_p * std::exp(std::log(rho_1 / rho_p) * t * t);
+  }
+  const double t = (double)(l - l_p) / (double)(L - l_p);
+  return rho_p * std::exp(std::log(rho_L / rho_p) * t * t);
+}
+
+extern "C" int spa_budget_k(int N, double rho) {
+  if (N < 1 || !std::isfinite(rho) || !(rho > 0)) return -1;
+  const double x = std::ceil((double)N * rho);
+  if (x >= (double)N) return N;
+  if (x < 1.0) return 1;
+  return (int)x;
+}
+
+extern "C" int spa_singular_proxy_host(const float* w_v, int d, int r, float* w_r_out) {
+  if (!w_v || !w_r_out) return fail(SPA_ERR_INVALID, "spa_singular_proxy_host: null pointer");
+  if (d < 1 || r < 1 || r > d) return fail(SPA_ERR_SHAPE, "spa_singular_proxy_host: bad d=%d r=%d", d, r);
+  try {
+    if (singular_proxy_host(w_v, d, r, w_r_out, 24) != 0)
+      return fail(SPA_ERR_INVALID, "spa_singular_proxy_host failed");
+  } catch (const std::bad_alloc&) {
+    return fail(SPA_ERR_NOMEM, "spa_singular_proxy_host: host allocation failed");
+  }
+  return SPA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// handles
+// ---------------------------------------------------------------------------
+struct spa_workspace {
+  spa_layer_desc desc;
+  int device = 0;
+  int max_B = 0, max_N = 0, cap = 0;  // cap = max_B * max_N token rows
+  size_t elem = 4;
+  float* a_hat = nullptr;   // [cap, r]
+  float* score = nullptr;   // [cap]
+  int32_t* idx = nullptr;   // [cap]
+  void* X = nullptr;        // [cap, d]
+  void* Q = nullptr;        // [cap, d]
+  void* O = nullptr;        // [cap, d]
+  void* H1 = nullptr;       // [cap, d]
+  void* X2 = nullptr;       // [cap, d]
+  void* A = nullptr;        // [cap, F]
+  float* part_o = nullptr;  // attention split partials
+  float* part_ml = nullptr;
+  int part_rows = 0;
+  int* err = nullptr;       // [2]
+  float* rope_cos = nullptr;  // [max_N, hd/2]
+  float* rope_sin = nullptr;
+  CUtensorMap tmX, tmO, tmX2, tmA;
+  int num_sms = 148;
+  std::vector<void*> allocs;
+};
+
+struct spa_layer {
+  spa_layer_desc desc;
+  spa_layer_weights w;
+  spa_workspace* ws = nullptr;
+  void* w_r = nullptr;      // [r, d] dtype
+  CUtensorMap tm_wq, tm_wk, tm_wv, tm_wo, tm_wg, tm_wu, tm_wd, tm_wr;
+};
+
+struct spa_model {
+  spa_model_desc desc;
+  std::vector<spa_layer*> layers;
+  std::vector<spa_layer_cache> caches;
+  std::vector<int> k;
+  void* h0 = nullptr;
+  const void* embed = nullptr;
+  const void* final_norm = nullptr;
+  const void* lm_head = nullptr;
+  int32_t* idx_all = nullptr;  // [L, B, N] index sets of the last step
+  float* amax_val = nullptr;   // [B*N, n_tiles]
+  int32_t* amax_idx = nullptr;
+  int lm_tiles = 0;
+  CUtensorMap tm_lm;
+};
+
+static int check_desc(const spa_layer_desc* d) {
+  if (!d) return fail(SPA_ERR_INVALID, "null layer descriptor");
+  if (d->dtype != SPA_F32 && d->dtype != SPA_BF16) return fail(SPA_ERR_INVALID, "dtype must be SPA_F32 or SPA_BF16");
+  if (d->d < 4 || d->n_heads < 1 || d->head_dim < 2 || d->ffn < 4 || d->r < 1)
+    return fail(SPA_ERR_SHAPE, "non-positive dimension");
+  if (d->n_heads * d->head_dim != d->d) return fail(SPA_ERR_SHAPE, "d != n_heads * head_dim");
+  if (d->head_dim % 8 != 0 || d->head_dim > 128) return fail(SPA_ERR_UNSUPPORTED, "head_dim must be a multiple of 8, <= 128");
+  if (d->r > d->d) return fail(SPA_ERR_SHAPE, "r > d");
+  if (!(d->rms_eps > 0.f) || !(d->rope_theta > 0.f)) return fail(SPA_ERR_INVALID, "eps and theta must be positive");
+  if (d->dtype == SPA_BF16) {
+    if (d->d % 256 != 0) return fail(SPA_ERR_UNSUPPORTED, "bf16: d must be a multiple of 256");
+    if (d->ffn % 128 != 0) return fail(SPA_ERR_UNSUPPORTED, "bf16: ffn must be a multiple of 128");
+    if (d->r > 256) return fail(SPA_ERR_UNSUPPORTED, "bf16: r must be <= 256");
+  } else {
+    if (d->d % 4 != 0 || d->ffn % 4 != 0) return fail(SPA_ERR_UNSUPPORTED, "f32: d and ffn must be multiples of 4");
+    if (d->r > 128) return fail(SPA_ERR_UNSUPPORTED, "f32: r must be <= 128");
+    if (128 % d->head_dim != 0) return fail(SPA_ERR_UNSUPPORTED, "f32: head_dim must divide 128");
+  }
+  return SPA_OK;
+}
+
+static int ws_alloc(spa_workspace* ws, void** p, size_t bytes) {
+  if (bytes == 0) bytes = 16;
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(SPA_ERR_NOMEM, "cudaMalloc(%zu) failed: %s", bytes, cudaGetErrorString(e));
+  }
+  ws->allocs.push_back(*p);
+  return SPA_OK;
+}
+
+extern "C" void spa_workspace_free(spa_workspace* ws) {
+  if (!ws) return;
+  for (void* p : ws->allocs) cudaFree(p);
+  delete ws;
+}
+
+extern "C" int spa_workspace_create(const spa_layer_desc* desc, int max_B, int max_N,
+                                    spa_workspace** out) {
+  if (!out) return fail(SPA_ERR_INVALID, "null output handle");
+  *out = nullptr;
+  SPA_TRY(check_desc(desc));
+  if (max_B < 1 || max_N < 1) return fail(SPA_ERR_SHAPE, "max_B and max_N must be >= 1");
+  if (max_N > 8192) return fail(SPA_ERR_UNSUPPORTED, "N > 8192 is not supported by the top-k select");
+  if ((long long)max_B * max_N > (1ll << 24)) return fail(SPA_ERR_SHAPE, "max_B * max_N too large");
+  spa_workspace* ws = new (std::nothrow) spa_workspace();
+  if (!ws) return fail(SPA_ERR_NOMEM, "host allocation failed");
+  ws->desc = *desc;
+  ws->max_B = max_B;
+  ws->max_N = max_N;
+  ws->cap = max_B * max_N;
+  ws->elem = desc->dtype == SPA_BF16 ? 2 : 4;
+  cudaGetDevice(&ws->device);
+  cudaDeviceGetAttribute(&ws->num_sms, cudaDevAttrMultiProcessorCount, ws->device);
+  const size_t cap = ws->cap, d = desc->d, F = desc->ffn, r = desc->r, e = ws->elem;
+  ws->part_rows = (int)std::min<size_t>(cap, 4096) * 4;
+  int st = SPA_OK;
+  void* p;
+#define WS_ALLOC(field, bytes) \
+  if (st == SPA_OK) { st = ws_alloc(ws, &p, (bytes)); if (st == SPA_OK) ws->field = (decltype(ws->field))p; }
+  WS_ALLOC(a_hat, cap * r * 4)
+  WS_ALLOC(score, cap * 4)
+  WS_ALLOC(idx, cap * 4)
+  WS_ALLOC(X, cap * d * e)
+  WS_ALLOC(Q, cap * d * e)
+  WS_ALLOC(O, cap * d * e)
+  WS_ALLOC(H1, cap * d * e)
+  WS_ALLOC(X2, cap * d * e)
+  WS_ALLOC(A, cap * F * e)
+  WS_ALLOC(part_o, (size_t)ws->part_rows * d * 4)
+  WS_ALLOC(part_ml, (size_t)ws->part_rows * desc->n_heads * 2 * 4)
+  WS_ALLOC(err, 2 * sizeof(int))
+  WS_ALLOC(rope_cos, (size_t)max_N * (desc->head_dim / 2) * 4)
+  WS_ALLOC(rope_sin, (size_t)max_N * (desc->head_dim / 2) * 4)
+#undef WS_ALLOC
+  if (st != SPA_OK) {
+    spa_workspace_free(ws);
+    return st;
+  }
+  // RoPE table in double precision: angle = pos * theta^(-2i/hd)
+  const int hh = desc->head_dim / 2;
+  std::vector<float> cs((size_t)max_N * hh), sn((size_t)max_N * hh);
+  for (int pos = 0; pos < max_N; ++pos)
+    for (int i = 0; i < hh; ++i) {
+      const double inv = std::pow((double)desc->rope_theta, -2.0 * i / (double)desc->head_dim);
+      const double a = (double)pos * inv;
+      cs[(size_t)pos * hh + i] = (float)std::cos(a);
+      sn[(size_t)pos * hh + i] = (float)std::sin(a);
+    }
+  if (cudaMemcpy(ws->rope_cos, cs.data(), cs.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy(ws->rope_sin, sn.data(), sn.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemset(ws->err, 0, 2 * sizeof(int)) != cudaSuccess) {
+    spa_workspace_free(ws);
+    return fail(SPA_ERR_CUDA, "workspace initialisation copy failed");
+  }
+  if (desc->dtype == SPA_BF16) {
+    if (encode_bf16_map(&ws->tmX, ws->X, cap, d) || encode_bf16_map(&ws->tmO, ws->O, cap, d) ||
+        encode_bf16_map(&ws->tmX2, ws->X2, cap, d) || encode_bf16_map(&ws->tmA, ws->A, cap, F)) {
+      spa_workspace_free(ws);
+      return fail(SPA_ERR_CUDA, "tensor map encoding failed");
+    }
+  }
+  *out = ws;
+  return SPA_OK;
+}
+
+extern "C" int spa_workspace_status(spa_workspace* ws, void* stream) {
+  if (!ws) return fail(SPA_ERR_INVALID, "null workspace");
+  SPA_CK(cudaStreamSynchronize((cudaStream_t)stream));
+  int h[2] = {0, 0};
+  SPA_CK(cudaMemcpy(h, ws->err, sizeof(h), cudaMemcpyDeviceToHost));
+  if (h[0] == 0) return SPA_OK;
+  SPA_CK(cudaMemset(ws->err, 0, sizeof(h)));
+  if (h[0] & DEVERR_TIMEOUT) return fail(SPA_ERR_TIMEOUT, "device wait timed out (site %d)", h[1]);
+  return fail(SPA_ERR_DEVICE, "device check failed: bits 0x%x site %d", h[0], h[1]);
+}
+
+extern "C" int spa_workspace_intermediates(const spa_workspace* ws, spa_intermediates* out) {
+  if (!ws || !out) return fail(SPA_ERR_INVALID, "null argument");
+  out->x = ws->X;
+  out->q = ws->Q;
+  out->o = ws->O;
+  out->h1 = ws->H1;
+  out->x2 = ws->X2;
+  out->a = ws->A;
+  out->a_hat = ws->a_hat;
+  out->score = ws->score;
+  return SPA_OK;
+}
+
+extern "C" void spa_free_layer(spa_layer* layer) {
+  if (!layer) return;
+  if (layer->w_r) cudaFree(layer->w_r);
+  delete layer;
+}
+
+extern "C" int spa_init_layer(const spa_layer_desc* desc, const spa_layer_weights* w,
+                              const float* w_r_host, spa_workspace* ws, spa_layer** out) {
+  if (!out) return fail(SPA_ERR_INVALID, "null output handle");
+  *out = nullptr;
+  SPA_TRY(check_desc(desc));
+  if (!w || !ws) return fail(SPA_ERR_INVALID, "null weights or workspace");
+  if (!w->wq || !w->wk || !w->wv || !w->wo || !w->w_gate || !w->w_up || !w->w_down ||
+      !w->attn_norm || !w->ffn_norm)
+    return fail(SPA_ERR_INVALID, "null weight pointer");
+  if (std::memcmp(desc, &ws->desc, sizeof(spa_layer_desc)) != 0)
+    return fail(SPA_ERR_SHAPE, "layer descriptor differs from the workspace's");
+  const int d = desc->d, r = desc->r;
+  std::vector<float> wr;
+  try {
+    wr.resize((size_t)r * d);
+    if (w_r_host) {
+      std::memcpy(wr.data(), w_r_host, wr.size() * 4);
+    } else {
+      std::vector<float> wv((size_t)d * d);
+      if (desc->dtype == SPA_BF16) {
+        std::vector<__nv_bfloat16> tmp((size_t)d * d);
+        SPA_CK(cudaMemcpy(tmp.data(), w->wv, tmp.size() * 2, cudaMemcpyDeviceToHost));
+        for (size_t i = 0; i < tmp.size(); ++i) wv[i] = __bfloat162float(tmp[i]);
+      } else {
+        SPA_CK(cudaMemcpy(wv.data(), w->wv, wv.size() * 4, cudaMemcpyDeviceToHost));
+      }
+      SPA_TRY(spa_singular_proxy_host(wv.data(), d, r, wr.data()));
+    }
+  } catch (const std::bad_alloc&) {
+    return fail(SPA_ERR_NOMEM, "host allocation failed");
+  }
+  spa_layer* L = new (std::nothrow) spa_layer();
+  if (!L) return fail(SPA_ERR_NOMEM, "host allocation failed");
+  L->desc = *desc;
+  L->w = *w;
+  L->ws = ws;
+  const size_t e = desc->dtype == SPA_BF16 ? 2 : 4;
+  if (cudaMalloc(&L->w_r, (size_t)r * d * e) != cudaSuccess) {
+    cudaGetLastError();
+    delete L;
+    return fail(SPA_ERR_NOMEM, "cudaMalloc of the proxy weights failed");
+  }
+  int st = SPA_OK;
+  if (desc->dtype == SPA_BF16) {
+    std::vector<__nv_bfloat16> b((size_t)r * d);
+    for (size_t i = 0; i < b.size(); ++i) b[i] = __float2bfloat16_rn(wr[i]);
+    if (cudaMemcpy(L->w_r, b.data(), b.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess)
+      st = fail(SPA_ERR_CUDA, "proxy weight upload failed");
+    const uint64_t D = d, F = desc->ffn;
+    if (st == SPA_OK &&
+        (encode_bf16_map(&L->tm_wq, w->wq, D, D) || encode_bf16_map(&L->tm_wk, w->wk, D, D) ||
+         encode_bf16_map(&L->tm_wv, w->wv, D, D) || encode_bf16_map(&L->tm_wo, w->wo, D, D) ||
+         encode_bf16_map(&L->tm_wg, w->w_gate, F, D) || encode_bf16_map(&L->tm_wu, w->w_up, F, D) ||
+         encode_bf16_map(&L->tm_wd, w->w_down, D, F) || encode_bf16_map(&L->tm_wr, L->w_r, r, D)))
+      st = fail(SPA_ERR_CUDA, "tensor map encoding failed (weights must be 16-byte aligned)");
+  } else {
+    if (cudaMemcpy(L->w_r, wr.data(), wr.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess)
+      st = fail(SPA_ERR_CUDA, "proxy weight upload failed");
+  }
+  if (st != SPA_OK) {
+    spa_free_layer(L);
+    return st;
+  }
+  *out = L;
+  return SPA_OK;
+}
+
+extern "C" int spa_layer_proxy_weights(const spa_layer* layer, float* w_r_out) {
+  if (!layer || !w_r_out) return fail(SPA_ERR_INVALID, "null argument");
+  const size_t n = (size_t)layer->desc.r * layer->desc.d;
+  if (layer->desc.dtype == SPA_BF16) {
+    std::vector<__nv_bfloat16> b(n);
+    SPA_CK(cudaMemcpy(b.data(), layer->w_r, n * 2, cudaMemcpyDeviceToHost));
+    for (size_t i = 0; i < n; ++i) w_r_out[i] = __bfloat162float(b[i]);
+  } else {
+    SPA_CK(cudaMemcpy(w_r_out, layer->w_r, n * 4, cudaMemcpyDeviceToHost));
+  }
+  return SPA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// launch helpers
+// ---------------------------------------------------------------------------
+static EpiParams base_epi(const spa_layer* L, int M, int tps, int N, const int32_t* idx) {
+  EpiParams ep;
+  std::memset(&ep, 0, sizeof(ep));
+  ep.M = M;
+  ep.d = L->desc.d;
+  ep.head_dim = L->desc.head_dim;
+  ep.tokens_per_seq = tps;
+  ep.N = N;
+  ep.idx = idx;
+  ep.rope_cos = L->ws->rope_cos;
+  ep.rope_sin = L->ws->rope_sin;
+  ep.err = L->ws->err;
+  return ep;
+}
+
+// Number of K-splits for a weight-streaming GEMM: as many CTAs as fit one
+// wave of the SMs, at least 4 k-blocks of 64 per CTA, cluster size <= 8.
+static int choose_splits(int tiles, int KB, int sms) {
+  int best = 1;
+  for (int s = 1; s <= 8; ++s) {
+    if (KB / s < 4) break;
+    if (tiles * s <= sms) best = s;
+  }
+  return best;
+}
+
+static int run_tc(int mode, int BN, TcGemmParams& p, int M, int n_tiles, int splits, cudaStream_t s) {
+  const int m_tiles = (M + 127) / 128;
+  if (m_tiles == 0) return SPA_OK;
+  if (m_tiles > 65535 || n_tiles > 65535) return fail(SPA_ERR_SHAPE, "GEMM grid too large");
+  cudaError_t e = launch_tc_gemm(mode, BN, p, m_tiles, n_tiles, splits, s);
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "tc GEMM launch (mode %d): %s", mode, cudaGetErrorString(e));
+  return SPA_OK;
+}
+
+static int run_simt(int mode, SimtGemmParams& p, int M, int n_tiles, cudaStream_t s) {
+  const int m_tiles = (M + 63) / 64;
+  if (m_tiles == 0) return SPA_OK;
+  cudaError_t e = launch_simt_gemm(mode, p, m_tiles, n_tiles, s);
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "SIMT GEMM launch (mode %d): %s", mode, cudaGetErrorString(e));
+  return SPA_OK;
+}
+
+static int check_cache(const spa_layer* L, const spa_layer_cache* c) {
+  if (!c) return fail(SPA_ERR_INVALID, "null cache");
+  if (!c->k_cache || !c->v_cache || !c->h_cache || !c->p_cache) return fail(SPA_ERR_INVALID, "null cache buffer");
+  if (c->B < 1 || c->N < 1 || c->B > L->ws->max_B || c->N > L->ws->max_N ||
+      (long long)c->B * c->N > L->ws->cap)
+    return fail(SPA_ERR_SHAPE, "cache B=%d N=%d exceeds the workspace (B<=%d, N<=%d)", c->B, c->N,
+                L->ws->max_B, L->ws->max_N);
+  return SPA_OK;
+}
+
+// Phase 1: proxy GEMM with the fused norm / score epilogue (or the P^c fill).
+static int run_proxy(spa_layer* L, const void* H, const spa_layer_cache* c, float* score, int fill,
+                     cudaStream_t s) {
+  const int M = c->B * c->N, d = L->desc.d, r = L->desc.r;
+  EpiParams ep = base_epi(L, M, c->N, c->N, nullptr);
+  ep.n_out = r;
+  ep.a_hat = L->ws->a_hat;
+  ep.p_cache = c->p_cache;
+  ep.score = score;
+  ep.proxy_fill = fill;
+  if (L->desc.dtype == SPA_BF16) {
+    TcGemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    if (encode_bf16_map(&p.tmA, H, (uint64_t)M, (uint64_t)d))
+      return fail(SPA_ERR_CUDA, "tensor map for H failed (H must be 16-byte aligned)");
+    p.tmB[0] = L->tm_wr;
+    p.K = d;
+    p.b_mode = B_SINGLE;
+    p.b_rows_per_src = r;
+    p.ep = ep;
+    // split count depends on d only, so a row's proxy bits never depend on B or N
+    const int splits = std::max(1, std::min(8, (d / 64) / 4));
+    return run_tc(EPI_PROXY, r <= 128 ? 128 : 256, p, M, 1, splits, s);
+  }
+  SimtGemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.A = (const float*)H;
+  p.B[0] = (const float*)L->w_r;
+  p.K = d;
+  p.b_mode = B_SINGLE;
+  p.b_rows_per_src = r;
+  p.ep = ep;
+  return run_simt(EPI_PROXY, p, M, 1, s);
+}
+
+// Phases 2 and 3 for M = B * tps tokens; idx == null means every row (rho = 1).
+static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
+                     const spa_layer_cache* c, cudaStream_t s) {
+  spa_workspace* ws = L->ws;
+  const spa_layer_desc& D = L->desc;
+  const int d = D.d, F = D.ffn, M = c->B * tps, N = c->N;
+  const bool bf = D.dtype == SPA_BF16;
+  cudaError_t e;
+  // x = RMSNorm(H[I])
+  e = launch_rmsnorm_rows(D.dtype, H, 1, idx, tps, N, M, d, L->w.attn_norm, D.rms_eps, ws->X, ws->err, s);
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "rmsnorm launch: %s", cudaGetErrorString(e));
+  // Q, K, V with RoPE; K, V scattered into the caches
+  {
+    EpiParams ep = base_epi(L, M, tps, N, idx);
+    ep.n_out = 3 * d;
+    ep.out = ws->Q;
+    ep.k_cache = c->k_cache;
+    ep.v_cache = c->v_cache;
+    if (bf) {
+      TcGemmParams p;
+      std::memset(&p, 0, sizeof(p));
+      p.tmA = ws->tmX;
+      p.tmB[0] = L->tm_wq; p.tmB[1] = L->tm_wk; p.tmB[2] = L->tm_wv;
+      p.K = d; p.b_mode = B_CONCAT3; p.b_rows_per_src = d; p.ep = ep;
+      const int nt = 3 * d / 256, mt = (M + 127) / 128;
+      SPA_TRY(run_tc(EPI_QKV, 256, p, M, nt, choose_splits(nt * mt, d / 64, ws->num_sms), s));
+    } else {
+      SimtGemmParams p;
+      std::memset(&p, 0, sizeof(p));
+      p.A = (const float*)ws->X;
+      p.B[0] = (const float*)L->w.wq; p.B[1] = (const float*)L->w.wk; p.B[2] = (const float*)L->w.wv;
+      p.K = d; p.b_mode = B_CONCAT3; p.b_rows_per_src = d; p.ep = ep;
+      SPA_TRY(run_simt(EPI_QKV, p, M, (3 * d + 127) / 128, s));
+    }
+  }
+  // O = attention over the whole cache
+  e = launch_attention(D.dtype, ws->Q, c->k_cache, c->v_cache, ws->O, c->B, tps, N, D.n_heads,
+                       D.head_dim, ws->part_o, ws->part_ml, ws->part_rows, ws->err, s);
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
+  // H1 = H[I] + O W_o^T
+  {
+    EpiParams ep = base_epi(L, M, tps, N, idx);
+    ep.n_out = d;
+    ep.out = ws->H1;
+    ep.resid = H;
+    if (bf) {
+      TcGemmParams p;
+      std::memset(&p, 0, sizeof(p));
+      p.tmA = ws->tmO; p.tmB[0] = L->tm_wo;
+      p.K = d; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
+      const int nt = d / 256, mt = (M + 127) / 128;
+      SPA_TRY(run_tc(EPI_RESID, 256, p, M, nt, choose_splits(nt * mt, d / 64, ws->num_sms), s));
+    } else {
+      SimtGemmParams p;
+      std::memset(&p, 0, sizeof(p));
+      p.A = (const float*)ws->O; p.B[0] = (const float*)L->w.wo;
+      p.K = d; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
+      SPA_TRY(run_simt(EPI_RESID, p, M, (d + 127) / 128, s));
+    }
+  }
+  // x2 = RMSNorm(H1)
+  e = launch_rmsnorm_rows(D.dtype, ws->H1, 0, nullptr, tps, N, M, d, L->w.ffn_norm, D.rms_eps, ws->X2, ws->err, s);
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "rmsnorm launch: %s", cudaGetErrorString(e));
+  // A = silu(x2 W_gate^T) * (x2 W_up^T)
+  {
+    EpiParams ep = base_epi(L, M, tps, N, idx);
+    ep.n_out = F;
+    ep.out = ws->A;
+    if (bf) {
+      TcGemmParams p;
+      std::memset(&p, 0, sizeof(p));
+      p.tmA = ws->tmX2; p.tmB[0] = L->tm_wg; p.tmB[1] = L->tm_wu;
+      p.K = d; p.b_mode = B_GATEUP; p.b_rows_per_src = F; p.ep = ep;
+      const int nt = F / 128, mt = (M + 127) / 128;
+      SPA_TRY(run_tc(EPI_SWIGLU, 256, p, M, nt, choose_splits(nt * mt, d / 64, ws->num_sms), s));
+    } else {
+      SimtGemmParams p;
+      std::memset(&p, 0, sizeof(p));
+      p.A = (const float*)ws->X2; p.B[0] = (const float*)L->w.w_gate; p.B[1] = (const float*)L->w.w_up;
+      p.K = d; p.b_mode = B_GATEUP; p.b_rows_per_src = F; p.ep = ep;
+      SPA_TRY(run_simt(EPI_SWIGLU, p, M, (F + 63) / 64, s));
+    }
+  }
+  // H^c[I] = H1 + A W_down^T
+  {
+    EpiParams ep = base_epi(L, M, tps, N, idx);
+    ep.n_out = d;
+    ep.out = c->h_cache;
+    ep.resid = ws->H1;
+    if (bf) {
+      TcGemmParams p;
+      std::memset(&p, 0, sizeof(p));
+      p.tmA = ws->tmA; p.tmB[0] = L->tm_wd;
+      p.K = F; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
+      const int nt = d / 256, mt = (M + 127) / 128;
+      SPA_TRY(run_tc(EPI_RESID_SCATTER, 256, p, M, nt, choose_splits(nt * mt, F / 64, ws->num_sms), s));
+    } else {
+      SimtGemmParams p;
+      std::memset(&p, 0, sizeof(p));
+      p.A = (const float*)ws->A; p.B[0] = (const float*)L->w.w_down;
+      p.K = F; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
+      SPA_TRY(run_simt(EPI_RESID_SCATTER, p, M, (d + 127) / 128, s));
+    }
+  }
+  return SPA_OK;
+}
+
+static int check_H(const void* H) {
+  if (!H) return fail(SPA_ERR_INVALID, "null H");
+  if (reinterpret_cast<uintptr_t>(H) % 16 != 0) return fail(SPA_ERR_INVALID, "H must be 16-byte aligned");
+  return SPA_OK;
+}
+
+extern "C" int spa_proxy_select(spa_layer* L, const void* H, const spa_layer_cache* c, int k,
+                                int32_t* idx, float* score, void* stream) {
+  if (!L) return fail(SPA_ERR_INVALID, "null layer");
+  SPA_TRY(check_H(H));
+  SPA_TRY(check_cache(L, c));
+  if (!idx) return fail(SPA_ERR_INVALID, "null idx");
+  if (k < 1 || k > c->N) return fail(SPA_ERR_SHAPE, "k=%d outside [1, N=%d]", k, c->N);
+  cudaStream_t s = (cudaStream_t)stream;
+  float* sc = score ? score : L->ws->score;
+  SPA_TRY(run_proxy(L, H, c, sc, 0, s));
+  cudaError_t e = launch_topk_select(sc, c->B, c->N, k, idx, L->ws->a_hat, c->p_cache, L->desc.r, L->ws->err, s);
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "top-k launch: %s", cudaGetErrorString(e));
+  return SPA_OK;
+}
+
+extern "C" int spa_partial_block(spa_layer* L, const void* H, const int32_t* idx, int k,
+                                 const spa_layer_cache* c, void* stream) {
+  if (!L) return fail(SPA_ERR_INVALID, "null layer");
+  SPA_TRY(check_H(H));
+  SPA_TRY(check_cache(L, c));
+  if (!idx) return fail(SPA_ERR_INVALID, "null idx");
+  if (k < 1 || k > c->N) return fail(SPA_ERR_SHAPE, "k=%d outside [1, N=%d]", k, c->N);
+  return run_block(L, H, idx, k, c, (cudaStream_t)stream);
+}
+
+extern "C" int spa_layer_step(spa_layer* L, const void* H, const spa_layer_cache* c, int k,
+                              int32_t* idx, void* stream) {
+  SPA_TRY(spa_proxy_select(L, H, c, k, idx, nullptr, stream));
+  return run_block(L, H, idx, k, c, (cudaStream_t)stream);
+}
+
+extern "C" int spa_full_block(spa_layer* L, const void* H, const spa_layer_cache* c, int fill_proxy,
+                              void* stream) {
+  if (!L) return fail(SPA_ERR_INVALID, "null layer");
+  SPA_TRY(check_H(H));
+  SPA_TRY(check_cache(L, c));
+  cudaStream_t s = (cudaStream_t)stream;
+  if (fill_proxy) SPA_TRY(run_proxy(L, H, c, nullptr, 1, s));
+  return run_block(L, H, nullptr, c->N, c, s);
+}
+
+// ---------------------------------------------------------------------------
+// model / decode
+// ---------------------------------------------------------------------------
+extern "C" void spa_model_free(spa_model* m) {
+  if (!m) return;
+  if (m->idx_all) cudaFree(m->idx_all);
+  if (m->amax_val) cudaFree(m->amax_val);
+  if (m->amax_idx) cudaFree(m->amax_idx);
+  delete m;
+}
+
+extern "C" int spa_model_create(const spa_model_desc* desc, spa_layer* const* layers,
+                                const spa_layer_cache* caches, void* h0, const void* embed,
+                                const void* final_norm, const void* lm_head, spa_model** out) {
+  if (!out) return fail(SPA_ERR_INVALID, "null output handle");
+  *out = nullptr;
+  if (!desc || !layers || !caches || !h0 || !embed || !final_norm || !lm_head)
+    return fail(SPA_ERR_INVALID, "null argument");
+  if (desc->n_layers < 1 || desc->vocab < 2 || desc->B < 1 || desc->N < 1)
+    return fail(SPA_ERR_SHAPE, "bad model sizes");
+  spa_workspace* ws = layers[0] ? layers[0]->ws : nullptr;
+  if (!ws) return fail(SPA_ERR_INVALID, "null layer");
+  for (int l = 0; l < desc->n_layers; ++l) {
+    if (!layers[l] || layers[l]->ws != ws) return fail(SPA_ERR_INVALID, "every layer must share one workspace");
+    SPA_TRY(check_cache(layers[l], &caches[l]));
+    if (caches[l].B != desc->B || caches[l].N != desc->N) return fail(SPA_ERR_SHAPE, "cache shape differs from the model's");
+  }
+  spa_model* m = new (std::nothrow) spa_model();
+  if (!m) return fail(SPA_ERR_NOMEM, "host allocation failed");
+  m->desc = *desc;
+  m->layers.assign(layers, layers + desc->n_layers);
+  m->caches.assign(caches, caches + desc->n_layers);
+  m->h0 = h0;
+  m->embed = embed;
+  m->final_norm = final_norm;
+  m->lm_head = lm_head;
+  for (int l = 1; l <= desc->n_layers; ++l) {
+    const double rho = spa_rho(l, desc->n_layers, desc->rho_p, desc->l_p, desc->rho_1, desc->rho_L);
+    const int k = spa_budget_k(desc->N, rho);
+    if (k < 1) {
+      delete m;
+      return fail(SPA_ERR_INVALID, "invalid rho parameters");
+    }
+    m->k.push_back(k);
+  }
+  const spa_layer_desc& D = ws->desc;
+  const int BN = D.dtype == SPA_BF16 ? 256 : 128;
+  m->lm_tiles = (desc->vocab + BN - 1) / BN;
+  const size_t rows = (size_t)desc->B * desc->N;
+  if (cudaMalloc(&m->idx_all, (size_t)desc->n_layers * rows * 4) != cudaSuccess ||
+      cudaMalloc(&m->amax_val, rows * m->lm_tiles * 4) != cudaSuccess ||
+      cudaMalloc(&m->amax_idx, rows * m->lm_tiles * 4) != cudaSuccess) {
+    cudaGetLastError();
+    spa_model_free(m);
+    return fail(SPA_ERR_NOMEM, "model buffers: cudaMalloc failed");
+  }
+  if (D.dtype == SPA_BF16 && encode_bf16_map(&m->tm_lm, lm_head, desc->vocab, D.d)) {
+    spa_model_free(m);
+    return fail(SPA_ERR_CUDA, "tensor map for the LM head failed");
+  }
+  *out = m;
+  return SPA_OK;
+}
+
+extern "C" int spa_model_layer_k(const spa_model* m, int layer) {
+  if (!m || layer < 0 || layer >= (int)m->k.size()) return -1;
+  return m->k[layer];
+}
+
+extern "C" int spa_model_embed(spa_model* m, const int32_t* tokens, void* stream) {
+  if (!m || !tokens) return fail(SPA_ERR_INVALID, "null argument");
+  spa_workspace* ws = m->layers[0]->ws;
+  cudaError_t e = launch_embed_rows(ws->desc.dtype, m->embed, tokens, nullptr, m->desc.B, m->desc.N,
+                                    m->desc.N, ws->desc.d, m->desc.vocab, m->h0, ws->err,
+                                    (cudaStream_t)stream);
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "embed launch: %s", cudaGetErrorString(e));
+  return SPA_OK;
+}
+
+extern "C" int spa_decode_step(spa_model* m, const int32_t* pos, const int32_t* tok_in, int u,
+                               int full, int32_t* tok_out, void* stream) {
+  if (!m || !pos || !tok_out) return fail(SPA_ERR_INVALID, "null argument");
+  if (full < 0 || full > 2) return fail(SPA_ERR_INVALID, "full must be 0, 1 or 2");
+  if (u < 1 || u > m->desc.N) return fail(SPA_ERR_SHAPE, "u=%d outside [1, N]", u);
+  cudaStream_t s = (cudaStream_t)stream;
+  spa_workspace* ws = m->layers[0]->ws;
+  const spa_layer_desc& D = ws->desc;
+  const int L = m->desc.n_layers, B = m->desc.B, N = m->desc.N, d = D.d;
+  const size_t rows = (size_t)B * N;
+  for (int l = 0; l < L; ++l) {
+    const void* H = (l == 0) ? m->h0 : m->caches[l - 1].h_cache;
+    if (full) {
+      SPA_TRY(spa_full_block(m->layers[l], H, &m->caches[l], full == 1 ? 1 : 0, stream));
+    } else {
+      SPA_TRY(spa_layer_step(m->layers[l], H, &m->caches[l], m->k[l], m->idx_all + l * rows, stream));
+    }
+  }
+  // final RMSNorm at the u positions, LM head, argmax
+  cudaError_t e = launch_gather_final(D.dtype, m->caches[L - 1].h_cache, pos, B, u, N, d,
+                                      m->final_norm, D.rms_eps, ws->X, ws->err, s);
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "final norm launch: %s", cudaGetErrorString(e));
+  const int M = B * u;
+  EpiParams ep;
+  std::memset(&ep, 0, sizeof(ep));
+  ep.M = M;
+  ep.n_out = m->desc.vocab;
+  ep.d = d;
+  ep.tokens_per_seq = u;
+  ep.N = N;
+  ep.amax_val = m->amax_val;
+  ep.amax_idx = m->amax_idx;
+  ep.n_tiles = m->lm_tiles;
+  ep.err = ws->err;
+  if (D.dtype == SPA_BF16) {
+    TcGemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.tmA = ws->tmX;
+    p.tmB[0] = m->tm_lm;
+    p.K = d; p.b_mode = B_SINGLE; p.b_rows_per_src = m->desc.vocab; p.ep = ep;
+    SPA_TRY(run_tc(EPI_ARGMAX, 256, p, M, m->lm_tiles, 1, s));
+  } else {
+    SimtGemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.A = (const float*)ws->X; p.B[0] = (const float*)m->lm_head;
+    p.K = d; p.b_mode = B_SINGLE; p.b_rows_per_src = m->desc.vocab; p.ep = ep;
+    SPA_TRY(run_simt(EPI_ARGMAX, p, M, m->lm_tiles, s));
+  }
+  e = launch_argmax_reduce(m->amax_val, m->amax_idx, M, m->lm_tiles, tok_out, s);
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "argmax launch: %s", cudaGetErrorString(e));
+  // next step's layer-0 input: embeddings of the written ids at pos
+  e = launch_embed_rows(D.dtype, m->embed, tok_in ? tok_in : tok_out, pos, B, u, N, d, m->desc.vocab,
+                        m->h0, ws->err, s);
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "embed launch: %s", cudaGetErrorString(e));
+  return SPA_OK;
+}

@@ -1,0 +1,502 @@
+// GEMMs of the SPA-Cache layer step with their fused epilogues.
+//
+// tc_gemm_kernel (bf16, sm_100a tensor cores): one CTA computes a 128 x BN
+// fp32 tile of D = A . B^T in TMEM.  Warp 0 streams A (token rows) and B
+// (weight rows) tiles of 64 columns through a STAGES-deep TMA ring with
+// 128-byte swizzling; one thread of warp 1 issues tcgen05.mma (M = 128,
+// N = BN, K = 16) and frees each stage with tcgen05.commit.  Split-K runs
+// across the CTAs of a thread-block cluster: each CTA stages its partial tile
+// in shared memory, and CTA q sums rows [q*128/S, (q+1)*128/S) of all S
+// partials through distributed shared memory in the fixed order 0..S-1, so
+// results are deterministic and each output row depends only on its own
+// input row.  The epilogue then applies the step's fused operation.
+//
+// simt_gemm_kernel (fp32, CUDA cores): 64 x 128 tiles with the same epilogues,
+// for the fp32 configurations.
+#include <cstdio>
+
+#include <cudaTypedefs.h>
+
+#include "spa_device.cuh"
+#include "spa_internal.h"
+
+namespace spa {
+
+// ---------------------------------------------------------------------------
+// Epilogues over an fp32 tile held in shared memory (row-major, stride ld).
+// ---------------------------------------------------------------------------
+struct TokenRow {
+  int b, pos;
+  bool ok;
+};
+
+__device__ __forceinline__ TokenRow token_row(const EpiParams& ep, int t) {
+  TokenRow r;
+  r.b = t / ep.tokens_per_seq;
+  r.pos = ep.idx ? ep.idx[t] : (t % ep.tokens_per_seq);
+  r.ok = (r.pos >= 0 && r.pos < ep.N);
+  if (!r.ok) report_error(ep.err, DEVERR_INDEX, 101);
+  return r;
+}
+
+__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+
+template <int MODE, int BN, typename T>
+__device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_end, int gm0,
+                             int n_tile, const EpiParams& ep, int tid, int nthr) {
+  const int nrows = row_end - row_begin;
+  if (nrows <= 0) return;
+
+  if constexpr (MODE == EPI_STORE || MODE == EPI_RESID || MODE == EPI_RESID_SCATTER) {
+    constexpr int C4 = BN / 4;
+    const int gn0 = n_tile * BN;
+    for (int it = tid; it < nrows * C4; it += nthr) {
+      const int row = row_begin + it / C4, c = (it % C4) * 4;
+      const int t = gm0 + row, gn = gn0 + c;
+      if (t >= ep.M || gn >= ep.n_out) continue;
+      float4 v = *reinterpret_cast<const float4*>(tile + row * ld + c);
+      if constexpr (MODE == EPI_STORE) {
+        store4(reinterpret_cast<T*>(ep.out) + (size_t)t * ep.n_out + gn, v);
+      } else if constexpr (MODE == EPI_RESID) {
+        TokenRow tr = token_row(ep, t);
+        if (!tr.ok) continue;
+        float4 h = load4(reinterpret_cast<const T*>(ep.resid) +
+                         ((size_t)tr.b * ep.N + tr.pos) * ep.d + gn);
+        v.x += h.x; v.y += h.y; v.z += h.z; v.w += h.w;
+        store4(reinterpret_cast<T*>(ep.out) + (size_t)t * ep.d + gn, v);
+      } else {
+        TokenRow tr = token_row(ep, t);
+        if (!tr.ok) continue;
+        float4 h = load4(reinterpret_cast<const T*>(ep.resid) + (size_t)t * ep.d + gn);
+        v.x += h.x; v.y += h.y; v.z += h.z; v.w += h.w;
+        store4(reinterpret_cast<T*>(ep.out) + ((size_t)tr.b * ep.N + tr.pos) * ep.d + gn, v);
+      }
+    }
+  } else if constexpr (MODE == EPI_SWIGLU) {
+    constexpr int HALF = BN / 2, C4 = HALF / 4;
+    const int f0 = n_tile * HALF;
+    for (int it = tid; it < nrows * C4; it += nthr) {
+      const int row = row_begin + it / C4, c = (it % C4) * 4;
+      const int t = gm0 + row, f = f0 + c;
+      if (t >= ep.M || f >= ep.n_out) continue;
+      float4 g = *reinterpret_cast<const float4*>(tile + row * ld + c);
+      float4 u = *reinterpret_cast<const float4*>(tile + row * ld + HALF + c);
+      float4 a = make_float4(silu(g.x) * u.x, silu(g.y) * u.y, silu(g.z) * u.z, silu(g.w) * u.w);
+      store4(reinterpret_cast<T*>(ep.out) + (size_t)t * ep.n_out + f, a);
+    }
+  } else if constexpr (MODE == EPI_QKV) {
+    // Item = 4 rotary pairs (j..j+3, j+hd/2..j+hd/2+3) of one head of one row.
+    const int hd = ep.head_dim, hh = hd / 2;
+    const int items_per_head = hh / 4;
+    const int items = (BN / hd) * items_per_head;
+    const int gn0 = n_tile * BN;
+    for (int it = tid; it < nrows * items; it += nthr) {
+      const int row = row_begin + it / items, w = it % items;
+      const int t = gm0 + row;
+      if (t >= ep.M) continue;
+      const int hl = w / items_per_head, j = (w % items_per_head) * 4;
+      const int c1 = hl * hd + j, c2 = c1 + hh;
+      const int g1 = gn0 + c1;
+      if (g1 >= ep.n_out) continue;
+      const int part = g1 / ep.d, col1 = g1 % ep.d, col2 = col1 + hh;
+      float4 x1 = *reinterpret_cast<const float4*>(tile + row * ld + c1);
+      float4 x2 = *reinterpret_cast<const float4*>(tile + row * ld + c2);
+      TokenRow tr = token_row(ep, t);
+      if (!tr.ok) continue;
+      if (part < 2) {
+        const float4 cs = *reinterpret_cast<const float4*>(ep.rope_cos + (size_t)tr.pos * hh + j);
+        const float4 sn = *reinterpret_cast<const float4*>(ep.rope_sin + (size_t)tr.pos * hh + j);
+        float4 y1, y2;
+        y1.x = x1.x * cs.x - x2.x * sn.x; y2.x = x2.x * cs.x + x1.x * sn.x;
+        y1.y = x1.y * cs.y - x2.y * sn.y; y2.y = x2.y * cs.y + x1.y * sn.y;
+        y1.z = x1.z * cs.z - x2.z * sn.z; y2.z = x2.z * cs.z + x1.z * sn.z;
+        y1.w = x1.w * cs.w - x2.w * sn.w; y2.w = x2.w * cs.w + x1.w * sn.w;
+        x1 = y1; x2 = y2;
+      }
+      T* dst;
+      if (part == 0) dst = reinterpret_cast<T*>(ep.out) + (size_t)t * ep.d;
+      else dst = reinterpret_cast<T*>(part == 1 ? ep.k_cache : ep.v_cache) +
+                 ((size_t)tr.b * ep.N + tr.pos) * ep.d;
+      store4(dst + col1, x1);
+      store4(dst + col2, x2);
+    }
+  } else if constexpr (MODE == EPI_PROXY) {
+    // One warp per token row: norm, unit proxy, drift score.
+    const int lane = tid & 31, wid = tid >> 5, nw = nthr >> 5;
+    const int r = ep.n_out;
+    for (int row = row_begin + wid; row < row_end; row += nw) {
+      const int t = gm0 + row;
+      if (t >= ep.M) continue;
+      const float* src = tile + row * ld;
+      float ss = 0.f;
+      for (int c = lane; c < r; c += 32) ss += src[c] * src[c];
+      ss = warp_sum(ss);
+      const float nrm = sqrtf(ss);
+      float sd = 0.f;
+      for (int c = lane; c < r; c += 32) {
+        const float a = ss > 0.f ? src[c] / nrm : 0.f;
+        if (ep.proxy_fill) {
+          ep.p_cache[(size_t)t * r + c] = a;
+        } else {
+          ep.a_hat[(size_t)t * r + c] = a;
+          const float df = a - ep.p_cache[(size_t)t * r + c];
+          sd += df * df;
+        }
+      }
+      if (!ep.proxy_fill) {
+        sd = warp_sum(sd);
+        if (lane == 0) ep.score[t] = 0.5f * sd;
+      }
+    }
+  } else if constexpr (MODE == EPI_ARGMAX) {
+    const int lane = tid & 31, wid = tid >> 5, nw = nthr >> 5;
+    const int gn0 = n_tile * BN;
+    for (int row = row_begin + wid; row < row_end; row += nw) {
+      const int t = gm0 + row;
+      if (t >= ep.M) continue;
+      float best = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int c = lane; c < BN; c += 32) {
+        const int gn = gn0 + c;
+        if (gn >= ep.n_out) break;
+        const float v = tile[row * ld + c];
+        if (v > best) { best = v; bi = gn; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > best || (ov == best && oi < bi)) { best = ov; bi = oi; }
+      }
+      if (lane == 0) {
+        ep.amax_val[(size_t)t * ep.n_tiles + n_tile] = best;
+        ep.amax_idx[(size_t)t * ep.n_tiles + n_tile] = bi;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// tcgen05 GEMM
+// ---------------------------------------------------------------------------
+template <int BN>
+__device__ __forceinline__ void b_source(const TcGemmParams& p, int n_tile, int half, int& src,
+                                         int& row) {
+  if (p.b_mode == B_GATEUP) {
+    src = half;
+    row = n_tile * 128;
+  } else if (p.b_mode == B_CONCAT3) {
+    const int g = n_tile * BN + half * 128;
+    src = g / p.b_rows_per_src;
+    row = g % p.b_rows_per_src;
+  } else {
+    src = 0;
+    row = n_tile * BN + half * 128;
+  }
+}
+
+constexpr int kTcStages = 4;
+constexpr int kTcABytes = 128 * 128;  // 128 rows x 64 bf16
+
+__host__ __device__ constexpr int tc_smem_bytes(int BN) {
+  return kTcStages * (kTcABytes + BN * 128) + 1024;
+}
+
+template <int MODE, int BN>
+__global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
+  constexpr int B_BYTES = BN * 128;
+  constexpr int STAGE_BYTES = kTcABytes + B_BYTES;
+  constexpr int LD = BN + 4;
+  static_assert(128 * LD * 4 <= kTcStages * STAGE_BYTES, "epilogue tile must fit the ring");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full_bar[kTcStages];
+  __shared__ __align__(8) uint64_t empty_bar[kTcStages];
+  __shared__ __align__(8) uint64_t accum_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x, S = gridDim.x;
+  const int n_tile = blockIdx.y, m_tile = blockIdx.z;
+  const int KB = p.K / 64;
+  const int kb0 = (split * KB) / S, kb1 = ((split + 1) * KB) / S;
+  const int nk = kb1 - kb0;
+  int* err = p.ep.err;
+
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&accum_bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // TMA producer
+    tma_prefetch_desc(&p.tmA);
+    for (int it = 0; it < nk; ++it) {
+      const int s = it % kTcStages;
+      if (it >= kTcStages &&
+          !mbar_wait(&empty_bar[s], ((it / kTcStages) - 1) & 1, &abort_flag, err, 201))
+        break;
+      uint8_t* sa = smem + s * STAGE_BYTES;
+      uint8_t* sb = sa + kTcABytes;
+      mbar_arrive_expect_tx(&full_bar[s], STAGE_BYTES);
+      const int kx = (kb0 + it) * 64;
+      tma_load_2d(sa, &p.tmA, &full_bar[s], kx, m_tile * 128);
+#pragma unroll
+      for (int h = 0; h < BN / 128; ++h) {
+        int src, row;
+        b_source<BN>(p, n_tile, h, src, row);
+        tma_load_2d(sb + h * 128 * 128, &p.tmB[src], &full_bar[s], kx, row);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // MMA issuer
+    constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
+    for (int it = 0; it < nk; ++it) {
+      const int s = it % kTcStages;
+      if (!mbar_wait(&full_bar[s], (it / kTcStages) & 1, &abort_flag, err, 202)) break;
+      tc_fence_after();
+      const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
+      const uint64_t da = smem_desc_sw128(sa);
+      const uint64_t db = smem_desc_sw128(sa + kTcABytes);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        umma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+      umma_commit(&empty_bar[s]);
+    }
+    umma_commit(&accum_bar);
+  }
+  __syncwarp();
+
+  mbar_wait(&accum_bar, 0, &abort_flag, err, 203);
+  __syncthreads();
+  const bool good = (abort_flag == 0);
+  tc_fence_after();
+
+  float* tile = reinterpret_cast<float*>(smem);
+  if (good) {
+    const int row = warp * 32 + lane;
+    float* dst = tile + row * LD;
+    if (nk > 0) {
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(dst + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      }
+    } else {
+      for (int c = 0; c < BN; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(0, 0, 0, 0);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, BN);
+
+  const int gm0 = m_tile * 128;
+  if (S > 1) {
+    cluster_sync();
+    const int q = (int)cluster_ctarank();
+    const int r0 = (q * 128) / S, r1 = ((q + 1) * 128) / S;
+    if (good) {
+      constexpr int C4 = BN / 4;
+      for (int it = threadIdx.x; it < (r1 - r0) * C4; it += 128) {
+        const int row = r0 + it / C4, c = (it % C4) * 4;
+        const uint32_t local = smem_u32(tile + row * LD + c);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int src = 0; src < S; ++src) {
+          const float4 v = ld_dsmem_f4(mapa_shared(local, (uint32_t)src));
+          acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        *reinterpret_cast<float4*>(tile + row * LD + c) = acc;
+      }
+    }
+    cluster_sync();
+    if (good)
+      run_epilogue<MODE, BN, __nv_bfloat16>(tile, LD, r0, r1, gm0, n_tile, p.ep, threadIdx.x, 128);
+  } else {
+    if (good)
+      run_epilogue<MODE, BN, __nv_bfloat16>(tile, LD, 0, 128, gm0, n_tile, p.ep, threadIdx.x, 128);
+  }
+}
+
+template <int MODE, int BN>
+static cudaError_t launch_tc_typed(const TcGemmParams& p, int m_tiles, int n_tiles, int splits,
+                                   cudaStream_t stream) {
+  auto kern = tc_gemm_kernel<MODE, BN>;
+  const int smem = tc_smem_bytes(BN);
+  static bool configured = false;  // per instantiation
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(splits, n_tiles, m_tiles);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+cudaError_t launch_tc_gemm(int mode, int BN, const TcGemmParams& p, int m_tiles, int n_tiles,
+                           int splits, cudaStream_t stream) {
+#define SPA_TC_CASE(M_, BN_)                                           \
+  if (mode == M_ && BN == BN_) return launch_tc_typed<M_, BN_>(p, m_tiles, n_tiles, splits, stream);
+  SPA_TC_CASE(EPI_STORE, 128)
+  SPA_TC_CASE(EPI_STORE, 256)
+  SPA_TC_CASE(EPI_QKV, 256)
+  SPA_TC_CASE(EPI_RESID, 256)
+  SPA_TC_CASE(EPI_SWIGLU, 256)
+  SPA_TC_CASE(EPI_RESID_SCATTER, 256)
+  SPA_TC_CASE(EPI_PROXY, 128)
+  SPA_TC_CASE(EPI_PROXY, 256)
+  SPA_TC_CASE(EPI_ARGMAX, 256)
+#undef SPA_TC_CASE
+  return cudaErrorInvalidValue;
+}
+
+// ---------------------------------------------------------------------------
+// fp32 CUDA-core GEMM (64 x 128 tiles, 256 threads, 4 x 8 outputs per thread)
+// ---------------------------------------------------------------------------
+constexpr int kSBM = 64, kSBN = 128, kSBK = 16;
+
+__device__ __forceinline__ const float* simt_b_row(const SimtGemmParams& p, int n_tile, int c) {
+  int src, row;
+  if (p.b_mode == B_GATEUP) {
+    src = c < kSBN / 2 ? 0 : 1;
+    row = n_tile * (kSBN / 2) + (c % (kSBN / 2));
+  } else if (p.b_mode == B_CONCAT3) {
+    const int g = n_tile * kSBN + c;
+    src = g / p.b_rows_per_src;
+    row = g % p.b_rows_per_src;
+    if (src > 2) return nullptr;
+  } else {
+    src = 0;
+    row = n_tile * kSBN + c;
+  }
+  if (row >= p.b_rows_per_src) return nullptr;
+  return p.B[src] + (size_t)row * p.K;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtGemmParams p) {
+  __shared__ __align__(16) float As[kSBK][kSBM + 4];
+  __shared__ __align__(16) float Bs[kSBK][kSBN + 4];
+  __shared__ __align__(16) float tile[kSBM * (kSBN + 4)];
+  const int tid = threadIdx.x;
+  const int n_tile = blockIdx.x, m_tile = blockIdx.y;
+  const int ty = tid / 16, tx = tid % 16;
+  float acc[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+  // loaders: A: 64 rows x 16 k (4 per thread); B: 128 rows x 16 k (8 per thread)
+  const int a_row = tid / 4, a_k = (tid % 4) * 4;
+  const int ga = m_tile * kSBM + a_row;
+  const float* a_ptr = ga < p.ep.M ? p.A + (size_t)ga * p.K : nullptr;
+  const int b_row = tid / 2, b_k = (tid % 2) * 8;
+  const float* b_ptr = simt_b_row(p, n_tile, b_row);
+
+  for (int k0 = 0; k0 < p.K; k0 += kSBK) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int k = k0 + a_k + j;
+      As[a_k + j][a_row] = (a_ptr && k < p.K) ? a_ptr[k] : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int k = k0 + b_k + j;
+      Bs[b_k + j][b_row] = (b_ptr && k < p.K) ? b_ptr[k] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < kSBK; ++k) {
+      float a[4], b[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[k][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) b[j] = Bs[k][tx * 8 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  constexpr int LD = kSBN + 4;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) tile[(ty * 4 + i) * LD + tx * 8 + j] = acc[i][j];
+  __syncthreads();
+  run_epilogue<MODE, kSBN, float>(tile, LD, 0, kSBM, m_tile * kSBM, n_tile, p.ep, tid, 256);
+}
+
+cudaError_t launch_simt_gemm(int mode, const SimtGemmParams& p, int m_tiles, int n_tiles,
+                             cudaStream_t stream) {
+  dim3 grid(n_tiles, m_tiles), block(256);
+  switch (mode) {
+    case EPI_STORE: simt_gemm_kernel<EPI_STORE><<<grid, block, 0, stream>>>(p); break;
+    case EPI_QKV: simt_gemm_kernel<EPI_QKV><<<grid, block, 0, stream>>>(p); break;
+    case EPI_RESID: simt_gemm_kernel<EPI_RESID><<<grid, block, 0, stream>>>(p); break;
+    case EPI_SWIGLU: simt_gemm_kernel<EPI_SWIGLU><<<grid, block, 0, stream>>>(p); break;
+    case EPI_RESID_SCATTER: simt_gemm_kernel<EPI_RESID_SCATTER><<<grid, block, 0, stream>>>(p); break;
+    case EPI_PROXY: simt_gemm_kernel<EPI_PROXY><<<grid, block, 0, stream>>>(p); break;
+    case EPI_ARGMAX: simt_gemm_kernel<EPI_ARGMAX><<<grid, block, 0, stream>>>(p); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaPeekAtLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Tensor maps
+// ---------------------------------------------------------------------------
+int encode_bf16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (!encode) {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return -1;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -1;
+}
+
+}  // namespace spa

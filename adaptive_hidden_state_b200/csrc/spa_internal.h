@@ -1,0 +1,118 @@
+// Internal interfaces between the host API (spa_api.cu) and the kernel files.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace spa {
+
+// Bits of the device error word.
+enum : int {
+  DEVERR_TIMEOUT = 1,  // a bounded wait ran out
+  DEVERR_INDEX = 2,    // a gather/scatter index fell outside [0, N)
+  DEVERR_SHAPE = 4,    // a launch saw a shape it cannot handle
+};
+
+// What a GEMM does with its fp32 accumulator tile (rows = tokens, columns =
+// output features).  Every mode is a step of the cached layer update.
+enum EpiMode : int {
+  EPI_STORE = 0,          // out[t, n] = acc (dtype)                    - tests
+  EPI_QKV = 1,            // RoPE(Q) -> compact Q; RoPE(K), V -> K^c, V^c rows I
+  EPI_RESID = 2,          // H1[t] = acc + H[b, I[t]]
+  EPI_SWIGLU = 3,         // A[t, f] = silu(acc_gate) * acc_up
+  EPI_RESID_SCATTER = 4,  // H^c[b, I[t]] = acc + H1[t]
+  EPI_PROXY = 5,          // a_hat = acc/|acc|; s = 1/2|a_hat - P^c|^2 (or fill P^c)
+  EPI_ARGMAX = 6,         // per-tile (max, argmax) of the logits of each row
+};
+
+// How column tile n maps to rows of the weight sources.
+enum BMode : int {
+  B_SINGLE = 0,   // one matrix, rows n*BN ...
+  B_CONCAT3 = 1,  // [W_q; W_k; W_v] stacked, rows_per_src rows each
+  B_GATEUP = 2,   // first half of the tile from W_gate, second from W_up (same rows)
+};
+
+struct EpiParams {
+  int M;               // valid rows (tokens) of the GEMM
+  int n_out;           // logical output width (STORE: n; QKV: 3d; SWIGLU: F; PROXY: r; ARGMAX: vocab)
+  int d;               // model width (row stride of caches and compact buffers)
+  int head_dim;
+  int tokens_per_seq;  // token t belongs to sequence t / tokens_per_seq
+  int N;               // cache rows per sequence
+  const int32_t* idx;  // [B * tokens_per_seq] cache row of each token; null: row = t % tokens_per_seq
+  void* out;
+  void* k_cache;
+  void* v_cache;
+  const void* resid;
+  const float* rope_cos;  // [N, head_dim / 2]
+  const float* rope_sin;
+  float* a_hat;        // PROXY: [M, r]
+  float* p_cache;      // PROXY: [M, r]
+  float* score;        // PROXY: [M]
+  int proxy_fill;      // PROXY: 1 = write a_hat straight into p_cache
+  float* amax_val;     // ARGMAX: [M, n_tiles]
+  int32_t* amax_idx;
+  int n_tiles;
+  int* err;            // device error word
+};
+
+struct alignas(64) TcGemmParams {
+  CUtensorMap tmA;     // [M, K] bf16, box 64 x 128, 128-byte swizzle
+  CUtensorMap tmB[3];  // weight sources, box 64 x 128, 128-byte swizzle
+  int K;
+  int b_mode;
+  int b_rows_per_src;
+  EpiParams ep;
+};
+
+struct SimtGemmParams {
+  const float* A;      // [M, K]
+  const float* B[3];
+  int K;
+  int b_mode;
+  int b_rows_per_src;  // rows of each source matrix
+  EpiParams ep;
+};
+
+// tcgen05 GEMM: D[M, n] = A[M, K] . B[n, K]^T, BM = 128, BN = 128 or 256,
+// split-K across a thread-block cluster of `splits` CTAs with a fixed-order
+// reduction through distributed shared memory.
+cudaError_t launch_tc_gemm(int mode, int BN, const TcGemmParams& p, int m_tiles, int n_tiles,
+                           int splits, cudaStream_t stream);
+// fp32 CUDA-core GEMM with the same epilogues, BM = 64, BN = 128.
+cudaError_t launch_simt_gemm(int mode, const SimtGemmParams& p, int m_tiles, int n_tiles,
+                             cudaStream_t stream);
+
+// Encodes a 2D bf16 tensor map (rows x cols, row-major) with a 64 x 128 box.
+int encode_bf16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols);
+
+// ---- small kernels (spa_kernels.cu) ----
+// X[t] = RMSNorm(src[row(t)]) * gamma, row(t) = b * N + (idx ? idx[t] : t % tps) when
+// src_is_cache, else t.
+cudaError_t launch_rmsnorm_rows(int dtype, const void* src, int src_is_cache, const int32_t* idx,
+                                int tokens_per_seq, int N, int M, int d, const void* gamma,
+                                float eps, void* X, int* err, cudaStream_t stream);
+// Per sequence: top-k of score (ties to the lowest index) -> idx ascending,
+// then P^c[I] <- a_hat[I].
+cudaError_t launch_topk_select(const float* score, int B, int N, int k, int32_t* idx,
+                               const float* a_hat, float* p_cache, int r, int* err,
+                               cudaStream_t stream);
+// Sparse-query attention: O[t] = softmax(Q_t K^cT / sqrt(hd)) V^c per head.
+cudaError_t launch_attention(int dtype, const void* Q, const void* Kc, const void* Vc, void* O,
+                             int B, int k, int N, int n_heads, int head_dim, float* part_o,
+                             float* part_ml, int max_splits, int* err, cudaStream_t stream);
+// h0[b, pos] <- embed[tok] for the listed (or all) positions.
+cudaError_t launch_embed_rows(int dtype, const void* embed, const int32_t* tokens,
+                              const int32_t* pos, int B, int u, int N, int d, int vocab,
+                              void* h0, int* err, cudaStream_t stream);
+// Gathers final-layer rows at pos and applies the final RMSNorm.
+cudaError_t launch_gather_final(int dtype, const void* hc, const int32_t* pos, int B, int u, int N,
+                                int d, const void* gamma, float eps, void* X, int* err,
+                                cudaStream_t stream);
+// Reduces per-tile (max, argmax) partials to one id per row, lowest id on ties.
+cudaError_t launch_argmax_reduce(const float* val, const int32_t* idx, int rows, int n_tiles,
+                                 int32_t* out, cudaStream_t stream);
+// Copies a [rows] int32 array (device) element-wise.
+cudaError_t launch_copy_i32(const int32_t* src, int32_t* dst, int n, cudaStream_t stream);
+
+}  // namespace spa

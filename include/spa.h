@@ -1,0 +1,209 @@
+/*
+ * spa.h -- C ABI of libspa, the SPA-Cache cached transformer-block update on
+ * one NVIDIA B200 (sm_100a).
+ *
+ * SPA-Cache ("Singular Proxies for Adaptive Caching in Diffusion Language
+ * Models") refreshes only the k = ceil(N * rho(l)) tokens of layer l whose
+ * low-rank proxy drifted most since they were last refreshed, and reuses
+ * cached rows for the rest.  The operations below follow the three phases of
+ * the method's Algorithm 1 as given on the papernotes.org page (方法详解 >
+ * 整体框架) and the gist.science technical summary (Methodology, items 1-3).
+ *
+ * Conventions for every call:
+ *   - Returns a spa_status (0 = SPA_OK).  Arguments and shapes are checked
+ *     before anything is launched; a failing call launches nothing.
+ *   - Device work is enqueued on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream) and is asynchronous: no call below
+ *     synchronises the host unless it says so.
+ *   - Pointers marked "device" must point to device memory of the current
+ *     device; "host" pointers to host memory.  Matrices are row-major.
+ *     Weight matrices are stored [out, in] (y = W x).
+ *   - Element type: dtype SPA_F32 (float) or SPA_BF16 (__nv_bfloat16) for
+ *     weights, hidden states, K^c, V^c and H^c.  Proxies P^c, scores and the
+ *     proxy weights given from the host are always float.  Index sets are
+ *     int32, ascending.
+ *   - Ownership: the caller owns activations, caches and weights (borrowed:
+ *     they must outlive the handles that use them).  The library owns what
+ *     its create/init calls allocate and frees it in the matching free call.
+ *   - Device-side checks (gather/scatter indices out of range, a bounded wait
+ *     that ran out) do not fault: they set an error word in the workspace,
+ *     which spa_workspace_status() reads and clears.
+ *   - Handles are not thread-safe.  Calls that share a workspace must be
+ *     ordered on one stream.
+ */
+#ifndef SPA_H
+#define SPA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SPA_OK = 0,
+  SPA_ERR_INVALID = -1,     /* null pointer or a bad argument value */
+  SPA_ERR_SHAPE = -2,       /* a size outside what the handle was created for */
+  SPA_ERR_CUDA = -3,        /* a CUDA runtime/driver call or a launch failed */
+  SPA_ERR_NOMEM = -4,       /* device or host allocation failed */
+  SPA_ERR_UNSUPPORTED = -5, /* valid, but not built for this configuration */
+  SPA_ERR_TIMEOUT = -6,     /* a device-side bounded wait ran out */
+  SPA_ERR_DEVICE = -7       /* a device-side index check failed */
+} spa_status;
+
+enum { SPA_F32 = 0, SPA_BF16 = 1 };
+
+/* Static, NUL-terminated name of a status.  Thread-safe. */
+const char *spa_status_string(int status);
+/* Detail message of the last failing call on this host thread ("" if none). */
+const char *spa_last_error(void);
+/* Library version, 100*major + minor. */
+int spa_version(void);
+
+/* ---------------------------------------------------------------- budget --
+ * rho(l): piecewise-Gaussian update ratio of layer l (1-based) of L layers,
+ * peak rho_p at layer l_p, rho_1 at layer 1, rho_L at layer L (papernotes.org,
+ * 关键设计 3).  For l <= l_p: rho_p*exp(ln(rho_1/rho_p)*((l-l_p)/(l_p-1))^2);
+ * for l > l_p the same with rho_L and (L-l_p) (the branch the page calls
+ * symmetric, read so that rho(L) = rho_L).  Returns NaN on invalid input. */
+double spa_rho(int l, int L, double rho_p, int l_p, double rho_1, double rho_L);
+/* k = ceil(N * rho) clamped to [1, N] (Algorithm 1, phase 1: "k = N rho").
+ * Returns -1 on invalid input (N < 1, rho not finite or <= 0). */
+int spa_budget_k(int N, double rho);
+
+/* ------------------------------------------------------------ layer setup -- */
+typedef struct {
+  int d;          /* model width; multiple of 256 for SPA_BF16, of 4 for SPA_F32 */
+  int n_heads;    /* d = n_heads * head_dim */
+  int head_dim;   /* even; <= 128 */
+  int ffn;        /* SwiGLU hidden width F; multiple of 128 for SPA_BF16 */
+  int r;          /* proxy rank, 1 <= r <= min(d, 256) (SPA_F32: <= 128) */
+  int dtype;      /* SPA_F32 or SPA_BF16 */
+  float rms_eps;  /* RMSNorm epsilon */
+  float rope_theta;
+} spa_layer_desc;
+
+/* Device pointers of one layer's weights, dtype elements, borrowed.
+ * wq, wk, wv, wo: [d, d]; w_gate, w_up: [F, d]; w_down: [d, F];
+ * attn_norm, ffn_norm: [d] RMSNorm gains. */
+typedef struct {
+  const void *wq, *wk, *wv, *wo, *w_gate, *w_up, *w_down, *attn_norm, *ffn_norm;
+} spa_layer_weights;
+
+/* Host routine: W_r = Lambda_r V_r^T (r x d) from the truncated SVD of the
+ * Value weights, W_v ~= U Lambda V^T (papernotes.org, 关键设计 2).  w_v is the
+ * host [d, d] float matrix as stored ([out, in]); w_r_out receives r*d
+ * floats, each row's largest-magnitude entry made positive.  Randomised
+ * subspace iteration in double precision with oversampling; accuracy ~1e-6
+ * relative for spectra with a gap beyond r.  Synchronous, host only. */
+int spa_singular_proxy_host(const float *w_v, int d, int r, float *w_r_out);
+
+/* Scratch for the layer calls: sized for at most max_B sequences of max_N
+ * tokens.  One workspace can serve many layers of the same shape. */
+typedef struct spa_workspace spa_workspace;
+int spa_workspace_create(const spa_layer_desc *desc, int max_B, int max_N, spa_workspace **out);
+void spa_workspace_free(spa_workspace *ws);
+/* Synchronises `stream`, then reads and clears the device error word:
+ * SPA_OK, SPA_ERR_TIMEOUT or SPA_ERR_DEVICE. */
+int spa_workspace_status(spa_workspace *ws, void *stream);
+
+/* Device addresses of the workspace buffers that hold the intermediates of
+ * the last layer call, for inspection (valid until the workspace is freed;
+ * overwritten by the next call).  Rows t = b*k + i are the selected tokens in
+ * index-set order (k = N for spa_full_block): x = RMSNorm(H[I]) [B*k, d],
+ * q = RoPE(Q_I) [B*k, d], o = attention output [B*k, d], h1 = H[I] + o W_o^T
+ * [B*k, d], x2 = RMSNorm(h1) [B*k, d], a = silu(x2 W_gate^T) * (x2 W_up^T)
+ * [B*k, F] (dtype elements); a_hat [B*N, r] and score [B*N] (float) from
+ * the last spa_proxy_select. */
+typedef struct {
+  void *x, *q, *o, *h1, *x2, *a;
+  float *a_hat, *score;
+} spa_intermediates;
+int spa_workspace_intermediates(const spa_workspace *ws, spa_intermediates *out);
+
+/* A layer handle: borrows `w` and `ws`, owns its proxy weights W_r (stored in
+ * the layer dtype) and the RoPE table.  w_r_host (host, [r, d] float) is a
+ * proxy computed offline; NULL makes the library copy W_v to the host and run
+ * spa_singular_proxy_host (synchronous). */
+typedef struct spa_layer spa_layer;
+int spa_init_layer(const spa_layer_desc *desc, const spa_layer_weights *w, const float *w_r_host,
+                   spa_workspace *ws, spa_layer **out);
+void spa_free_layer(spa_layer *layer);
+/* Copies the stored proxy weights (as float) to host w_r_out [r, d]. */
+int spa_layer_proxy_weights(const spa_layer *layer, float *w_r_out);
+
+/* Caches of one layer for B sequences of N tokens (device, caller-owned):
+ * k_cache, v_cache: [B, N, d] post-RoPE keys and values; h_cache: [B, N, d]
+ * layer outputs; p_cache: [B, N, r] float unit proxies. */
+typedef struct {
+  void *k_cache, *v_cache, *h_cache;
+  float *p_cache;
+  int B, N;
+} spa_layer_cache;
+
+/* ----------------------------------------------------------- layer step --
+ * Phase 1, update identification (Algorithm 1; gist.science Methodology
+ * item 1): a = W_r h for every token of H ([B, N, d] device, the layer
+ * input), a_hat = a/|a|, s = 1/2 |a_hat - P^c|^2 (= 1 - cosine to the cached
+ * proxy), I = the k largest s per sequence with ties to the lowest index,
+ * written ascending to idx ([B, k] int32 device); then P^c[I] <- a_hat[I].
+ * score ([B, N] float device) receives s when non-NULL. */
+int spa_proxy_select(spa_layer *layer, const void *H, const spa_layer_cache *cache, int k,
+                     int32_t *idx, float *score, void *stream);
+
+/* Phases 2 and 3 for a given index set idx ([B, k] int32 device, ascending,
+ * entries in [0, N)): x = RMSNorm(H[I]); Q, K, V = x W^T; RoPE on Q, K at
+ * positions I; K^c[I] <- K, V^c[I] <- V; O = softmax(Q K^cT / sqrt(d_h)) V^c
+ * over all N cached rows; H1 = H[I] + O W_o^T;
+ * H^c[I] <- H1 + W_down(silu(W_gate x2) * W_up x2), x2 = RMSNorm(H1).
+ * Rows of H^c outside I are not touched. */
+int spa_partial_block(spa_layer *layer, const void *H, const int32_t *idx, int k,
+                      const spa_layer_cache *cache, void *stream);
+
+/* Phases 1-3 in one call: spa_proxy_select then spa_partial_block. */
+int spa_layer_step(spa_layer *layer, const void *H, const spa_layer_cache *cache, int k,
+                   int32_t *idx, void *stream);
+
+/* rho = 1 pass (the uncached forward): every row of K^c, V^c and H^c is
+ * recomputed from H.  fill_proxy = 1 also writes P^c = a_hat of every row
+ * (the cache fill that starts a decode); 0 skips the proxy entirely. */
+int spa_full_block(spa_layer *layer, const void *H, const spa_layer_cache *cache, int fill_proxy,
+                   void *stream);
+
+/* ---------------------------------------------------------- decode loop -- */
+typedef struct {
+  int n_layers, vocab, B, N;
+  double rho_p, rho_1, rho_L; /* rho(l) parameters; uniform budget: all equal */
+  int l_p;
+} spa_model_desc;
+
+/* A model: n_layers layer handles (borrowed, all sharing one workspace), a
+ * cache per layer (caches[l], borrowed), the layer-0 input buffer h0
+ * ([B, N, d] device, borrowed), token embeddings embed [vocab, d], final
+ * RMSNorm gain final_norm [d] and LM head lm_head [vocab, d] (device,
+ * borrowed).  The per-layer budgets k_l come from rho(l) at creation. */
+typedef struct spa_model spa_model;
+int spa_model_create(const spa_model_desc *desc, spa_layer *const *layers,
+                     const spa_layer_cache *caches, void *h0, const void *embed,
+                     const void *final_norm, const void *lm_head, spa_model **out);
+void spa_model_free(spa_model *model);
+/* k_l of layer l (0-based), or -1. */
+int spa_model_layer_k(const spa_model *model, int layer);
+/* h0[b, i] <- embed[tokens[b, i]] for every position (tokens: [B, N] int32 device). */
+int spa_model_embed(spa_model *model, const int32_t *tokens, void *stream);
+
+/* One decoding step: full = 0 runs the cached layer step with k_l at every
+ * layer; full = 1 runs every layer at rho = 1 and fills all caches, P^c
+ * included (step 0); full = 2 runs every layer at rho = 1 without the proxy
+ * (vanilla decoding, the uncached baseline).  Then the final RMSNorm and LM head at the u
+ * positions pos ([B, u] int32 device) give argmax ids (lowest id on ties)
+ * into tok_out ([B, u] int32 device).  The ids written back into h0 at pos
+ * for the next step are tok_in ([B, u] device) when non-NULL (teacher
+ * forcing), else the argmax. */
+int spa_decode_step(spa_model *model, const int32_t *pos, const int32_t *tok_in, int u, int full,
+                    int32_t *tok_out, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPA_H */

@@ -1,0 +1,102 @@
+"""GPU parity of the decode loop (through the C ABI) against the oracle on the
+tiny fp32 model: 2 layers, d=256, 4x64 heads, F=688, vocab 1024, N=64 with
+half the positions masked, r=16, uniform rho=0.25 (k=16), 8 steps of 2
+unmaskings, step 0 the rho=1 fill.  Teacher-forced so that one argmax near a
+tie cannot fork the two runs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from adaptive_hidden_state_b200 import synth
+from spa_testutil import LayerPair, assert_close, assert_index_set, np64
+
+pytestmark = pytest.mark.gpu
+
+spa = pytest.importorskip("adaptive_hidden_state_b200.spa")
+
+
+def _tiny_model(dtype, shape, L, vocab, B, N, rho, seed, N_max=None):
+    bf = dtype == spa.SPA_BF16
+    rng = np.random.default_rng(seed)
+    embed = rng.standard_normal((vocab, shape.d)).astype(np.float32)
+    lm = (rng.standard_normal((vocab, shape.d)) * 0.02).astype(np.float32)
+    if bf:
+        embed, lm = synth.bf16_round(embed), synth.bf16_round(lm)
+    fnorm = np.ones(shape.d, np.float32)
+    lps, ws = [], None
+    for l in range(L):
+        lp = LayerPair(spa, shape, seed=seed + 1 + l, dtype=dtype, max_B=B, max_N=N, ws=ws)
+        ws = lp.ws
+        lps.append(lp)
+    tdt = spa.torch_dtype(dtype)
+    dev = lambda a: torch.from_numpy(a).to("cuda", tdt)
+    caches = [lp.cache(B, N) for lp in lps]
+    h0 = torch.zeros((B, N, shape.d), dtype=tdt, device="cuda")
+    e_d, f_d, l_d = dev(embed), dev(fnorm), dev(lm)
+    model = spa.Model([lp.layer for lp in lps], caches, h0, e_d, f_d, l_d, vocab, B, N,
+                      rho_p=rho, l_p=1, rho_1=rho, rho_L=rho)
+    om = O.OracleModel(layers=[lp.ol for lp in lps], embed=embed, final_norm=fnorm, lm_head=lm,
+                       eps=shape.rms_eps)
+    keep = (e_d, f_d, l_d)
+    return model, om, lps, caches, h0, keep
+
+
+def test_tiny_decode_loop_teacher_forced():
+    B, N, vocab, steps, u = 1, 64, 1024, 8, 2
+    model, om, lps, caches, h0, keep = _tiny_model(spa.SPA_F32, synth.TINY_LAYER, 2, vocab, B, N,
+                                                   0.25, seed=0)
+    assert model.k == [16, 16]
+    job = synth.decode_inputs(B=B, N=N, n_prompt=32, vocab=vocab, steps=steps, u=u, seed=5)
+    toks = torch.from_numpy(job.tokens.astype(np.int32)).cuda()
+    model.embed_tokens(toks)
+    state = O.init_decode_state(om, job.tokens)
+    tok_out = torch.empty((B, u), dtype=torch.int32, device="cuda")
+    for t in range(steps):
+        pos = torch.from_numpy(job.positions[t].astype(np.int32)).cuda()
+        forced = torch.from_numpy(job.forced[t].astype(np.int32)).cuda()
+        spa.spa_decode_step(model, pos, forced, u, 1 if t == 0 else 0, tok_out)
+        lps[0].ws.check()
+        ref = O.decode_step(om, state, job.positions[t], model.k, full=(t == 0),
+                            forced=job.forced[t])
+        # argmax ids: equal wherever the oracle's top-2 logit gap is clear
+        got = tok_out.cpu().numpy()
+        lg = ref["logits"]
+        for b in range(B):
+            for j in range(u):
+                top2 = np.sort(lg[b, j])[-2:]
+                if top2[1] - top2[0] > 1e-3 * max(1.0, abs(top2[1])):
+                    assert got[b, j] == ref["argmax"][b, j]
+                else:
+                    assert lg[b, j, got[b, j]] >= top2[1] - 1e-3
+        for l, lp in enumerate(lps):
+            c = caches[l]
+            assert_close(c.h, np.stack([state.caches[l][b].H_c for b in range(B)]), False,
+                         f"step {t} layer {l} H^c")
+            assert_close(c.k, np.stack([state.caches[l][b].K_c for b in range(B)]), False,
+                         f"step {t} layer {l} K^c")
+        assert_close(h0, state.H0, False, f"step {t} h0")
+
+
+def test_tiny_decode_full_k_matches_vanilla():
+    # with k = N at every layer the cached loop is vanilla decoding
+    B, N, vocab, u = 2, 32, 256, 2
+    model, om, lps, caches, h0, keep = _tiny_model(spa.SPA_F32, synth.TINY_LAYER, 2, vocab, B, N,
+                                                   1.0, seed=7)
+    job = synth.decode_inputs(B=B, N=N, n_prompt=8, vocab=vocab, steps=3, u=u, seed=8)
+    toks = torch.from_numpy(job.tokens.astype(np.int32)).cuda()
+    model.embed_tokens(toks)
+    out_cached = []
+    tok_out = torch.empty((B, u), dtype=torch.int32, device="cuda")
+    for t in range(3):
+        pos = torch.from_numpy(job.positions[t].astype(np.int32)).cuda()
+        forced = torch.from_numpy(job.forced[t].astype(np.int32)).cuda()
+        spa.spa_decode_step(model, pos, forced, u, 1 if t == 0 else 0, tok_out)
+        out_cached.append(caches[-1].h.clone())
+    model.embed_tokens(toks)
+    for t in range(3):
+        pos = torch.from_numpy(job.positions[t].astype(np.int32)).cuda()
+        forced = torch.from_numpy(job.forced[t].astype(np.int32)).cuda()
+        spa.spa_decode_step(model, pos, forced, u, 2, tok_out)
+        assert_close(caches[-1].h, np64(out_cached[t]), False, f"vanilla step {t}")
+    lps[0].ws.check()

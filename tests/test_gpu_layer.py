@@ -1,0 +1,197 @@
+"""GPU parity of the cached layer step (through the C ABI) against the CPU
+oracle: the tiny fp32 layer, edge cases of the bf16 path at small widths,
+and one LLaDA-8B-shaped bf16 layer (d=4096, 32x128 heads, F=12288, r=128,
+N=512, rho=0.25)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from adaptive_hidden_state_b200 import synth
+from spa_testutil import LayerPair, assert_close, assert_index_set, np64
+
+pytestmark = pytest.mark.gpu
+
+spa = pytest.importorskip("adaptive_hidden_state_b200.spa")
+
+
+def _run_fill(lp: LayerPair, H: np.ndarray):
+    """rho = 1 fill on both sides; returns (gpu cache, oracle caches per seq)."""
+    B, N, _ = H.shape
+    cache = lp.cache(B, N)
+    spa.spa_full_block(lp.layer, lp.to_dev(H), cache, True)
+    lp.ws.check()
+    ocs = [O.full_block(lp.ol, H[b])[0] for b in range(B)]
+    return cache, ocs
+
+
+def _compare_cache(lp, cache, ocs, what):
+    bf = lp.bf16
+    assert_close(cache.k, np.stack([c.K_c for c in ocs]), bf, what + " K^c")
+    assert_close(cache.v, np.stack([c.V_c for c in ocs]), bf, what + " V^c")
+    assert_close(cache.h, np.stack([c.H_c for c in ocs]), bf, what + " H^c")
+    p = np64(cache.p)
+    assert np.max(np.abs(p - np.stack([c.P_c for c in ocs]))) < (2e-3 if bf else 1e-5), what + " P^c"
+
+
+def _step(lp, cache, ocs, H2, k, check_intermediates=True):
+    """Cached step on both sides, compared phase by phase."""
+    B, N, d = H2.shape
+    H2d = lp.to_dev(H2)
+    idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
+    score = torch.empty((B, N), dtype=torch.float32, device="cuda")
+    spa.spa_proxy_select(lp.layer, H2d, cache, k, idx, score)
+    lp.ws.check()
+    outs = [O.layer_step(lp.ol, H2[b], ocs[b], k) for b in range(B)]
+    s_gpu = np64(score)
+    I_gpu = idx.cpu().numpy()
+    for b in range(B):
+        s_ref = outs[b]["s"]
+        zero = s_ref == 0.0
+        assert np.all(s_gpu[b][zero] == 0.0), "unchanged rows must score exactly 0"
+        assert np.max(np.abs(s_gpu[b] - s_ref)) < (5e-3 if lp.bf16 else 1e-5)
+        assert_index_set(I_gpu[b], s_ref, k, outs[b]["I"], f"I[{b}]")
+        # continue the oracle with the GPU's index set when several were valid
+        if not np.array_equal(I_gpu[b], outs[b]["I"]):
+            raise AssertionError("index sets differ; inputs should carry a margin")
+    spa.spa_partial_block(lp.layer, H2d, idx, k, cache)
+    lp.ws.check()
+    if check_intermediates:
+        dt = spa.torch_dtype(lp.dtype)
+        M = B * k
+        for name, key, width in (("q", "Q", d), ("o", "O", d), ("h1", "H1", d),
+                                 ("a", "A", lp.shape.ffn)):
+            got = lp.ws.view(name, (M, width), dt)
+            ref = np.concatenate([outs[b][key] for b in range(B)])
+            assert_close(got, ref, lp.bf16, "step " + key)
+    _compare_cache(lp, cache, ocs, "step")
+    return I_gpu, outs
+
+
+# ----------------------------------------------------------------- tiny fp32 layer
+
+def test_tiny_fp32_layer_fill_and_cached_step():
+    lp = LayerPair(spa, synth.TINY_LAYER, seed=0, dtype=spa.SPA_F32, max_B=1, max_N=64)
+    H = synth.hidden_states(1, 64, 256, seed=1, bf16=False)
+    cache, ocs = _run_fill(lp, H)
+    _compare_cache(lp, cache, ocs, "fill")
+    for name, key, width in (("q", "Q", 256), ("o", "O", 256), ("h1", "H1", 256), ("a", "A", 688)):
+        got = lp.ws.view(name, (64, width), torch.float32)
+        ref = O.full_block(lp.ol, H[0])[1][key]
+        assert_close(got, ref, False, "fill " + key)
+    H2, rows = synth.drift_rows(H, 0.05, 0.3, seed=2, bf16=False)
+    I, _ = _step(lp, cache, ocs, H2, 16)
+    assert set(rows[0].tolist()) <= set(I[0].tolist())
+
+
+def test_tiny_fp32_graded_drift_exact_selection():
+    lp = LayerPair(spa, synth.TINY_LAYER, seed=3, dtype=spa.SPA_F32, max_B=2, max_N=64)
+    H = synth.hidden_states(2, 64, 256, seed=4, bf16=False)
+    cache, ocs = _run_fill(lp, H)
+    # re-seed until the oracle's k-th/(k+1)-th scores are >= 1e-4 apart
+    for seed in range(100, 200):
+        H2 = synth.graded_drift(H, 0.01, 0.1, seed=seed, bf16=False)
+        ok = True
+        for b in range(2):
+            _, s = O.proxy_identify(H2[b], lp.ol.W_r, ocs[b].P_c)
+            srt = np.sort(s)[::-1]
+            ok &= srt[15] - srt[16] >= 1e-4
+        if ok:
+            break
+    _step(lp, cache, ocs, H2, 16)
+
+
+# ----------------------------------------------------------------- bf16 edge cases
+
+SMALL_BF16 = synth.LayerShape(d=256, n_heads=2, head_dim=128, ffn=384, r=16)
+
+
+@pytest.mark.parametrize("B,N,k", [(1, 1, 1), (1, 7, 3), (2, 130, 1), (1, 130, 130),
+                                   (2, 257, 40), (1, 300, 299)])
+def test_bf16_small_layer_shapes(B, N, k):
+    lp = LayerPair(spa, SMALL_BF16, seed=10 + N, dtype=spa.SPA_BF16, max_B=2, max_N=300, std=0.05)
+    H = synth.hidden_states(B, N, 256, seed=N, bf16=True)
+    cache, ocs = _run_fill(lp, H)
+    _compare_cache(lp, cache, ocs, "fill")
+    H2, _ = synth.drift_rows(H, 0.2, 0.5, seed=N + 1, bf16=True)
+    _step(lp, cache, ocs, H2, k)
+
+
+def test_bf16_zero_drift_selects_lowest_indices():
+    lp = LayerPair(spa, SMALL_BF16, seed=21, dtype=spa.SPA_BF16, max_B=1, max_N=200, std=0.05)
+    H = synth.hidden_states(1, 200, 256, seed=22, bf16=True)
+    cache, ocs = _run_fill(lp, H)
+    h_before = cache.h.clone()
+    I, _ = _step(lp, cache, ocs, H, 37)
+    assert I[0].tolist() == list(range(37))
+    assert_close(cache.h, np64(h_before), True, "zero-drift H^c")
+
+
+def test_bf16_step_is_deterministic():
+    lp = LayerPair(spa, SMALL_BF16, seed=23, dtype=spa.SPA_BF16, max_B=2, max_N=256, std=0.05)
+    H = synth.hidden_states(2, 256, 256, seed=24, bf16=True)
+    H2, _ = synth.drift_rows(H, 0.1, 0.4, seed=25, bf16=True)
+    outs = []
+    for _ in range(2):
+        cache = lp.cache(2, 256)
+        spa.spa_full_block(lp.layer, lp.to_dev(H), cache, True)
+        idx = torch.empty((2, 64), dtype=torch.int32, device="cuda")
+        spa.spa_layer_step(lp.layer, lp.to_dev(H2), cache, 64, idx)
+        lp.ws.check()
+        outs.append((idx.clone(), cache.k.clone(), cache.v.clone(), cache.h.clone(), cache.p.clone()))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+def test_device_index_check_reports_without_fault():
+    lp = LayerPair(spa, SMALL_BF16, seed=26, dtype=spa.SPA_BF16, max_B=1, max_N=64, std=0.05)
+    H = lp.to_dev(synth.hidden_states(1, 64, 256, seed=27, bf16=True))
+    cache = lp.cache(1, 64)
+    idx = torch.tensor([[0, 5, 64, 70]], dtype=torch.int32, device="cuda")  # 64, 70 out of range
+    spa.spa_partial_block(lp.layer, H, idx, 4, cache)
+    assert lp.ws.status() == -7
+    assert lp.ws.status() == 0       # cleared
+
+
+# ----------------------------------------------------------------- LLaDA-shaped bf16 layer
+
+@pytest.fixture(scope="module")
+def llada():
+    lp = LayerPair(spa, synth.LLADA_LAYER, seed=0, dtype=spa.SPA_BF16, max_B=1, max_N=512)
+    H = synth.hidden_states(1, 512, 4096, seed=1, bf16=True)
+    return lp, H
+
+
+def test_llada_proxy_weights_match_oracle_svd(llada):
+    lp, _ = llada
+    got = lp.layer.proxy_weights().numpy().astype(np.float64)
+    ref = lp.W_r
+    sgn = np.sign(np.sum(got * ref, axis=1))[:, None]
+    assert np.all(sgn == 1)
+    diff = np.abs(got - ref)
+    ulp = np.abs(ref) * 2.0 ** -7 + 1e-30
+    assert np.mean(diff > 0) < 1e-3          # bf16 storage: identical but for rare ties
+    assert np.all(diff <= ulp)
+
+
+def test_llada_fill_then_cached_step(llada):
+    lp, H = llada
+    cache, ocs = _run_fill(lp, H)
+    _compare_cache(lp, cache, ocs, "fill")
+    H2, rows = synth.drift_rows(H, 0.05, 0.3, seed=2, bf16=True)   # 26 drifted rows
+    I, _ = _step(lp, cache, ocs, H2, 128)
+    assert set(rows[0].tolist()) <= set(I[0].tolist())
+
+
+def test_llada_graded_drift_exact_selection(llada):
+    lp, H = llada
+    cache, ocs = _run_fill(lp, H)
+    for seed in range(300, 400):
+        H2 = synth.graded_drift(H, 0.01, 0.1, seed=seed, bf16=True)
+        _, s = O.proxy_identify(H2[0], lp.ol.W_r, ocs[0].P_c)
+        srt = np.sort(s)[::-1]
+        if srt[127] - srt[128] >= 1e-4:
+            break
+    else:
+        pytest.fail("no seed with a 1e-4 margin")
+    _step(lp, cache, ocs, H2, 128)
