@@ -44,6 +44,71 @@ static int fail(int status, const char* fmt, ...) {
     if (s_ != SPA_OK) return s_; \
   } while (0)
 
+// ---------------------------------------------------------------------------
+// kernel timing (events per launch, off by default) and the launch counter
+// ---------------------------------------------------------------------------
+static long long g_launches = 0;
+
+struct ProfRec {
+  int cls;
+  cudaEvent_t a, b;
+  double bytes, flops;
+};
+
+struct Profiler {
+  bool on = false;
+  std::vector<cudaEvent_t> free_events;
+  std::vector<ProfRec> recs;
+  cudaEvent_t get() {
+    if (!free_events.empty()) {
+      cudaEvent_t e = free_events.back();
+      free_events.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    return e;
+  }
+  void release_all() {
+    for (auto& r : recs) {
+      free_events.push_back(r.a);
+      free_events.push_back(r.b);
+    }
+    recs.clear();
+  }
+  ~Profiler() {
+    release_all();
+    for (cudaEvent_t e : free_events) cudaEventDestroy(e);
+  }
+};
+
+// Brackets one kernel launch with events when profiling is on; counts it.
+struct ProfScope {
+  Profiler* p;
+  int cls;
+  double bytes, flops;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr, b = nullptr;
+  ProfScope(Profiler* prof, int c, double by, double fl, cudaStream_t st)
+      : p(prof), cls(c), bytes(by), flops(fl), s(st) {
+    ++g_launches;
+    if (p && p->on) {
+      a = p->get();
+      b = p->get();
+      if (a && b) cudaEventRecord(a, s);
+    }
+  }
+  ~ProfScope() {
+    if (a && b) {
+      cudaEventRecord(b, s);
+      p->recs.push_back({cls, a, b, bytes, flops});
+    }
+  }
+};
+
 extern "C" const char* spa_status_string(int status) {
   switch (status) {
     case SPA_OK: return "SPA_OK";
@@ -123,6 +188,7 @@ struct spa_workspace {
   CUtensorMap tmX, tmO, tmX2, tmA;
   int num_sms = 148;
   std::vector<void*> allocs;
+  Profiler prof;
 };
 
 struct spa_layer {
@@ -280,6 +346,38 @@ extern "C" int spa_workspace_intermediates(const spa_workspace* ws, spa_intermed
   return SPA_OK;
 }
 
+extern "C" int spa_profile_enable(spa_workspace* ws, int enable) {
+  if (!ws) return fail(SPA_ERR_INVALID, "null workspace");
+  ws->prof.on = enable != 0;
+  return SPA_OK;
+}
+
+extern "C" int spa_profile_read(spa_workspace* ws, int* launches, double* ms, double* bytes,
+                                double* flops) {
+  if (!ws || !launches || !ms || !bytes || !flops) return fail(SPA_ERR_INVALID, "null argument");
+  for (int c = 0; c < SPA_PROF_CLASSES; ++c) {
+    launches[c] = 0;
+    ms[c] = bytes[c] = flops[c] = 0.0;
+  }
+  int st = SPA_OK;
+  for (auto& r : ws->prof.recs) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) {
+      cudaGetLastError();
+      st = fail(SPA_ERR_CUDA, "reading kernel timing events failed");
+      continue;
+    }
+    launches[r.cls] += 1;
+    ms[r.cls] += t;
+    bytes[r.cls] += r.bytes;
+    flops[r.cls] += r.flops;
+  }
+  ws->prof.release_all();
+  return st;
+}
+
+extern "C" long long spa_launch_count(void) { return g_launches; }
+
 extern "C" void spa_free_layer(spa_layer* layer) {
   if (!layer) return;
   if (layer->w_r) cudaFree(layer->w_r);
@@ -395,18 +493,28 @@ static int choose_splits(int tiles, int KB, int sms) {
   return best;
 }
 
-static int run_tc(int mode, int BN, TcGemmParams& p, int M, int n_tiles, int splits, cudaStream_t s) {
+// Algorithmic work of one launch, for the kernel timing record.
+struct Work {
+  int cls;
+  double bytes, flops;
+};
+
+static int run_tc(int mode, int BN, TcGemmParams& p, int M, int n_tiles, int splits, cudaStream_t s,
+                  Profiler* prof, Work w) {
   const int m_tiles = (M + 127) / 128;
   if (m_tiles == 0) return SPA_OK;
+  ProfScope ps(prof, w.cls, w.bytes, w.flops, s);
   if (m_tiles > 65535 || n_tiles > 65535) return fail(SPA_ERR_SHAPE, "GEMM grid too large");
   cudaError_t e = launch_tc_gemm(mode, BN, p, m_tiles, n_tiles, splits, s);
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "tc GEMM launch (mode %d): %s", mode, cudaGetErrorString(e));
   return SPA_OK;
 }
 
-static int run_simt(int mode, SimtGemmParams& p, int M, int n_tiles, cudaStream_t s) {
+static int run_simt(int mode, SimtGemmParams& p, int M, int n_tiles, cudaStream_t s, Profiler* prof,
+                    Work w) {
   const int m_tiles = (M + 63) / 64;
   if (m_tiles == 0) return SPA_OK;
+  ProfScope ps(prof, w.cls, w.bytes, w.flops, s);
   cudaError_t e = launch_simt_gemm(mode, p, m_tiles, n_tiles, s);
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "SIMT GEMM launch (mode %d): %s", mode, cudaGetErrorString(e));
   return SPA_OK;
@@ -432,6 +540,11 @@ static int run_proxy(spa_layer* L, const void* H, const spa_layer_cache* c, floa
   ep.p_cache = c->p_cache;
   ep.score = score;
   ep.proxy_fill = fill;
+  const double e = L->desc.dtype == SPA_BF16 ? 2.0 : 4.0;
+  // H read, W_r read, P^c read + a_hat write (or P^c write), scores
+  const Work w{SPA_PROF_PROXY,
+               (double)M * d * e + (double)r * d * e + (fill ? 1.0 : 2.0) * M * r * 4 + (fill ? 0 : 4.0 * M),
+               2.0 * M * d * r};
   if (L->desc.dtype == SPA_BF16) {
     TcGemmParams p;
     std::memset(&p, 0, sizeof(p));
@@ -444,7 +557,7 @@ static int run_proxy(spa_layer* L, const void* H, const spa_layer_cache* c, floa
     p.ep = ep;
     // split count depends on d only, so a row's proxy bits never depend on B or N
     const int splits = std::max(1, std::min(8, (d / 64) / 4));
-    return run_tc(EPI_PROXY, r <= 128 ? 128 : 256, p, M, 1, splits, s);
+    return run_tc(EPI_PROXY, r <= 128 ? 128 : 256, p, M, 1, splits, s, &L->ws->prof, w);
   }
   SimtGemmParams p;
   std::memset(&p, 0, sizeof(p));
@@ -454,7 +567,7 @@ static int run_proxy(spa_layer* L, const void* H, const spa_layer_cache* c, floa
   p.b_mode = B_SINGLE;
   p.b_rows_per_src = r;
   p.ep = ep;
-  return run_simt(EPI_PROXY, p, M, 1, s);
+  return run_simt(EPI_PROXY, p, M, 1, s, &L->ws->prof, w);
 }
 
 // Phases 2 and 3 for M = B * tps tokens; idx == null means every row (rho = 1).
@@ -464,9 +577,14 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
   const spa_layer_desc& D = L->desc;
   const int d = D.d, F = D.ffn, M = c->B * tps, N = c->N;
   const bool bf = D.dtype == SPA_BF16;
+  const double es = bf ? 2.0 : 4.0, Md = (double)M * d, Bn = (double)c->B * N;
+  Profiler* prof = &ws->prof;
   cudaError_t e;
   // x = RMSNorm(H[I])
-  e = launch_rmsnorm_rows(D.dtype, H, 1, idx, tps, N, M, d, L->w.attn_norm, D.rms_eps, ws->X, ws->err, s);
+  {
+    ProfScope ps(prof, SPA_PROF_NORM, 2.0 * Md * es + d * es, 4.0 * Md, s);
+    e = launch_rmsnorm_rows(D.dtype, H, 1, idx, tps, N, M, d, L->w.attn_norm, D.rms_eps, ws->X, ws->err, s);
+  }
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "rmsnorm launch: %s", cudaGetErrorString(e));
   // Q, K, V with RoPE; K, V scattered into the caches
   {
@@ -482,19 +600,24 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
       p.tmB[0] = L->tm_wq; p.tmB[1] = L->tm_wk; p.tmB[2] = L->tm_wv;
       p.K = d; p.b_mode = B_CONCAT3; p.b_rows_per_src = d; p.ep = ep;
       const int nt = 3 * d / 256, mt = (M + 127) / 128;
-      SPA_TRY(run_tc(EPI_QKV, 256, p, M, nt, choose_splits(nt * mt, d / 64, ws->num_sms), s));
+      SPA_TRY(run_tc(EPI_QKV, 256, p, M, nt, choose_splits(nt * mt, d / 64, ws->num_sms), s, prof,
+                     Work{SPA_PROF_QKV, 3.0 * d * d * es + Md * es + 3.0 * Md * es, 6.0 * Md * d}));
     } else {
       SimtGemmParams p;
       std::memset(&p, 0, sizeof(p));
       p.A = (const float*)ws->X;
       p.B[0] = (const float*)L->w.wq; p.B[1] = (const float*)L->w.wk; p.B[2] = (const float*)L->w.wv;
       p.K = d; p.b_mode = B_CONCAT3; p.b_rows_per_src = d; p.ep = ep;
-      SPA_TRY(run_simt(EPI_QKV, p, M, (3 * d + 127) / 128, s));
+      SPA_TRY(run_simt(EPI_QKV, p, M, (3 * d + 127) / 128, s, prof,
+                       Work{SPA_PROF_QKV, 3.0 * d * d * es + Md * es + 3.0 * Md * es, 6.0 * Md * d}));
     }
   }
   // O = attention over the whole cache
-  e = launch_attention(D.dtype, ws->Q, c->k_cache, c->v_cache, ws->O, c->B, tps, N, D.n_heads,
-                       D.head_dim, ws->part_o, ws->part_ml, ws->part_rows, ws->err, s);
+  {
+    ProfScope ps(prof, SPA_PROF_ATTN, 2.0 * Md * es + 2.0 * Bn * d * es, 4.0 * Md * N, s);
+    e = launch_attention(D.dtype, ws->Q, c->k_cache, c->v_cache, ws->O, c->B, tps, N, D.n_heads,
+                         D.head_dim, ws->part_o, ws->part_ml, ws->part_rows, ws->err, s);
+  }
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
   // H1 = H[I] + O W_o^T
   {
@@ -508,17 +631,22 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
       p.tmA = ws->tmO; p.tmB[0] = L->tm_wo;
       p.K = d; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
       const int nt = d / 256, mt = (M + 127) / 128;
-      SPA_TRY(run_tc(EPI_RESID, 256, p, M, nt, choose_splits(nt * mt, d / 64, ws->num_sms), s));
+      SPA_TRY(run_tc(EPI_RESID, 256, p, M, nt, choose_splits(nt * mt, d / 64, ws->num_sms), s, prof,
+                     Work{SPA_PROF_OPROJ, (double)d * d * es + 3.0 * Md * es, 2.0 * Md * d}));
     } else {
       SimtGemmParams p;
       std::memset(&p, 0, sizeof(p));
       p.A = (const float*)ws->O; p.B[0] = (const float*)L->w.wo;
       p.K = d; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
-      SPA_TRY(run_simt(EPI_RESID, p, M, (d + 127) / 128, s));
+      SPA_TRY(run_simt(EPI_RESID, p, M, (d + 127) / 128, s, prof,
+                       Work{SPA_PROF_OPROJ, (double)d * d * es + 3.0 * Md * es, 2.0 * Md * d}));
     }
   }
   // x2 = RMSNorm(H1)
-  e = launch_rmsnorm_rows(D.dtype, ws->H1, 0, nullptr, tps, N, M, d, L->w.ffn_norm, D.rms_eps, ws->X2, ws->err, s);
+  {
+    ProfScope ps(prof, SPA_PROF_NORM, 2.0 * Md * es + d * es, 4.0 * Md, s);
+    e = launch_rmsnorm_rows(D.dtype, ws->H1, 0, nullptr, tps, N, M, d, L->w.ffn_norm, D.rms_eps, ws->X2, ws->err, s);
+  }
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "rmsnorm launch: %s", cudaGetErrorString(e));
   // A = silu(x2 W_gate^T) * (x2 W_up^T)
   {
@@ -531,13 +659,15 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
       p.tmA = ws->tmX2; p.tmB[0] = L->tm_wg; p.tmB[1] = L->tm_wu;
       p.K = d; p.b_mode = B_GATEUP; p.b_rows_per_src = F; p.ep = ep;
       const int nt = F / 128, mt = (M + 127) / 128;
-      SPA_TRY(run_tc(EPI_SWIGLU, 256, p, M, nt, choose_splits(nt * mt, d / 64, ws->num_sms), s));
+      SPA_TRY(run_tc(EPI_SWIGLU, 256, p, M, nt, choose_splits(nt * mt, d / 64, ws->num_sms), s, prof,
+                     Work{SPA_PROF_GATEUP, 2.0 * F * d * es + Md * es + (double)M * F * es, 4.0 * Md * F}));
     } else {
       SimtGemmParams p;
       std::memset(&p, 0, sizeof(p));
       p.A = (const float*)ws->X2; p.B[0] = (const float*)L->w.w_gate; p.B[1] = (const float*)L->w.w_up;
       p.K = d; p.b_mode = B_GATEUP; p.b_rows_per_src = F; p.ep = ep;
-      SPA_TRY(run_simt(EPI_SWIGLU, p, M, (F + 63) / 64, s));
+      SPA_TRY(run_simt(EPI_SWIGLU, p, M, (F + 63) / 64, s, prof,
+                       Work{SPA_PROF_GATEUP, 2.0 * F * d * es + Md * es + (double)M * F * es, 4.0 * Md * F}));
     }
   }
   // H^c[I] = H1 + A W_down^T
@@ -552,13 +682,15 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
       p.tmA = ws->tmA; p.tmB[0] = L->tm_wd;
       p.K = F; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
       const int nt = d / 256, mt = (M + 127) / 128;
-      SPA_TRY(run_tc(EPI_RESID_SCATTER, 256, p, M, nt, choose_splits(nt * mt, F / 64, ws->num_sms), s));
+      SPA_TRY(run_tc(EPI_RESID_SCATTER, 256, p, M, nt, choose_splits(nt * mt, F / 64, ws->num_sms), s, prof,
+                     Work{SPA_PROF_DOWN, (double)d * F * es + (double)M * F * es + 2.0 * Md * es, 2.0 * Md * F}));
     } else {
       SimtGemmParams p;
       std::memset(&p, 0, sizeof(p));
       p.A = (const float*)ws->A; p.B[0] = (const float*)L->w.w_down;
       p.K = F; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
-      SPA_TRY(run_simt(EPI_RESID_SCATTER, p, M, (d + 127) / 128, s));
+      SPA_TRY(run_simt(EPI_RESID_SCATTER, p, M, (d + 127) / 128, s, prof,
+                       Work{SPA_PROF_DOWN, (double)d * F * es + (double)M * F * es + 2.0 * Md * es, 2.0 * Md * F}));
     }
   }
   return SPA_OK;
@@ -580,7 +712,12 @@ extern "C" int spa_proxy_select(spa_layer* L, const void* H, const spa_layer_cac
   cudaStream_t s = (cudaStream_t)stream;
   float* sc = score ? score : L->ws->score;
   SPA_TRY(run_proxy(L, H, c, sc, 0, s));
-  cudaError_t e = launch_topk_select(sc, c->B, c->N, k, idx, L->ws->a_hat, c->p_cache, L->desc.r, L->ws->err, s);
+  cudaError_t e;
+  {
+    const double Bn = (double)c->B * c->N, Bk = (double)c->B * k;
+    ProfScope ps(&L->ws->prof, SPA_PROF_TOPK, 4.0 * Bn + 8.0 * Bk * L->desc.r + 4.0 * Bk, 0.0, s);
+    e = launch_topk_select(sc, c->B, c->N, k, idx, L->ws->a_hat, c->p_cache, L->desc.r, L->ws->err, s);
+  }
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "top-k launch: %s", cudaGetErrorString(e));
   return SPA_OK;
 }
@@ -683,6 +820,7 @@ extern "C" int spa_model_layer_k(const spa_model* m, int layer) {
 extern "C" int spa_model_embed(spa_model* m, const int32_t* tokens, void* stream) {
   if (!m || !tokens) return fail(SPA_ERR_INVALID, "null argument");
   spa_workspace* ws = m->layers[0]->ws;
+  ProfScope ps(&ws->prof, SPA_PROF_MISC, 0.0, 0.0, (cudaStream_t)stream);
   cudaError_t e = launch_embed_rows(ws->desc.dtype, m->embed, tokens, nullptr, m->desc.B, m->desc.N,
                                     m->desc.N, ws->desc.d, m->desc.vocab, m->h0, ws->err,
                                     (cudaStream_t)stream);
@@ -709,10 +847,17 @@ extern "C" int spa_decode_step(spa_model* m, const int32_t* pos, const int32_t* 
     }
   }
   // final RMSNorm at the u positions, LM head, argmax
-  cudaError_t e = launch_gather_final(D.dtype, m->caches[L - 1].h_cache, pos, B, u, N, d,
-                                      m->final_norm, D.rms_eps, ws->X, ws->err, s);
+  const double es = D.dtype == SPA_BF16 ? 2.0 : 4.0;
+  cudaError_t e;
+  {
+    ProfScope ps(&ws->prof, SPA_PROF_MISC, 2.0 * B * u * d * es, 0.0, s);
+    e = launch_gather_final(D.dtype, m->caches[L - 1].h_cache, pos, B, u, N, d, m->final_norm,
+                            D.rms_eps, ws->X, ws->err, s);
+  }
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "final norm launch: %s", cudaGetErrorString(e));
   const int M = B * u;
+  const Work wl{SPA_PROF_LMHEAD, (double)m->desc.vocab * d * es + (double)M * d * es,
+                2.0 * M * d * m->desc.vocab};
   EpiParams ep;
   std::memset(&ep, 0, sizeof(ep));
   ep.M = M;
@@ -730,19 +875,25 @@ extern "C" int spa_decode_step(spa_model* m, const int32_t* pos, const int32_t* 
     p.tmA = ws->tmX;
     p.tmB[0] = m->tm_lm;
     p.K = d; p.b_mode = B_SINGLE; p.b_rows_per_src = m->desc.vocab; p.ep = ep;
-    SPA_TRY(run_tc(EPI_ARGMAX, 256, p, M, m->lm_tiles, 1, s));
+    SPA_TRY(run_tc(EPI_ARGMAX, 256, p, M, m->lm_tiles, 1, s, &ws->prof, wl));
   } else {
     SimtGemmParams p;
     std::memset(&p, 0, sizeof(p));
     p.A = (const float*)ws->X; p.B[0] = (const float*)m->lm_head;
     p.K = d; p.b_mode = B_SINGLE; p.b_rows_per_src = m->desc.vocab; p.ep = ep;
-    SPA_TRY(run_simt(EPI_ARGMAX, p, M, m->lm_tiles, s));
+    SPA_TRY(run_simt(EPI_ARGMAX, p, M, m->lm_tiles, s, &ws->prof, wl));
   }
-  e = launch_argmax_reduce(m->amax_val, m->amax_idx, M, m->lm_tiles, tok_out, s);
+  {
+    ProfScope ps(&ws->prof, SPA_PROF_MISC, 8.0 * M * m->lm_tiles, 0.0, s);
+    e = launch_argmax_reduce(m->amax_val, m->amax_idx, M, m->lm_tiles, tok_out, s);
+  }
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "argmax launch: %s", cudaGetErrorString(e));
   // next step's layer-0 input: embeddings of the written ids at pos
-  e = launch_embed_rows(D.dtype, m->embed, tok_in ? tok_in : tok_out, pos, B, u, N, d, m->desc.vocab,
-                        m->h0, ws->err, s);
+  {
+    ProfScope ps(&ws->prof, SPA_PROF_MISC, 2.0 * M * d * es, 0.0, s);
+    e = launch_embed_rows(D.dtype, m->embed, tok_in ? tok_in : tok_out, pos, B, u, N, d,
+                          m->desc.vocab, m->h0, ws->err, s);
+  }
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "embed launch: %s", cudaGetErrorString(e));
   return SPA_OK;
 }

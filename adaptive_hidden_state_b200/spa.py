@@ -30,11 +30,19 @@ STATUS = {0: "SPA_OK", -1: "SPA_ERR_INVALID", -2: "SPA_ERR_SHAPE", -3: "SPA_ERR_
 EXPORTS = [
     "spa_status_string", "spa_last_error", "spa_version", "spa_rho", "spa_budget_k",
     "spa_singular_proxy_host", "spa_workspace_create", "spa_workspace_free",
-    "spa_workspace_status", "spa_workspace_intermediates", "spa_init_layer", "spa_free_layer", "spa_layer_proxy_weights",
+    "spa_workspace_status", "spa_workspace_intermediates", "spa_profile_enable",
+    "spa_profile_read", "spa_launch_count", "spa_init_layer", "spa_free_layer", "spa_layer_proxy_weights",
     "spa_proxy_select", "spa_partial_block", "spa_layer_step", "spa_full_block",
     "spa_model_create", "spa_model_free", "spa_model_layer_k", "spa_model_embed",
     "spa_decode_step",
 ]
+
+
+PROF_CLASSES = ["proxy", "topk", "norm", "qkv", "attn", "oproj", "gateup", "down", "lmhead", "misc"]
+
+
+def spa_launch_count() -> int:
+    return lib.spa_launch_count()
 
 
 class SpaError(RuntimeError):
@@ -85,6 +93,10 @@ _sig("spa_workspace_create", c_int, POINTER(LayerDesc), c_int, c_int, POINTER(c_
 _sig("spa_workspace_free", None, c_void_p)
 _sig("spa_workspace_status", c_int, c_void_p, c_void_p)
 _sig("spa_workspace_intermediates", c_int, c_void_p, POINTER(Intermediates))
+_sig("spa_profile_enable", c_int, c_void_p, c_int)
+_sig("spa_profile_read", c_int, c_void_p, POINTER(c_int), POINTER(c_double), POINTER(c_double),
+     POINTER(c_double))
+_sig("spa_launch_count", ctypes.c_longlong)
 _sig("spa_init_layer", c_int, POINTER(LayerDesc), POINTER(LayerWeights), c_void_p, c_void_p,
      POINTER(c_void_p))
 _sig("spa_free_layer", None, c_void_p)
@@ -170,6 +182,16 @@ class Workspace:
 
     def check(self, stream=None):
         _check(self.status(stream), "spa_workspace_status")
+
+    def profile_enable(self, on: bool = True):
+        _check(lib.spa_profile_enable(self.handle, int(on)), "spa_profile_enable")
+
+    def profile_read(self) -> dict:
+        """{class name: (launches, ms, algorithmic bytes, flops)} since the last read."""
+        n = len(PROF_CLASSES)
+        la, ms, by, fl = (c_int * n)(), (c_double * n)(), (c_double * n)(), (c_double * n)()
+        _check(lib.spa_profile_read(self.handle, la, ms, by, fl), "spa_profile_read")
+        return {PROF_CLASSES[i]: (la[i], ms[i], by[i], fl[i]) for i in range(n)}
 
     def intermediates(self) -> dict:
         """Device addresses of the compact intermediates of the last layer call."""

@@ -1,0 +1,449 @@
+#!/usr/bin/env python
+"""SPA-Cache decode-step benchmark on B200.
+
+Workload (default): a LLaDA-8B-shaped 32-layer bidirectional DLM with random
+bf16 weights (d=4096, 32 heads x 128, SwiGLU 12288, vocab 126464, W_v with
+power-law singular values i^-0.8), one sequence of N=1024 tokens (256 random
+prompt ids + 768 masks), proxy rank r=128 and the piecewise-Gaussian budget
+rho(l) with rho_p=0.25 at l_p=12 and rho_1=rho_L=0.06.  Step 0 (the rho=1
+cache fill) is setup; every timed step is one cached decode step: 32 cached
+layer steps, the LM head at the 2 positions unmasked that step, argmax, and
+the embedding update.  `value` = tokens unmasked per second.
+
+Also reported: us/layer, the dominant kernel's roofline fraction (CUDA events
+per kernel over the timed region), the end-to-end figure with host buffers
+(positions host->device and token ids device->host inside the timed region),
+the rho=1 vanilla decode step on the same GPU, clocks during the timed
+region, the CPU oracle on a bounded sample, and the kernel launch count.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl spa|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SPA-Cache decode-step tokens/s and µs/layer at 1 B200; % of HBM/tensor roofline"
+CFG = dict(L=32, d=4096, n_heads=32, head_dim=128, ffn=12288, vocab=126464, B=1, N=1024,
+           n_prompt=256, r=128, rho_p=0.25, l_p=12, rho_1=0.06, rho_L=0.06, u=2)
+WORKLOAD = ("LLaDA-8B-shaped 32-layer bf16 DLM decode step: B=1, N=1024 (256 prompt + 768 masked), "
+            "r=128, piecewise-Gaussian rho(l) (rho_p=0.25, l_p=12, rho_1=rho_L=0.06), "
+            "2 tokens unmasked per step")
+PROF_CLASSES = ["proxy", "topk", "norm", "qkv", "attn", "oproj", "gateup", "down", "lmhead", "misc"]
+LAYER_CLASSES = ["proxy", "topk", "norm", "qkv", "attn", "oproj", "gateup", "down"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["spa", "reference"], default="spa")
+    ap.add_argument("--vanilla-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained", p["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f".clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as fh:
+            for line in fh:
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm.append(float(f[1]))
+                    smax = float(f[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, f[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ model setup
+
+def build_model(spa, torch, seed: int):
+    c = CFG
+    d, F, r, V = c["d"], c["ffn"], c["r"], c["vocab"]
+    dev = "cuda"
+    g = torch.Generator(device=dev).manual_seed(seed)
+
+    def randn(shape, std):
+        return (torch.randn(shape, generator=g, device=dev, dtype=torch.float32) * std).to(torch.bfloat16)
+
+    def haar(n):
+        q, rr = torch.linalg.qr(torch.randn((n, n), generator=g, device=dev, dtype=torch.float32))
+        return q * torch.sign(torch.diagonal(rr))[None, :]
+
+    sigma = torch.arange(1, d + 1, device=dev, dtype=torch.float32) ** -0.8
+    desc = spa.LayerDesc(d=d, n_heads=c["n_heads"], head_dim=c["head_dim"], ffn=F, r=r,
+                         dtype=spa.SPA_BF16, rms_eps=1e-5, rope_theta=1e4)
+    ws = spa.Workspace(desc, c["B"], c["N"])
+    layers, caches, weights = [], [], []
+    ones = torch.ones(d, device=dev, dtype=torch.bfloat16)
+    for l in range(c["L"]):
+        U, Vm = haar(d), haar(d)
+        wv = ((U * sigma[None, :]) @ Vm.T).to(torch.bfloat16)
+        # the offline proxy: W_r = Lambda_r V_r^T, exact for this construction
+        w_r = (sigma[:r, None] * Vm[:, :r].T).float().cpu()
+        del U
+        w = {"wq": randn((d, d), .02), "wk": randn((d, d), .02), "wv": wv, "wo": randn((d, d), .02),
+             "w_gate": randn((F, d), .02), "w_up": randn((F, d), .02), "w_down": randn((d, F), .02),
+             "attn_norm": ones, "ffn_norm": ones}
+        layers.append(spa.Layer(desc, w, ws, w_r_host=w_r))
+        weights.append(w)
+        caches.append(spa.Cache(c["B"], c["N"], d, r, spa.SPA_BF16))
+    embed = randn((V, d), 1.0)
+    lm_head = randn((V, d), .02)
+    h0 = torch.zeros((c["B"], c["N"], d), device=dev, dtype=torch.bfloat16)
+    model = spa.Model(layers, caches, h0, embed, ones, lm_head, V, c["B"], c["N"], c["rho_p"],
+                      c["l_p"], c["rho_1"], c["rho_L"])
+    return model, ws, layers, caches, weights, (embed, lm_head, h0, ones)
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+
+class OracleSample:
+    """The oracle's cached layer step (fp64 numpy, as it stands) at the
+    workload's layer shape and N=1024: the rho=1 fill is setup, each call of
+    step() times one cached layer step with budget k."""
+
+    def __init__(self, weights_l: dict, seed: int):
+        import oracle as O
+        from adaptive_hidden_state_b200 import synth
+        c = CFG
+        self.O = O
+        w = {k_: v.float().cpu().numpy() for k_, v in weights_l.items()}
+        # Which proxy the step uses does not change its cost; the oracle's own
+        # SVD of a 4096^2 matrix is offline setup, so a seeded proxy stands in.
+        W_r = np.random.default_rng(seed).standard_normal((c["r"], c["d"])) * 0.02
+        self.layer = O.OracleLayer.from_weights(w, W_r, c["n_heads"])
+        H = synth.hidden_states(1, c["N"], c["d"], seed=seed, bf16=True)[0]
+        self.cache, _ = O.full_block(self.layer, H)
+        H2, _ = synth.drift_rows(H[None], 0.05, 0.3, seed=seed + 1, bf16=True)
+        self.H2 = H2[0]
+
+    def step(self, k: int) -> float:
+        cc = self.cache.copy()
+        t0 = time.perf_counter()
+        self.O.layer_step(self.layer, self.H2, cc, k)
+        return time.perf_counter() - t0
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
+
+
+# ------------------------------------------------------------------ traffic record
+
+def traffic_record(cls: str):
+    """Per-launch DRAM bytes of `cls` from the committed ncu summary, or None
+    when the kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic_llada_decode.md")
+    if not os.path.exists(path):
+        return None
+    src = os.path.join(ROOT, "adaptive_hidden_state_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(src)):
+        if name.endswith((".cu", ".cuh", ".h", ".cpp")):
+            with open(os.path.join(src, name), "rb") as fh:
+                h.update(fh.read())
+    sha = h.hexdigest()[:16]
+    with open(path) as fh:
+        for line in fh:
+            m = re.match(r"^traffic\s+(\w+)\s+bytes_per_launch=(\d+)\s+source_sha=(\w+)", line.strip())
+            if m and m.group(1) == cls:
+                return int(m.group(2)) if m.group(3) == sha else None
+    return None
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args, rank: int):
+    if rank != 0:
+        return
+    import torch
+    from oracle import budget_table
+    c = CFG
+    ks = budget_table(c["N"], c["L"], c["rho_p"], c["l_p"], c["rho_1"], c["rho_L"])
+    kbar = int(round(sum(ks) / len(ks)))
+    g = torch.Generator().manual_seed(args.seed)
+    d, F = c["d"], c["ffn"]
+    rn = lambda shape, std: (torch.randn(shape, generator=g) * std).to(torch.bfloat16)
+    w = {"wq": rn((d, d), .02), "wk": rn((d, d), .02), "wv": rn((d, d), .02), "wo": rn((d, d), .02),
+         "w_gate": rn((F, d), .02), "w_up": rn((F, d), .02), "w_down": rn((d, F), .02),
+         "attn_norm": torch.ones(d), "ffn_norm": torch.ones(d)}
+    sample_run = OracleSample(w, args.seed)
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        t = sample_run.step(kbar)
+        if i >= args.warmup:
+            per_step.append(t * c["L"])
+    step_s = float(np.mean(per_step))
+    value = c["B"] * c["u"] / step_s
+    sample = (f"each step: one oracle cached layer step (fp64 numpy) at N=1024, k={kbar} (mean of "
+              f"the 32-layer budget table), x32 layers; LM head excluded")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main arm
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from adaptive_hidden_state_b200 import spa, synth
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    c = CFG
+    B, N, u = c["B"], c["N"], c["u"]
+    total_steps = 1 + args.warmup + args.steps
+    assert total_steps <= (N - c["n_prompt"]) // u, "more steps than masked positions"
+    model, ws, layers, caches, weights, keep = build_model(spa, torch, args.seed + 1000 * rank)
+    job = synth.decode_inputs(B=B, N=N, n_prompt=c["n_prompt"], vocab=c["vocab"],
+                              steps=total_steps, u=u, seed=args.seed + rank)
+    toks = torch.from_numpy(job.tokens.astype(np.int32)).cuda()
+    pos_dev = [torch.from_numpy(p.astype(np.int32)).cuda() for p in job.positions]
+    tok_out = torch.empty((total_steps, B, u), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # step 0: rho = 1 fill (setup)
+    model.embed_tokens(toks)
+    spa.spa_decode_step(model, pos_dev[0], None, u, 1, tok_out[0])
+    for t in range(1, 1 + args.warmup):
+        spa.spa_decode_step(model, pos_dev[t], None, u, 0, tok_out[t])
+    ws.check()
+
+    # ---- timed region: K cached decode steps, inputs resident in HBM
+    gpu_id = str(local)
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(gpu_id)
+    ws.profile_enable(True)
+    ws.profile_read()
+    n0 = spa.spa_launch_count()
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for t in range(1 + args.warmup, total_steps):
+        spa.spa_decode_step(model, pos_dev[t], None, u, 0, tok_out[t])
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    launches = spa.spa_launch_count() - n0
+    prof = ws.profile_read()
+    ws.profile_enable(False)
+    ws.check()
+    t_ms = max_over_ranks(ev0.elapsed_time(ev1))
+    K = args.steps
+    tokens = world * B * u * K
+    value = tokens / (t_ms / 1e3)
+    ms_step = t_ms / K
+
+    layer_ms = sum(prof[k][1] for k in LAYER_CLASSES) / K
+    us_per_layer = layer_ms * 1e3 / c["L"]
+    dom = max(LAYER_CLASSES + ["lmhead"], key=lambda k: prof[k][1])
+    n_l, ms_l, by_l, fl_l = prof[dom]
+    hbm, tf_burst, tf_sus, peak_kind = load_peaks()
+    avg_s = ms_l / n_l / 1e3
+    intensity = fl_l / by_l if by_l else 0.0
+    ridge = tf_sus * 1e12 / (hbm * 1e9)
+    if intensity < ridge:
+        roof = {"bound": "hbm", "achieved": by_l / n_l / avg_s / 1e9, "peak": hbm, "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": fl_l / n_l / avg_s / 1e12, "peak": tf_sus,
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic_record(dom)
+    roof["kernel"] = dom
+    roof["launches"] = n_l
+    roof["avg_us"] = avg_s * 1e6
+    roof["algorithmic_bytes_per_launch"] = by_l / n_l
+    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs / bf16_tflops_sustained)"
+    kernels = {k: {"launches": prof[k][0], "ms_per_step": prof[k][1] / K,
+                   "GBps": (prof[k][2] / (prof[k][1] / 1e3) / 1e9) if prof[k][1] else None}
+               for k in PROF_CLASSES if prof[k][0]}
+    # step roofline: all kernels' algorithmic bytes and flops at measured peaks
+    tot_b = sum(prof[k][2] for k in PROF_CLASSES) / K
+    tot_f = sum(prof[k][3] for k in PROF_CLASSES) / K
+    step_roof_ms = max(tot_b / (hbm * 1e9), tot_f / (tf_sus * 1e12)) * 1e3
+
+    # ---- end to end: positions host->device and ids device->host inside the region
+    pos_host = [torch.from_numpy(p.astype(np.int32)).pin_memory() for p in job.positions]
+    tok_host = torch.empty((total_steps, B, u), dtype=torch.int32).pin_memory()
+    pos_buf = torch.empty((B, u), dtype=torch.int32, device="cuda")
+    # rewind: refill from the same prompt so the e2e steps redo the same work
+    model.embed_tokens(toks)
+    spa.spa_decode_step(model, pos_dev[0], None, u, 1, tok_out[0])
+    for t in range(1, 1 + args.warmup):
+        spa.spa_decode_step(model, pos_dev[t], None, u, 0, tok_out[t])
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for t in range(1 + args.warmup, total_steps):
+        pos_buf.copy_(pos_host[t], non_blocking=True)
+        spa.spa_decode_step(model, pos_buf, None, u, 0, tok_out[t])
+        tok_host[t].copy_(tok_out[t], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e = {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": B * u * 4, "d2h_bytes_per_step": B * u * 4}
+
+    # ---- rho = 1 vanilla decoding (full recompute, no proxy) on the same GPU
+    vk = max(1, args.vanilla_steps)
+    spa.spa_decode_step(model, pos_dev[1], None, u, 2, tok_out[1])
+    barrier()
+    torch.cuda.synchronize()
+    v0, v1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    v0.record(stream)
+    for t in range(vk):
+        spa.spa_decode_step(model, pos_dev[1 + t], None, u, 2, tok_out[1 + t])
+    v1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    v_ms = max_over_ranks(v0.elapsed_time(v1)) / vk
+    ws.check()
+
+    # ---- CPU oracle on a bounded sample (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import budget_table
+        ks = budget_table(N, c["L"], c["rho_p"], c["l_p"], c["rho_1"], c["rho_L"])
+        kbar = int(round(sum(ks) / len(ks)))
+        sample_run = OracleSample(weights[c["l_p"] - 1], args.seed)
+        times, t_start = [], time.perf_counter()
+        while len(times) < 5 and time.perf_counter() - t_start < 25:
+            times.append(sample_run.step(kbar))
+        t_layer, n_rep = float(np.median(times)), len(times)
+        cpu = {"value": B * u / (t_layer * c["L"]), "unit": "tokens/s", "cores": cpu_cores(),
+               "kind": "oracle",
+               "sample": (f"{n_rep} oracle cached layer steps (fp64 numpy) of layer {c['l_p']} "
+                          f"at N=1024, k={kbar} (mean budget), median x 32 layers; LM head "
+                          f"excluded")}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "steps": K, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic (random LLaDA-8B-shaped weights, seeded)",
+                "config": {"workload": WORKLOAD,
+                           "parallelism": "replicas" if world > 1 else "single",
+                           "l2": "inputs larger than L2: 14 GB of layer weights streamed per step",
+                           "budget_k": model.k},
+                "us_per_layer": us_per_layer,
+                "step_roofline_ms": step_roof_ms,
+                "step_roofline_frac": step_roof_ms / ms_step,
+                "vanilla_rho1": {"tokens_per_s": world * B * u / (v_ms / 1e3), "ms_per_step": v_ms,
+                                 "speedup_spa_over_vanilla": v_ms / ms_step},
+                "roofline": roof, "kernels": kernels, "e2e": e2e, "clocks": clk,
+                "gpu_launches": launches, "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -121,6 +121,31 @@ typedef struct {
 } spa_intermediates;
 int spa_workspace_intermediates(const spa_workspace *ws, spa_intermediates *out);
 
+/* Kernel timing.  While enabled, every kernel the library launches for this
+ * workspace (layers, and models built on it) is bracketed by two CUDA events
+ * on its stream.  spa_profile_read synchronises on the recorded events and
+ * fills, per kernel class (arrays of SPA_PROF_CLASSES entries), the number
+ * of launches, their summed device time in ms, and the algorithmic bytes and
+ * flops those launches move and perform (computed from the shapes: each
+ * operand read once, each result written once), then clears the record. */
+enum {
+  SPA_PROF_PROXY = 0, /* phase 1 proxy GEMM + norm + score */
+  SPA_PROF_TOPK,      /* top-k select + P^c scatter */
+  SPA_PROF_NORM,      /* RMSNorm (gathered rows) */
+  SPA_PROF_QKV,       /* Q/K/V GEMM + RoPE + K^c/V^c scatter */
+  SPA_PROF_ATTN,      /* sparse-query attention */
+  SPA_PROF_OPROJ,     /* output projection + residual */
+  SPA_PROF_GATEUP,    /* gate/up GEMM + SwiGLU */
+  SPA_PROF_DOWN,      /* down GEMM + residual + H^c scatter */
+  SPA_PROF_LMHEAD,    /* LM head GEMM + per-tile argmax */
+  SPA_PROF_MISC,      /* embedding rows, final norm, argmax reduction */
+  SPA_PROF_CLASSES
+};
+int spa_profile_enable(spa_workspace *ws, int enable);
+int spa_profile_read(spa_workspace *ws, int *launches, double *ms, double *bytes, double *flops);
+/* Number of kernels the library has launched in this process so far. */
+long long spa_launch_count(void);
+
 /* A layer handle: borrows `w` and `ws`, owns its proxy weights W_r (stored in
  * the layer dtype) and the RoPE table.  w_r_host (host, [r, d] float) is a
  * proxy computed offline; NULL makes the library copy W_v to the host and run
