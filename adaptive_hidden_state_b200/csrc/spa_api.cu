@@ -510,6 +510,27 @@ static int run_tc(int mode, int BN, TcGemmParams& p, int M, int n_tiles, int spl
   return SPA_OK;
 }
 
+// Weight-stationary tcgen05 GEMM for M <= 256 tokens: X is the [M, K] bf16
+// token operand (row-major, 16-byte aligned).
+static int run_ws(int mode, int nacc, TcWsParams& p, const void* X, int M, int K, int n_tiles,
+                  cudaStream_t s, Profiler* prof, Work w) {
+  if (M <= 0) return SPA_OK;
+  if (M > 256) return fail(SPA_ERR_SHAPE, "weight-stationary GEMM takes at most 256 tokens");
+  const int NT = ((M + 31) / 32) * 32;
+  if (encode_bf16_map_box(&p.tmX, X, (uint64_t)M, (uint64_t)K, (uint32_t)NT))
+    return fail(SPA_ERR_CUDA, "tensor map for the token operand failed");
+  int cols = 32;
+  while (cols < nacc * NT) cols *= 2;
+  p.NT = NT;
+  p.tmem_cols = cols;
+  p.K = K;
+  const int splits = plan_ws_splits(mode, nacc, n_tiles, K / 64);
+  ProfScope ps(prof, w.cls, w.bytes, w.flops, s);
+  cudaError_t e = launch_tc_ws(mode, nacc, p, n_tiles, splits, s);
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "weight-stationary GEMM launch (mode %d): %s", mode, cudaGetErrorString(e));
+  return SPA_OK;
+}
+
 static int run_simt(int mode, SimtGemmParams& p, int M, int n_tiles, cudaStream_t s, Profiler* prof,
                     Work w) {
   const int m_tiles = (M + 63) / 64;
@@ -593,7 +614,14 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
     ep.out = ws->Q;
     ep.k_cache = c->k_cache;
     ep.v_cache = c->v_cache;
-    if (bf) {
+    if (bf && M <= 256) {
+      TcWsParams p;
+      std::memset(&p, 0, sizeof(p));
+      p.tmW[0] = L->tm_wq; p.tmW[1] = L->tm_wk; p.tmW[2] = L->tm_wv;
+      p.b_mode = B_CONCAT3; p.b_rows_per_src = d; p.ep = ep;
+      SPA_TRY(run_ws(EPI_QKV, 1, p, ws->X, M, d, 3 * d / 128, s, prof,
+                     Work{SPA_PROF_QKV, 3.0 * d * d * es + Md * es + 3.0 * Md * es, 6.0 * Md * d}));
+    } else if (bf) {
       TcGemmParams p;
       std::memset(&p, 0, sizeof(p));
       p.tmA = ws->tmX;
@@ -625,7 +653,13 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
     ep.n_out = d;
     ep.out = ws->H1;
     ep.resid = H;
-    if (bf) {
+    if (bf && M <= 256) {
+      TcWsParams p;
+      std::memset(&p, 0, sizeof(p));
+      p.tmW[0] = L->tm_wo; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
+      SPA_TRY(run_ws(EPI_RESID, 1, p, ws->O, M, d, d / 128, s, prof,
+                     Work{SPA_PROF_OPROJ, (double)d * d * es + 3.0 * Md * es, 2.0 * Md * d}));
+    } else if (bf) {
       TcGemmParams p;
       std::memset(&p, 0, sizeof(p));
       p.tmA = ws->tmO; p.tmB[0] = L->tm_wo;
@@ -653,7 +687,13 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
     EpiParams ep = base_epi(L, M, tps, N, idx);
     ep.n_out = F;
     ep.out = ws->A;
-    if (bf) {
+    if (bf && M <= 256) {
+      TcWsParams p;
+      std::memset(&p, 0, sizeof(p));
+      p.tmW[0] = L->tm_wg; p.tmW[1] = L->tm_wu; p.b_mode = B_GATEUP; p.b_rows_per_src = F; p.ep = ep;
+      SPA_TRY(run_ws(EPI_SWIGLU, 2, p, ws->X2, M, d, F / 128, s, prof,
+                     Work{SPA_PROF_GATEUP, 2.0 * F * d * es + Md * es + (double)M * F * es, 4.0 * Md * F}));
+    } else if (bf) {
       TcGemmParams p;
       std::memset(&p, 0, sizeof(p));
       p.tmA = ws->tmX2; p.tmB[0] = L->tm_wg; p.tmB[1] = L->tm_wu;
@@ -676,7 +716,13 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
     ep.n_out = d;
     ep.out = c->h_cache;
     ep.resid = ws->H1;
-    if (bf) {
+    if (bf && M <= 256) {
+      TcWsParams p;
+      std::memset(&p, 0, sizeof(p));
+      p.tmW[0] = L->tm_wd; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
+      SPA_TRY(run_ws(EPI_RESID_SCATTER, 1, p, ws->A, M, F, d / 128, s, prof,
+                     Work{SPA_PROF_DOWN, (double)d * F * es + (double)M * F * es + 2.0 * Md * es, 2.0 * Md * F}));
+    } else if (bf) {
       TcGemmParams p;
       std::memset(&p, 0, sizeof(p));
       p.tmA = ws->tmA; p.tmB[0] = L->tm_wd;
@@ -794,8 +840,7 @@ extern "C" int spa_model_create(const spa_model_desc* desc, spa_layer* const* la
     m->k.push_back(k);
   }
   const spa_layer_desc& D = ws->desc;
-  const int BN = D.dtype == SPA_BF16 ? 256 : 128;
-  m->lm_tiles = (desc->vocab + BN - 1) / BN;
+  m->lm_tiles = (desc->vocab + 127) / 128;  // the widest split: 128-column tiles
   const size_t rows = (size_t)desc->B * desc->N;
   if (cudaMalloc(&m->idx_all, (size_t)desc->n_layers * rows * 4) != cudaSuccess ||
       cudaMalloc(&m->amax_val, rows * m->lm_tiles * 4) != cudaSuccess ||
@@ -867,16 +912,25 @@ extern "C" int spa_decode_step(spa_model* m, const int32_t* pos, const int32_t* 
   ep.N = N;
   ep.amax_val = m->amax_val;
   ep.amax_idx = m->amax_idx;
-  ep.n_tiles = m->lm_tiles;
   ep.err = ws->err;
-  if (D.dtype == SPA_BF16) {
+  int tiles = m->lm_tiles;
+  if (D.dtype == SPA_BF16 && M <= 256) {
+    ep.n_tiles = tiles;
+    TcWsParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.tmW[0] = m->tm_lm; p.b_mode = B_SINGLE; p.b_rows_per_src = m->desc.vocab; p.ep = ep;
+    SPA_TRY(run_ws(EPI_ARGMAX, 1, p, ws->X, M, d, tiles, s, &ws->prof, wl));
+  } else if (D.dtype == SPA_BF16) {
+    tiles = (m->desc.vocab + 255) / 256;
+    ep.n_tiles = tiles;
     TcGemmParams p;
     std::memset(&p, 0, sizeof(p));
     p.tmA = ws->tmX;
     p.tmB[0] = m->tm_lm;
     p.K = d; p.b_mode = B_SINGLE; p.b_rows_per_src = m->desc.vocab; p.ep = ep;
-    SPA_TRY(run_tc(EPI_ARGMAX, 256, p, M, m->lm_tiles, 1, s, &ws->prof, wl));
+    SPA_TRY(run_tc(EPI_ARGMAX, 256, p, M, tiles, 1, s, &ws->prof, wl));
   } else {
+    ep.n_tiles = tiles;
     SimtGemmParams p;
     std::memset(&p, 0, sizeof(p));
     p.A = (const float*)ws->X; p.B[0] = (const float*)m->lm_head;
@@ -885,7 +939,7 @@ extern "C" int spa_decode_step(spa_model* m, const int32_t* pos, const int32_t* 
   }
   {
     ProfScope ps(&ws->prof, SPA_PROF_MISC, 8.0 * M * m->lm_tiles, 0.0, s);
-    e = launch_argmax_reduce(m->amax_val, m->amax_idx, M, m->lm_tiles, tok_out, s);
+    e = launch_argmax_reduce(m->amax_val, m->amax_idx, M, tiles, tok_out, s);
   }
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "argmax launch: %s", cudaGetErrorString(e));
   // next step's layer-0 input: embeddings of the written ids at pos

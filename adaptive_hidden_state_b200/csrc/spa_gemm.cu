@@ -380,6 +380,278 @@ cudaError_t launch_tc_gemm(int mode, int BN, const TcGemmParams& p, int m_tiles,
 }
 
 // ---------------------------------------------------------------------------
+// tcgen05 GEMM, weight-stationary (swap-AB) for few tokens (M <= 256)
+//
+// The MMA's M side (128 TMEM lanes) is a tile of 128 weight rows (output
+// features) and its N side is all NT tokens, so every weight byte is streamed
+// from HBM once per call however many tokens there are.  NACC = 2 keeps two
+// accumulators (W_gate and W_up rows of the same features) side by side in
+// TMEM.  The epilogue moves the transposed accumulator to shared memory in
+// chunks of up to 128 tokens (tile[token][feature]) and reuses run_epilogue.
+// ---------------------------------------------------------------------------
+constexpr int kWsW = 128 * 128;  // one 128-row x 64-column weight tile (bytes)
+
+__host__ __device__ constexpr int ws_stages(int nacc) { return nacc == 1 ? 4 : 3; }
+__host__ __device__ constexpr int ws_smem_bytes(int nacc) {
+  return ws_stages(nacc) * (nacc * kWsW + 256 * 128) + 1024;
+}
+
+template <int MODE, int NACC>
+__global__ void __launch_bounds__(128, 1) tc_ws_kernel(const __grid_constant__ TcWsParams p) {
+  constexpr int STAGES = ws_stages(NACC);
+  constexpr int W_BYTES = NACC * kWsW;
+  constexpr int FEAT = NACC * 128;
+  constexpr int LD = FEAT + 4;
+  static_assert(128 * LD * 4 <= STAGES * (W_BYTES + 256 * 128), "epilogue tile must fit the ring");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full_bar[STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t accum_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x, S = gridDim.x;
+  const int n_tile = blockIdx.y;
+  const int NT = p.NT;                       // tokens per MMA, multiple of 32, <= 256
+  const int X_BYTES = NT * 128;
+  const int STAGE_BYTES = W_BYTES + X_BYTES;  // multiple of 1024
+  const int KB = p.K / 64;
+  const int kb0 = (split * KB) / S, kb1 = ((split + 1) * KB) / S;
+  const int nk = kb1 - kb0;
+  int* err = p.ep.err;
+
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&accum_bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, (uint32_t)p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tmX);
+    for (int it = 0; it < nk; ++it) {
+      const int s = it % STAGES;
+      if (it >= STAGES &&
+          !mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1, &abort_flag, err, 211))
+        break;
+      uint8_t* sw = smem + s * STAGE_BYTES;
+      uint8_t* sx = sw + W_BYTES;
+      mbar_arrive_expect_tx(&full_bar[s], (uint32_t)STAGE_BYTES);
+      const int kx = (kb0 + it) * 64;
+#pragma unroll
+      for (int a = 0; a < NACC; ++a) {
+        int src, row;
+        if (p.b_mode == B_GATEUP) {
+          src = a;
+          row = n_tile * 128;
+        } else if (p.b_mode == B_CONCAT3) {
+          const int g = n_tile * 128;
+          src = g / p.b_rows_per_src;
+          row = g % p.b_rows_per_src;
+        } else {
+          src = 0;
+          row = n_tile * FEAT + a * 128;
+        }
+        tma_load_2d(sw + a * kWsW, &p.tmW[src], &full_bar[s], kx, row);
+      }
+      tma_load_2d(sx, &p.tmX, &full_bar[s], kx, 0);
+    }
+  } else if (warp == 1 && lane == 0) {
+    const uint32_t idesc = idesc_bf16_f32(128, NT);
+    for (int it = 0; it < nk; ++it) {
+      const int s = it % STAGES;
+      if (!mbar_wait(&full_bar[s], (it / STAGES) & 1, &abort_flag, err, 212)) break;
+      tc_fence_after();
+      const uint32_t sw = smem_u32(smem + s * STAGE_BYTES);
+      const uint64_t dx = smem_desc_sw128(sw + W_BYTES);
+#pragma unroll
+      for (int a = 0; a < NACC; ++a) {
+        const uint64_t dw = smem_desc_sw128(sw + a * kWsW);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16(tmem + (uint32_t)(a * NT), dw + 2 * kk, dx + 2 * kk, idesc,
+                    (it > 0 || kk > 0) ? 1u : 0u);
+      }
+      umma_commit(&empty_bar[s]);
+    }
+    umma_commit(&accum_bar);
+  }
+  __syncwarp();
+
+  mbar_wait(&accum_bar, 0, &abort_flag, err, 213);
+  __syncthreads();
+  const bool good = (abort_flag == 0);
+  tc_fence_after();
+
+  float* tile = reinterpret_cast<float*>(smem);
+  const int M = p.ep.M;
+  for (int c0 = 0; c0 < NT; c0 += 128) {
+    const int nt = min(128, NT - c0);
+    if (good) {
+      const int f = warp * 32 + lane;
+#pragma unroll 1
+      for (int a = 0; a < NACC; ++a) {
+#pragma unroll 1
+        for (int c = 0; c < nt; c += 32) {
+          float v[32];
+          if (nk > 0) {
+            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(a * NT + c0 + c), v);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.f;
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) tile[(c + j) * LD + a * 128 + f] = v[j];
+        }
+      }
+    }
+    tc_fence_before();
+    if (S > 1) {
+      cluster_sync();
+      const int q = (int)cluster_ctarank();
+      const int r0 = (q * nt) / S, r1 = ((q + 1) * nt) / S;
+      if (good) {
+        constexpr int C4 = FEAT / 4;
+        for (int it = threadIdx.x; it < (r1 - r0) * C4; it += 128) {
+          const int row = r0 + it / C4, c = (it % C4) * 4;
+          const uint32_t local = smem_u32(tile + row * LD + c);
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int src = 0; src < S; ++src) {
+            const float4 v = ld_dsmem_f4(mapa_shared(local, (uint32_t)src));
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+          }
+          *reinterpret_cast<float4*>(tile + row * LD + c) = acc;
+        }
+      }
+      cluster_sync();
+      if (good && c0 + r0 < M)
+        run_epilogue<MODE, FEAT, __nv_bfloat16>(tile, LD, r0, r1, c0, n_tile, p.ep, threadIdx.x, 128);
+    } else {
+      __syncthreads();
+      if (good && c0 < M)
+        run_epilogue<MODE, FEAT, __nv_bfloat16>(tile, LD, 0, nt, c0, n_tile, p.ep, threadIdx.x, 128);
+    }
+    __syncthreads();
+  }
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, (uint32_t)p.tmem_cols);
+}
+
+template <int MODE, int NACC>
+static cudaError_t launch_ws_typed(const TcWsParams& p, int n_tiles, int splits,
+                                   cudaStream_t stream) {
+  auto kern = tc_ws_kernel<MODE, NACC>;
+  const int smem = ws_smem_bytes(NACC);
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(splits, n_tiles, 1);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+template <int MODE, int NACC>
+static int ws_max_clusters(int splits) {
+  static int cache[9] = {0};
+  if (splits < 1 || splits > 8) return 0;
+  if (cache[splits] == 0) {
+    auto kern = tc_ws_kernel<MODE, NACC>;
+    const int smem = ws_smem_bytes(NACC);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(splits, 1, 1);
+    cfg.blockDim = dim3(128, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    cache[splits] = n > 0 ? n : -1;
+  }
+  return cache[splits] > 0 ? cache[splits] : 0;
+}
+
+#define SPA_WS_MODES(X)            \
+  X(EPI_STORE, 1)                  \
+  X(EPI_QKV, 1)                    \
+  X(EPI_RESID, 1)                  \
+  X(EPI_SWIGLU, 2)                 \
+  X(EPI_RESID_SCATTER, 1)          \
+  X(EPI_ARGMAX, 1)
+
+cudaError_t launch_tc_ws(int mode, int nacc, const TcWsParams& p, int n_tiles, int splits,
+                         cudaStream_t stream) {
+#define SPA_WS_CASE(M_, A_) \
+  if (mode == M_ && nacc == A_) return launch_ws_typed<M_, A_>(p, n_tiles, splits, stream);
+  SPA_WS_MODES(SPA_WS_CASE)
+#undef SPA_WS_CASE
+  return cudaErrorInvalidValue;
+}
+
+// Split-K plan for the weight-stationary GEMM: estimated time ~ waves x
+// (k-blocks per CTA + fixed per-CTA cost), waves from how many clusters of
+// `splits` CTAs the GPU holds at once.
+int plan_ws_splits(int mode, int nacc, int n_tiles, int KB) {
+  int best = 1;
+  double best_cost = 1e30;
+  for (int s = 1; s <= 8; ++s) {
+    if (KB / s < 2) break;
+    int fit = 0;
+#define SPA_WS_FIT(M_, A_) \
+  if (mode == M_ && nacc == A_) fit = ws_max_clusters<M_, A_>(s);
+    SPA_WS_MODES(SPA_WS_FIT)
+#undef SPA_WS_FIT
+    if (fit <= 0) continue;
+    const int waves = (n_tiles + fit - 1) / fit;
+    const double cost = waves * ((KB + s - 1) / s + 6.0);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
+
+// ---------------------------------------------------------------------------
 // fp32 CUDA-core GEMM (64 x 128 tiles, 256 threads, 4 x 8 outputs per thread)
 // ---------------------------------------------------------------------------
 constexpr int kSBM = 64, kSBN = 128, kSBK = 16;
@@ -478,6 +750,11 @@ cudaError_t launch_simt_gemm(int mode, const SimtGemmParams& p, int m_tiles, int
 // Tensor maps
 // ---------------------------------------------------------------------------
 int encode_bf16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+  return encode_bf16_map_box(map, base, rows, cols, 128);
+}
+
+int encode_bf16_map_box(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                        uint32_t box_rows) {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   if (!encode) {
     cudaDriverEntryPointQueryResult q;
@@ -490,7 +767,7 @@ int encode_bf16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
   }
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,

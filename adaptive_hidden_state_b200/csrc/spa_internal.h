@@ -65,6 +65,17 @@ struct alignas(64) TcGemmParams {
   EpiParams ep;
 };
 
+struct alignas(64) TcWsParams {
+  CUtensorMap tmW[3];  // weight sources, box 64 x 128, 128-byte swizzle
+  CUtensorMap tmX;     // token rows [M, K], box 64 x NT, 128-byte swizzle
+  int K;
+  int NT;              // tokens per MMA (multiple of 32, <= 256)
+  int tmem_cols;       // power of two >= NACC * NT
+  int b_mode;
+  int b_rows_per_src;
+  EpiParams ep;
+};
+
 struct SimtGemmParams {
   const float* A;      // [M, K]
   const float* B[3];
@@ -79,6 +90,14 @@ struct SimtGemmParams {
 // reduction through distributed shared memory.
 cudaError_t launch_tc_gemm(int mode, int BN, const TcGemmParams& p, int m_tiles, int n_tiles,
                            int splits, cudaStream_t stream);
+// Weight-stationary tcgen05 GEMM for M <= 256 tokens: 128 weight rows per
+// CTA (NACC = 2: gate and up rows) against all tokens; same epilogues.
+cudaError_t launch_tc_ws(int mode, int nacc, const TcWsParams& p, int n_tiles, int splits,
+                         cudaStream_t stream);
+int plan_ws_splits(int mode, int nacc, int n_tiles, int KB);
+// Encodes a 2D bf16 tensor map with a 64 x box_rows box.
+int encode_bf16_map_box(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                        uint32_t box_rows);
 // fp32 CUDA-core GEMM with the same epilogues, BM = 64, BN = 128.
 cudaError_t launch_simt_gemm(int mode, const SimtGemmParams& p, int m_tiles, int n_tiles,
                              cudaStream_t stream);
