@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <string>
@@ -213,6 +214,8 @@ struct spa_model {
   int32_t* amax_idx = nullptr;
   int lm_tiles = 0;
   CUtensorMap tm_lm;
+  cudaGraphExec_t graph = nullptr;  // a captured cached decode step
+  int graph_u = 0;
 };
 
 static int check_desc(const spa_layer_desc* d) {
@@ -524,7 +527,11 @@ static int run_ws(int mode, int nacc, TcWsParams& p, const void* X, int M, int K
   p.NT = NT;
   p.tmem_cols = cols;
   p.K = K;
-  const int splits = plan_ws_splits(mode, nacc, n_tiles, K / 64);
+  int splits = plan_ws_splits(mode, nacc, n_tiles, K / 64);
+  if (const char* env = std::getenv("SPA_WS_SPLITS")) {  // tuning override, 1..8
+    const int v = std::atoi(env);
+    if (v >= 1 && v <= 8 && K / 64 >= v) splits = v;
+  }
   ProfScope ps(prof, w.cls, w.bytes, w.flops, s);
   cudaError_t e = launch_tc_ws(mode, nacc, p, n_tiles, splits, s);
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "weight-stationary GEMM launch (mode %d): %s", mode, cudaGetErrorString(e));
@@ -799,6 +806,7 @@ extern "C" int spa_full_block(spa_layer* L, const void* H, const spa_layer_cache
 // ---------------------------------------------------------------------------
 extern "C" void spa_model_free(spa_model* m) {
   if (!m) return;
+  if (m->graph) cudaGraphExecDestroy(m->graph);
   if (m->idx_all) cudaFree(m->idx_all);
   if (m->amax_val) cudaFree(m->amax_val);
   if (m->amax_idx) cudaFree(m->amax_idx);
@@ -949,5 +957,40 @@ extern "C" int spa_decode_step(spa_model* m, const int32_t* pos, const int32_t* 
                           m->desc.vocab, m->h0, ws->err, s);
   }
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "embed launch: %s", cudaGetErrorString(e));
+  return SPA_OK;
+}
+
+extern "C" int spa_decode_graph_capture(spa_model* m, const int32_t* pos, const int32_t* tok_in,
+                                        int u, int32_t* tok_out, void* stream) {
+  if (!m || !pos || !tok_out) return fail(SPA_ERR_INVALID, "null argument");
+  if (!stream) return fail(SPA_ERR_INVALID, "capture needs a non-default stream");
+  cudaStream_t s = (cudaStream_t)stream;
+  spa_workspace* ws = m->layers[0]->ws;
+  const bool prof_on = ws->prof.on;
+  ws->prof.on = false;  // no timing events inside the graph
+  SPA_CK(cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal));
+  const int st = spa_decode_step(m, pos, tok_in, u, 0, tok_out, stream);
+  cudaGraph_t g = nullptr;
+  const cudaError_t ec = cudaStreamEndCapture(s, &g);
+  ws->prof.on = prof_on;
+  if (st != SPA_OK) {
+    if (g) cudaGraphDestroy(g);
+    return st;
+  }
+  if (ec != cudaSuccess) return fail(SPA_ERR_CUDA, "stream capture failed: %s", cudaGetErrorString(ec));
+  cudaGraphExec_t ex = nullptr;
+  const cudaError_t ei = cudaGraphInstantiate(&ex, g, 0);
+  cudaGraphDestroy(g);
+  if (ei != cudaSuccess) return fail(SPA_ERR_CUDA, "graph instantiation failed: %s", cudaGetErrorString(ei));
+  if (m->graph) cudaGraphExecDestroy(m->graph);
+  m->graph = ex;
+  m->graph_u = u;
+  return SPA_OK;
+}
+
+extern "C" int spa_decode_graph_launch(spa_model* m, void* stream) {
+  if (!m) return fail(SPA_ERR_INVALID, "null model");
+  if (!m->graph) return fail(SPA_ERR_INVALID, "no decode step has been captured");
+  SPA_CK(cudaGraphLaunch(m->graph, (cudaStream_t)stream));
   return SPA_OK;
 }

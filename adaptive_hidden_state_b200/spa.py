@@ -34,7 +34,7 @@ EXPORTS = [
     "spa_profile_read", "spa_launch_count", "spa_init_layer", "spa_free_layer", "spa_layer_proxy_weights",
     "spa_proxy_select", "spa_partial_block", "spa_layer_step", "spa_full_block",
     "spa_model_create", "spa_model_free", "spa_model_layer_k", "spa_model_embed",
-    "spa_decode_step",
+    "spa_decode_step", "spa_decode_graph_capture", "spa_decode_graph_launch",
 ]
 
 
@@ -114,6 +114,8 @@ _sig("spa_model_free", None, c_void_p)
 _sig("spa_model_layer_k", c_int, c_void_p, c_int)
 _sig("spa_model_embed", c_int, c_void_p, c_void_p, c_void_p)
 _sig("spa_decode_step", c_int, c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p)
+_sig("spa_decode_graph_capture", c_int, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p)
+_sig("spa_decode_graph_launch", c_int, c_void_p, c_void_p)
 
 
 def _check(status: int, where: str):
@@ -329,3 +331,12 @@ class Model:
 def spa_decode_step(model: Model, pos, tok_in, u: int, full: int, tok_out, stream=None):
     _check(lib.spa_decode_step(model.handle, _ptr(pos), _ptr(tok_in), u, int(full), _ptr(tok_out),
                                _stream(stream)), "spa_decode_step")
+
+
+def spa_decode_graph_capture(model: Model, pos, tok_in, u: int, tok_out, stream=None):
+    _check(lib.spa_decode_graph_capture(model.handle, _ptr(pos), _ptr(tok_in), u, _ptr(tok_out),
+                                        _stream(stream)), "spa_decode_graph_capture")
+
+
+def spa_decode_graph_launch(model: Model, stream=None):
+    _check(lib.spa_decode_graph_launch(model.handle, _stream(stream)), "spa_decode_graph_launch")

@@ -53,6 +53,7 @@ def parse_args():
     ap.add_argument("--vanilla-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--workload", choices=["decode", "layer"], default="decode")
     return ap.parse_args()
 
 
@@ -260,6 +261,64 @@ def run_reference(args, rank: int):
 
 # ------------------------------------------------------------------ main arm
 
+def run_layer_workload(args, spa, torch):
+    """One LLaDA-shaped bf16 layer, N=512, r=128, rho=0.25 (k=128): the rho=1
+    fill, then cached layer steps whose input alternates between H and H'
+    (5% of rows drifted by N(0, 0.3)), so each step refreshes 26 drifted rows
+    plus the lowest-index ties.  Reports us per cached layer step."""
+    c = dict(CFG, N=512)
+    d, F, r = c["d"], c["ffn"], c["r"]
+    k = 128
+    g = torch.Generator(device="cuda").manual_seed(args.seed)
+    randn = lambda shape, std: (torch.randn(shape, generator=g, device="cuda") * std).to(torch.bfloat16)
+    q1 = torch.linalg.qr(torch.randn((d, d), generator=g, device="cuda"))[0]
+    q2 = torch.linalg.qr(torch.randn((d, d), generator=g, device="cuda"))[0]
+    sigma = torch.arange(1, d + 1, device="cuda", dtype=torch.float32) ** -0.8
+    ones = torch.ones(d, device="cuda", dtype=torch.bfloat16)
+    w = {"wq": randn((d, d), .02), "wk": randn((d, d), .02),
+         "wv": ((q1 * sigma[None, :]) @ q2.T).to(torch.bfloat16), "wo": randn((d, d), .02),
+         "w_gate": randn((F, d), .02), "w_up": randn((F, d), .02), "w_down": randn((d, F), .02),
+         "attn_norm": ones, "ffn_norm": ones}
+    w_r = (sigma[:r, None] * q2[:, :r].T).float().cpu()
+    desc = spa.LayerDesc(d=d, n_heads=c["n_heads"], head_dim=c["head_dim"], ffn=F, r=r,
+                         dtype=spa.SPA_BF16, rms_eps=1e-5, rope_theta=1e4)
+    ws = spa.Workspace(desc, 1, c["N"])
+    layer = spa.Layer(desc, w, ws, w_r_host=w_r)
+    cache = spa.Cache(1, c["N"], d, r, spa.SPA_BF16)
+    H = torch.randn((1, c["N"], d), generator=g, device="cuda").to(torch.bfloat16)
+    H2 = H.clone()
+    rows = torch.randperm(c["N"], generator=torch.Generator().manual_seed(args.seed))[:26]
+    H2[0, rows] = (H2[0, rows].float() + 0.3 * torch.randn((26, d), generator=g, device="cuda")).to(torch.bfloat16)
+    idx = torch.empty((1, k), dtype=torch.int32, device="cuda")
+    spa.spa_full_block(layer, H, cache, True)
+    for t in range(args.warmup):
+        spa.spa_layer_step(layer, H2 if t % 2 == 0 else H, cache, k, idx)
+    ws.check()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for t in range(args.steps):
+        spa.spa_layer_step(layer, H2 if t % 2 == 0 else H, cache, k, idx)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / args.steps
+    ws.profile_enable(True)
+    ws.profile_read()
+    for t in range(args.steps):
+        spa.spa_layer_step(layer, H2 if t % 2 == 0 else H, cache, k, idx)
+    prof = ws.profile_read()
+    ws.check()
+    kernels = {kk: {"launches": v[0], "us_per_step": v[1] * 1e3 / args.steps,
+                    "GBps": (v[2] / (v[1] / 1e3) / 1e9) if v[1] else None}
+               for kk, v in prof.items() if v[0]}
+    print(json.dumps({"metric": "cached layer step time (single LLaDA-8B-shaped layer)",
+                      "value": us, "unit": "us/layer", "higher_is_better": False,
+                      "steps": args.steps, "warmup": args.warmup, "dtype": "bf16",
+                      "config": {"workload": "single LLaDA-8B-shaped bf16 layer, B=1, N=512, "
+                                             "r=128, rho=0.25 (k=128), 5% drifted rows"},
+                      "kernels": kernels}), flush=True)
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", "0"))
@@ -274,6 +333,9 @@ def main():
     from adaptive_hidden_state_b200 import spa, synth
 
     torch.cuda.set_device(local)
+    if args.workload == "layer":
+        run_layer_workload(args, spa, torch)
+        return
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
@@ -288,7 +350,10 @@ def main():
     toks = torch.from_numpy(job.tokens.astype(np.int32)).cuda()
     pos_dev = [torch.from_numpy(p.astype(np.int32)).cuda() for p in job.positions]
     tok_out = torch.empty((total_steps, B, u), dtype=torch.int32, device="cuda")
-    stream = torch.cuda.current_stream()
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
+    pos_buf = torch.empty((B, u), dtype=torch.int32, device="cuda")
+    tok_buf = torch.empty((B, u), dtype=torch.int32, device="cuda")
 
     def barrier():
         if world > 1:
@@ -301,23 +366,29 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    # step 0: rho = 1 fill (setup)
-    model.embed_tokens(toks)
-    spa.spa_decode_step(model, pos_dev[0], None, u, 1, tok_out[0])
-    for t in range(1, 1 + args.warmup):
-        spa.spa_decode_step(model, pos_dev[t], None, u, 0, tok_out[t])
+    def rewind():
+        """Back to the state after step 0 and the warm-up steps."""
+        model.embed_tokens(toks)
+        spa.spa_decode_step(model, pos_dev[0], None, u, 1, tok_out[0])
+        for t in range(1, 1 + args.warmup):
+            spa.spa_decode_step(model, pos_dev[t], None, u, 0, tok_out[t])
+        torch.cuda.synchronize()
+
+    # capture one cached step into a CUDA graph (fixed pos/tok buffers)
+    rewind()
+    n_cap0 = spa.spa_launch_count()
+    spa.spa_decode_graph_capture(model, pos_buf, None, u, tok_buf)
+    launches_per_step = spa.spa_launch_count() - n_cap0
     ws.check()
 
-    # ---- timed region: K cached decode steps, inputs resident in HBM
+    # ---- timed region: K cached decode steps (graph replays), inputs resident in HBM
     gpu_id = str(local)
     try:
         gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
     except Exception:
         pass
+    rewind()
     clocks = ClockSampler(gpu_id)
-    ws.profile_enable(True)
-    ws.profile_read()
-    n0 = spa.spa_launch_count()
     clocks.start()
     time.sleep(0.3)
     barrier()
@@ -325,20 +396,35 @@ def main():
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
     for t in range(1 + args.warmup, total_steps):
-        spa.spa_decode_step(model, pos_dev[t], None, u, 0, tok_out[t])
+        pos_buf.copy_(pos_dev[t], non_blocking=True)
+        spa.spa_decode_graph_launch(model)
+        tok_out[t].copy_(tok_buf, non_blocking=True)
     ev1.record(stream)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
-    launches = spa.spa_launch_count() - n0
-    prof = ws.profile_read()
-    ws.profile_enable(False)
     ws.check()
     t_ms = max_over_ranks(ev0.elapsed_time(ev1))
     K = args.steps
     tokens = world * B * u * K
     value = tokens / (t_ms / 1e3)
     ms_step = t_ms / K
+
+    # ---- profiled region: the same K steps launched directly, CUDA events per kernel
+    rewind()
+    ws.profile_enable(True)
+    ws.profile_read()
+    n0 = spa.spa_launch_count()
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    for t in range(1 + args.warmup, total_steps):
+        spa.spa_decode_step(model, pos_dev[t], None, u, 0, tok_out[t])
+    p1.record(stream)
+    torch.cuda.synchronize()
+    prof = ws.profile_read()
+    ws.profile_enable(False)
+    ws.check()
+    prof_ms_step = p0.elapsed_time(p1) / K
 
     layer_ms = sum(prof[k][1] for k in LAYER_CLASSES) / K
     us_per_layer = layer_ms * 1e3 / c["L"]
@@ -359,11 +445,10 @@ def main():
     roof["launches"] = n_l
     roof["avg_us"] = avg_s * 1e6
     roof["algorithmic_bytes_per_launch"] = by_l / n_l
-    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs / bf16_tflops_sustained)"
+    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs; bf16_tflops_sustained)"
     kernels = {k: {"launches": prof[k][0], "ms_per_step": prof[k][1] / K,
                    "GBps": (prof[k][2] / (prof[k][1] / 1e3) / 1e9) if prof[k][1] else None}
                for k in PROF_CLASSES if prof[k][0]}
-    # step roofline: all kernels' algorithmic bytes and flops at measured peaks
     tot_b = sum(prof[k][2] for k in PROF_CLASSES) / K
     tot_f = sum(prof[k][3] for k in PROF_CLASSES) / K
     step_roof_ms = max(tot_b / (hbm * 1e9), tot_f / (tf_sus * 1e12)) * 1e3
@@ -371,20 +456,15 @@ def main():
     # ---- end to end: positions host->device and ids device->host inside the region
     pos_host = [torch.from_numpy(p.astype(np.int32)).pin_memory() for p in job.positions]
     tok_host = torch.empty((total_steps, B, u), dtype=torch.int32).pin_memory()
-    pos_buf = torch.empty((B, u), dtype=torch.int32, device="cuda")
-    # rewind: refill from the same prompt so the e2e steps redo the same work
-    model.embed_tokens(toks)
-    spa.spa_decode_step(model, pos_dev[0], None, u, 1, tok_out[0])
-    for t in range(1, 1 + args.warmup):
-        spa.spa_decode_step(model, pos_dev[t], None, u, 0, tok_out[t])
+    rewind()
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for t in range(1 + args.warmup, total_steps):
         pos_buf.copy_(pos_host[t], non_blocking=True)
-        spa.spa_decode_step(model, pos_buf, None, u, 0, tok_out[t])
-        tok_host[t].copy_(tok_out[t], non_blocking=True)
+        spa.spa_decode_graph_launch(model)
+        tok_host[t].copy_(tok_buf, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -394,6 +474,7 @@ def main():
 
     # ---- rho = 1 vanilla decoding (full recompute, no proxy) on the same GPU
     vk = max(1, args.vanilla_steps)
+    rewind()
     spa.spa_decode_step(model, pos_dev[1], None, u, 2, tok_out[1])
     barrier()
     torch.cuda.synchronize()
@@ -432,14 +513,19 @@ def main():
                 "config": {"workload": WORKLOAD,
                            "parallelism": "replicas" if world > 1 else "single",
                            "l2": "inputs larger than L2: 14 GB of layer weights streamed per step",
+                           "launch": "one CUDA graph replay per decode step",
                            "budget_k": model.k},
                 "us_per_layer": us_per_layer,
                 "step_roofline_ms": step_roof_ms,
                 "step_roofline_frac": step_roof_ms / ms_step,
                 "vanilla_rho1": {"tokens_per_s": world * B * u / (v_ms / 1e3), "ms_per_step": v_ms,
                                  "speedup_spa_over_vanilla": v_ms / ms_step},
-                "roofline": roof, "kernels": kernels, "e2e": e2e, "clocks": clk,
-                "gpu_launches": launches, "cpu_baseline": cpu}
+                "roofline": roof,
+                "profiled_region": {"ms_per_step": prof_ms_step,
+                                    "note": "same steps launched directly with CUDA events "
+                                            "around every kernel"},
+                "kernels": kernels, "e2e": e2e, "clocks": clk,
+                "gpu_launches": launches_per_step * K, "cpu_baseline": cpu}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -228,6 +228,17 @@ int spa_model_embed(spa_model *model, const int32_t *tokens, void *stream);
 int spa_decode_step(spa_model *model, const int32_t *pos, const int32_t *tok_in, int u, int full,
                     int32_t *tok_out, void *stream);
 
+/* CUDA-graph form of the cached decode step (full = 0).  Capture records one
+ * step with fixed device buffers pos ([B, u]), tok_in ([B, u] or NULL) and
+ * tok_out ([B, u]) on `stream` (must not be the legacy default stream; the
+ * step must not be running elsewhere), replacing any earlier capture.  Each
+ * launch replays it: the caller writes the step's positions (and forced ids)
+ * into those buffers first.  Kernel timing events are not recorded inside the
+ * graph.  The graph belongs to the model and is freed with it. */
+int spa_decode_graph_capture(spa_model *model, const int32_t *pos, const int32_t *tok_in, int u,
+                             int32_t *tok_out, void *stream);
+int spa_decode_graph_launch(spa_model *model, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
