@@ -226,6 +226,7 @@ static int check_desc(const spa_layer_desc* d) {
   if (d->n_heads * d->head_dim != d->d) return fail(SPA_ERR_SHAPE, "d != n_heads * head_dim");
   if (d->head_dim % 8 != 0 || d->head_dim > 128) return fail(SPA_ERR_UNSUPPORTED, "head_dim must be a multiple of 8, <= 128");
   if (d->r > d->d) return fail(SPA_ERR_SHAPE, "r > d");
+  if (d->d > 8192) return fail(SPA_ERR_UNSUPPORTED, "d must be <= 8192");
   if (!(d->rms_eps > 0.f) || !(d->rope_theta > 0.f)) return fail(SPA_ERR_INVALID, "eps and theta must be positive");
   if (d->dtype == SPA_BF16) {
     if (d->d % 256 != 0) return fail(SPA_ERR_UNSUPPORTED, "bf16: d must be a multiple of 256");

@@ -24,52 +24,84 @@ namespace spa {
 
 // ---------------------------------------------------------------------------
 // Epilogues over an fp32 tile held in shared memory (row-major, stride ld).
+//
+// The epilogues are latency-bound (a few dependent global accesses per
+// output), so each thread works on kUnroll items at a time with all their
+// global loads issued before any result is used, and the cache row of every
+// tile row (b, position in I) is staged in shared memory once per tile.
 // ---------------------------------------------------------------------------
-struct TokenRow {
-  int b, pos;
-  bool ok;
-};
-
-__device__ __forceinline__ TokenRow token_row(const EpiParams& ep, int t) {
-  TokenRow r;
-  r.b = t / ep.tokens_per_seq;
-  r.pos = ep.idx ? ep.idx[t] : (t % ep.tokens_per_seq);
-  r.ok = (r.pos >= 0 && r.pos < ep.N);
-  if (!r.ok) report_error(ep.err, DEVERR_INDEX, 101);
-  return r;
-}
+constexpr int kUnroll = 4;
 
 __device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
 
+// s_rows[row] = (sequence b, cache row) of token t = gm0 + row; (0, -1) when
+// t >= M or the index is out of range (the latter is reported).
+__device__ void stage_rows(const EpiParams& ep, int gm0, int row_begin, int row_end, int2* s_rows,
+                           int tid, int nthr) {
+  for (int row = row_begin + tid; row < row_end; row += nthr) {
+    const int t = gm0 + row;
+    int2 v = make_int2(0, -1);
+    if (t < ep.M) {
+      v.x = t / ep.tokens_per_seq;
+      v.y = ep.idx ? ep.idx[t] : (t % ep.tokens_per_seq);
+      if (v.y < 0 || v.y >= ep.N) {
+        report_error(ep.err, DEVERR_INDEX, 101);
+        v.y = -1;
+      }
+    }
+    s_rows[row] = v;
+  }
+}
+
 template <int MODE, int BN, typename T>
 __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_end, int gm0,
-                             int n_tile, const EpiParams& ep, int tid, int nthr) {
+                             int n_tile, const EpiParams& ep, const int2* s_rows, int tid,
+                             int nthr) {
   const int nrows = row_end - row_begin;
   if (nrows <= 0) return;
 
   if constexpr (MODE == EPI_STORE || MODE == EPI_RESID || MODE == EPI_RESID_SCATTER) {
     constexpr int C4 = BN / 4;
     const int gn0 = n_tile * BN;
-    for (int it = tid; it < nrows * C4; it += nthr) {
-      const int row = row_begin + it / C4, c = (it % C4) * 4;
-      const int t = gm0 + row, gn = gn0 + c;
-      if (t >= ep.M || gn >= ep.n_out) continue;
-      float4 v = *reinterpret_cast<const float4*>(tile + row * ld + c);
-      if constexpr (MODE == EPI_STORE) {
-        store4(reinterpret_cast<T*>(ep.out) + (size_t)t * ep.n_out + gn, v);
-      } else if constexpr (MODE == EPI_RESID) {
-        TokenRow tr = token_row(ep, t);
-        if (!tr.ok) continue;
-        float4 h = load4(reinterpret_cast<const T*>(ep.resid) +
-                         ((size_t)tr.b * ep.N + tr.pos) * ep.d + gn);
-        v.x += h.x; v.y += h.y; v.z += h.z; v.w += h.w;
-        store4(reinterpret_cast<T*>(ep.out) + (size_t)t * ep.d + gn, v);
-      } else {
-        TokenRow tr = token_row(ep, t);
-        if (!tr.ok) continue;
-        float4 h = load4(reinterpret_cast<const T*>(ep.resid) + (size_t)t * ep.d + gn);
-        v.x += h.x; v.y += h.y; v.z += h.z; v.w += h.w;
-        store4(reinterpret_cast<T*>(ep.out) + ((size_t)tr.b * ep.N + tr.pos) * ep.d + gn, v);
+    const int total = nrows * C4;
+    for (int base = tid; base < total; base += nthr * kUnroll) {
+      float4 v[kUnroll], h[kUnroll];
+      int row[kUnroll], c[kUnroll];
+      bool ok[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int it = base + u * nthr;
+        row[u] = row_begin + it / C4;
+        c[u] = (it % C4) * 4;
+        const int t = gm0 + row[u], gn = gn0 + c[u];
+        ok[u] = it < total && t < ep.M && gn < ep.n_out;
+        if (MODE != EPI_STORE && ok[u]) ok[u] = s_rows[row[u]].y >= 0;
+        if (ok[u]) {
+          v[u] = *reinterpret_cast<const float4*>(tile + row[u] * ld + c[u]);
+          if constexpr (MODE == EPI_RESID) {
+            const int2 br = s_rows[row[u]];
+            h[u] = load4(reinterpret_cast<const T*>(ep.resid) + ((size_t)br.x * ep.N + br.y) * ep.d + gn);
+          } else if constexpr (MODE == EPI_RESID_SCATTER) {
+            h[u] = load4(reinterpret_cast<const T*>(ep.resid) + (size_t)t * ep.d + gn);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        if (!ok[u]) continue;
+        const int t = gm0 + row[u], gn = gn0 + c[u];
+        float4 r = v[u];
+        if constexpr (MODE == EPI_STORE) {
+          store4(reinterpret_cast<T*>(ep.out) + (size_t)t * ep.n_out + gn, r);
+        } else {
+          r.x += h[u].x; r.y += h[u].y; r.z += h[u].z; r.w += h[u].w;
+          if constexpr (MODE == EPI_RESID) {
+            store4(reinterpret_cast<T*>(ep.out) + (size_t)t * ep.d + gn, r);
+          } else {
+            const int2 br = s_rows[row[u]];
+            store4(reinterpret_cast<T*>(ep.out) + ((size_t)br.x * ep.N + br.y) * ep.d + gn, r);
+          }
+        }
       }
     }
   } else if constexpr (MODE == EPI_SWIGLU) {
@@ -79,9 +111,9 @@ __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_e
       const int row = row_begin + it / C4, c = (it % C4) * 4;
       const int t = gm0 + row, f = f0 + c;
       if (t >= ep.M || f >= ep.n_out) continue;
-      float4 g = *reinterpret_cast<const float4*>(tile + row * ld + c);
-      float4 u = *reinterpret_cast<const float4*>(tile + row * ld + HALF + c);
-      float4 a = make_float4(silu(g.x) * u.x, silu(g.y) * u.y, silu(g.z) * u.z, silu(g.w) * u.w);
+      const float4 g = *reinterpret_cast<const float4*>(tile + row * ld + c);
+      const float4 u = *reinterpret_cast<const float4*>(tile + row * ld + HALF + c);
+      const float4 a = make_float4(silu(g.x) * u.x, silu(g.y) * u.y, silu(g.z) * u.z, silu(g.w) * u.w);
       store4(reinterpret_cast<T*>(ep.out) + (size_t)t * ep.n_out + f, a);
     }
   } else if constexpr (MODE == EPI_QKV) {
@@ -90,56 +122,85 @@ __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_e
     const int items_per_head = hh / 4;
     const int items = (BN / hd) * items_per_head;
     const int gn0 = n_tile * BN;
-    for (int it = tid; it < nrows * items; it += nthr) {
-      const int row = row_begin + it / items, w = it % items;
-      const int t = gm0 + row;
-      if (t >= ep.M) continue;
-      const int hl = w / items_per_head, j = (w % items_per_head) * 4;
-      const int c1 = hl * hd + j, c2 = c1 + hh;
-      const int g1 = gn0 + c1;
-      if (g1 >= ep.n_out) continue;
-      const int part = g1 / ep.d, col1 = g1 % ep.d, col2 = col1 + hh;
-      float4 x1 = *reinterpret_cast<const float4*>(tile + row * ld + c1);
-      float4 x2 = *reinterpret_cast<const float4*>(tile + row * ld + c2);
-      TokenRow tr = token_row(ep, t);
-      if (!tr.ok) continue;
-      if (part < 2) {
-        const float4 cs = *reinterpret_cast<const float4*>(ep.rope_cos + (size_t)tr.pos * hh + j);
-        const float4 sn = *reinterpret_cast<const float4*>(ep.rope_sin + (size_t)tr.pos * hh + j);
-        float4 y1, y2;
-        y1.x = x1.x * cs.x - x2.x * sn.x; y2.x = x2.x * cs.x + x1.x * sn.x;
-        y1.y = x1.y * cs.y - x2.y * sn.y; y2.y = x2.y * cs.y + x1.y * sn.y;
-        y1.z = x1.z * cs.z - x2.z * sn.z; y2.z = x2.z * cs.z + x1.z * sn.z;
-        y1.w = x1.w * cs.w - x2.w * sn.w; y2.w = x2.w * cs.w + x1.w * sn.w;
-        x1 = y1; x2 = y2;
+    const int total = nrows * items;
+    for (int base = tid; base < total; base += nthr * kUnroll) {
+      float4 x1[kUnroll], x2[kUnroll], cs[kUnroll], sn[kUnroll];
+      int row[kUnroll], c1[kUnroll], j[kUnroll];
+      bool ok[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int it = base + u * nthr;
+        row[u] = row_begin + it / items;
+        const int w = it % items;
+        const int hl = w / items_per_head;
+        j[u] = (w % items_per_head) * 4;
+        c1[u] = hl * hd + j[u];
+        const int g1 = gn0 + c1[u];
+        ok[u] = it < total && gm0 + row[u] < ep.M && g1 < ep.n_out && s_rows[row[u]].y >= 0;
+        if (ok[u]) {
+          x1[u] = *reinterpret_cast<const float4*>(tile + row[u] * ld + c1[u]);
+          x2[u] = *reinterpret_cast<const float4*>(tile + row[u] * ld + c1[u] + hh);
+          if (g1 / ep.d < 2) {
+            const size_t off = (size_t)s_rows[row[u]].y * hh + j[u];
+            cs[u] = *reinterpret_cast<const float4*>(ep.rope_cos + off);
+            sn[u] = *reinterpret_cast<const float4*>(ep.rope_sin + off);
+          }
+        }
       }
-      T* dst;
-      if (part == 0) dst = reinterpret_cast<T*>(ep.out) + (size_t)t * ep.d;
-      else dst = reinterpret_cast<T*>(part == 1 ? ep.k_cache : ep.v_cache) +
-                 ((size_t)tr.b * ep.N + tr.pos) * ep.d;
-      store4(dst + col1, x1);
-      store4(dst + col2, x2);
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        if (!ok[u]) continue;
+        const int g1 = gn0 + c1[u];
+        const int part = g1 / ep.d, col1 = g1 % ep.d, col2 = col1 + hh;
+        float4 a = x1[u], bb = x2[u];
+        if (part < 2) {
+          const float4 c = cs[u], s_ = sn[u];
+          a = make_float4(x1[u].x * c.x - x2[u].x * s_.x, x1[u].y * c.y - x2[u].y * s_.y,
+                          x1[u].z * c.z - x2[u].z * s_.z, x1[u].w * c.w - x2[u].w * s_.w);
+          bb = make_float4(x2[u].x * c.x + x1[u].x * s_.x, x2[u].y * c.y + x1[u].y * s_.y,
+                           x2[u].z * c.z + x1[u].z * s_.z, x2[u].w * c.w + x1[u].w * s_.w);
+        }
+        const int t = gm0 + row[u];
+        const int2 br = s_rows[row[u]];
+        T* dst;
+        if (part == 0) dst = reinterpret_cast<T*>(ep.out) + (size_t)t * ep.d;
+        else dst = reinterpret_cast<T*>(part == 1 ? ep.k_cache : ep.v_cache) +
+                   ((size_t)br.x * ep.N + br.y) * ep.d;
+        store4(dst + col1, a);
+        store4(dst + col2, bb);
+      }
     }
   } else if constexpr (MODE == EPI_PROXY) {
-    // One warp per token row: norm, unit proxy, drift score.
+    // One warp per token row: norm, unit proxy, drift score.  r <= 256, so a
+    // lane holds at most 8 columns (c = lane + 32 j).
     const int lane = tid & 31, wid = tid >> 5, nw = nthr >> 5;
     const int r = ep.n_out;
     for (int row = row_begin + wid; row < row_end; row += nw) {
       const int t = gm0 + row;
       if (t >= ep.M) continue;
       const float* src = tile + row * ld;
+      float a[8], pc[8];
       float ss = 0.f;
-      for (int c = lane; c < r; c += 32) ss += src[c] * src[c];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int c = lane + 32 * j;
+        a[j] = c < r ? src[c] : 0.f;
+        pc[j] = (!ep.proxy_fill && c < r) ? ep.p_cache[(size_t)t * r + c] : 0.f;
+        ss += a[j] * a[j];
+      }
       ss = warp_sum(ss);
       const float nrm = sqrtf(ss);
       float sd = 0.f;
-      for (int c = lane; c < r; c += 32) {
-        const float a = ss > 0.f ? src[c] / nrm : 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int c = lane + 32 * j;
+        if (c >= r) continue;
+        const float ah = ss > 0.f ? a[j] / nrm : 0.f;
         if (ep.proxy_fill) {
-          ep.p_cache[(size_t)t * r + c] = a;
+          ep.p_cache[(size_t)t * r + c] = ah;
         } else {
-          ep.a_hat[(size_t)t * r + c] = a;
-          const float df = a - ep.p_cache[(size_t)t * r + c];
+          ep.a_hat[(size_t)t * r + c] = ah;
+          const float df = ah - pc[j];
           sd += df * df;
         }
       }
@@ -176,8 +237,28 @@ __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_e
   }
 }
 
+// Rows [r0, r1) of the cluster's S partial tiles summed in the fixed order
+// 0..S-1 into this CTA's tile (all S loads of an element issued first).
+template <int W>
+__device__ void cluster_reduce_rows(float* tile, int ld, int r0, int r1, int S, int tid, int nthr) {
+  constexpr int C4 = W / 4;
+  for (int it = tid; it < (r1 - r0) * C4; it += nthr) {
+    const int row = r0 + it / C4, c = (it % C4) * 4;
+    const uint32_t local = smem_u32(tile + row * ld + c);
+    float4 v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (q < S) v[q] = ld_dsmem_f4(mapa_shared(local, (uint32_t)q));
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (q < S) { acc.x += v[q].x; acc.y += v[q].y; acc.z += v[q].z; acc.w += v[q].w; }
+    *reinterpret_cast<float4*>(tile + row * ld + c) = acc;
+  }
+}
+
 // ---------------------------------------------------------------------------
-// tcgen05 GEMM
+// tcgen05 GEMM (token rows on the MMA's M side; used for M > 256 and the proxy)
 // ---------------------------------------------------------------------------
 template <int BN>
 __device__ __forceinline__ void b_source(const TcGemmParams& p, int n_tile, int half, int& src,
@@ -195,27 +276,30 @@ __device__ __forceinline__ void b_source(const TcGemmParams& p, int n_tile, int 
   }
 }
 
-constexpr int kTcStages = 4;
 constexpr int kTcABytes = 128 * 128;  // 128 rows x 64 bf16
+constexpr int kThreads = 256;         // 8 warps: producer, MMA issuer, all 8 in the epilogue
 
+__host__ __device__ constexpr int tc_stages(int BN) { return BN == 256 ? 4 : 6; }
 __host__ __device__ constexpr int tc_smem_bytes(int BN) {
-  return kTcStages * (kTcABytes + BN * 128) + 1024;
+  return tc_stages(BN) * (kTcABytes + BN * 128) + 1024;
 }
 
 template <int MODE, int BN>
-__global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
+__global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
+  constexpr int STAGES = tc_stages(BN);
   constexpr int B_BYTES = BN * 128;
   constexpr int STAGE_BYTES = kTcABytes + B_BYTES;
   constexpr int LD = BN + 4;
-  static_assert(128 * LD * 4 <= kTcStages * STAGE_BYTES, "epilogue tile must fit the ring");
+  static_assert(128 * LD * 4 <= STAGES * STAGE_BYTES, "epilogue tile must fit the ring");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t full_bar[kTcStages];
-  __shared__ __align__(8) uint64_t empty_bar[kTcStages];
+  __shared__ __align__(8) uint64_t full_bar[STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[STAGES];
   __shared__ __align__(8) uint64_t accum_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  __shared__ int2 s_rows[128];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, S = gridDim.x;
@@ -227,7 +311,7 @@ __global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__
 
   if (threadIdx.x == 0) {
 #pragma unroll
-    for (int s = 0; s < kTcStages; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
@@ -245,12 +329,10 @@ __global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__
   const uint32_t tmem = tmem_slot;
 
   if (warp == 0 && lane == 0) {
-    // TMA producer
     tma_prefetch_desc(&p.tmA);
     for (int it = 0; it < nk; ++it) {
-      const int s = it % kTcStages;
-      if (it >= kTcStages &&
-          !mbar_wait(&empty_bar[s], ((it / kTcStages) - 1) & 1, &abort_flag, err, 201))
+      const int s = it % STAGES;
+      if (it >= STAGES && !mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1, &abort_flag, err, 201))
         break;
       uint8_t* sa = smem + s * STAGE_BYTES;
       uint8_t* sb = sa + kTcABytes;
@@ -265,11 +347,10 @@ __global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__
       }
     }
   } else if (warp == 1 && lane == 0) {
-    // MMA issuer
     constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
     for (int it = 0; it < nk; ++it) {
-      const int s = it % kTcStages;
-      if (!mbar_wait(&full_bar[s], (it / kTcStages) & 1, &abort_flag, err, 202)) break;
+      const int s = it % STAGES;
+      if (!mbar_wait(&full_bar[s], (it / STAGES) & 1, &abort_flag, err, 202)) break;
       tc_fence_after();
       const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
       const uint64_t da = smem_desc_sw128(sa);
@@ -290,19 +371,20 @@ __global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__
 
   float* tile = reinterpret_cast<float*>(smem);
   if (good) {
-    const int row = warp * 32 + lane;
-    float* dst = tile + row * LD;
-    if (nk > 0) {
+    const int q = warp & 3, half = warp >> 2;
+    float* dst = tile + (q * 32 + lane) * LD;
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        float v[32];
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
+    for (int c = 32 * half; c < BN; c += 64) {
+      float v[32];
+      if (nk > 0) {
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
+      } else {
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
-          *reinterpret_cast<float4*>(dst + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        for (int j = 0; j < 32; ++j) v[j] = 0.f;
       }
-    } else {
-      for (int c = 0; c < BN; c += 4) *reinterpret_cast<float4*>(dst + c) = make_float4(0, 0, 0, 0);
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        *reinterpret_cast<float4*>(dst + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
     }
   }
   tc_fence_before();
@@ -310,29 +392,20 @@ __global__ void __launch_bounds__(128, 1) tc_gemm_kernel(const __grid_constant__
   if (warp == 0) tmem_dealloc(tmem, BN);
 
   const int gm0 = m_tile * 128;
+  int r0 = 0, r1 = 128;
   if (S > 1) {
     cluster_sync();
     const int q = (int)cluster_ctarank();
-    const int r0 = (q * 128) / S, r1 = ((q + 1) * 128) / S;
-    if (good) {
-      constexpr int C4 = BN / 4;
-      for (int it = threadIdx.x; it < (r1 - r0) * C4; it += 128) {
-        const int row = r0 + it / C4, c = (it % C4) * 4;
-        const uint32_t local = smem_u32(tile + row * LD + c);
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int src = 0; src < S; ++src) {
-          const float4 v = ld_dsmem_f4(mapa_shared(local, (uint32_t)src));
-          acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-        }
-        *reinterpret_cast<float4*>(tile + row * LD + c) = acc;
-      }
-    }
+    r0 = (q * 128) / S;
+    r1 = ((q + 1) * 128) / S;
+    if (good) cluster_reduce_rows<BN>(tile, LD, r0, r1, S, threadIdx.x, kThreads);
     cluster_sync();
-    if (good)
-      run_epilogue<MODE, BN, __nv_bfloat16>(tile, LD, r0, r1, gm0, n_tile, p.ep, threadIdx.x, 128);
-  } else {
-    if (good)
-      run_epilogue<MODE, BN, __nv_bfloat16>(tile, LD, 0, 128, gm0, n_tile, p.ep, threadIdx.x, 128);
+  }
+  if (good) {
+    stage_rows(p.ep, gm0, r0, r1, s_rows, threadIdx.x, kThreads);
+    __syncthreads();
+    run_epilogue<MODE, BN, __nv_bfloat16>(tile, LD, r0, r1, gm0, n_tile, p.ep, s_rows, threadIdx.x,
+                                          kThreads);
   }
 }
 
@@ -349,7 +422,7 @@ static cudaError_t launch_tc_typed(const TcGemmParams& p, int m_tiles, int n_til
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(splits, n_tiles, m_tiles);
-  cfg.blockDim = dim3(128, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -386,36 +459,42 @@ cudaError_t launch_tc_gemm(int mode, int BN, const TcGemmParams& p, int m_tiles,
 // features) and its N side is all NT tokens, so every weight byte is streamed
 // from HBM once per call however many tokens there are.  NACC = 2 keeps two
 // accumulators (W_gate and W_up rows of the same features) side by side in
-// TMEM.  The epilogue moves the transposed accumulator to shared memory in
-// chunks of up to 128 tokens (tile[token][feature]) and reuses run_epilogue.
+// TMEM.  The TMA ring is as deep as a fixed shared-memory budget allows for
+// the stage size (fewer tokens -> more stages in flight).  The epilogue moves
+// the transposed accumulator to shared memory in chunks of up to 128 tokens
+// (tile[token][feature]) and reuses run_epilogue.
 // ---------------------------------------------------------------------------
-constexpr int kWsW = 128 * 128;  // one 128-row x 64-column weight tile (bytes)
+constexpr int kWsW = 128 * 128;          // one 128-row x 64-column weight tile (bytes)
+constexpr int kWsRing = 200 * 1024;      // bytes of the TMA ring
+constexpr int kWsMaxStages = 8;
+constexpr int kWsSmem = kWsRing + 1024;
 
-__host__ __device__ constexpr int ws_stages(int nacc) { return nacc == 1 ? 4 : 3; }
-__host__ __device__ constexpr int ws_smem_bytes(int nacc) {
-  return ws_stages(nacc) * (nacc * kWsW + 256 * 128) + 1024;
+__host__ __device__ inline int ws_stages(int nacc, int NT) {
+  const int st = kWsRing / (nacc * kWsW + NT * 128);
+  return st < kWsMaxStages ? st : kWsMaxStages;
 }
 
 template <int MODE, int NACC>
-__global__ void __launch_bounds__(128, 1) tc_ws_kernel(const __grid_constant__ TcWsParams p) {
-  constexpr int STAGES = ws_stages(NACC);
+__global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constant__ TcWsParams p) {
   constexpr int W_BYTES = NACC * kWsW;
   constexpr int FEAT = NACC * 128;
   constexpr int LD = FEAT + 4;
-  static_assert(128 * LD * 4 <= STAGES * (W_BYTES + 256 * 128), "epilogue tile must fit the ring");
+  static_assert(128 * LD * 4 <= kWsRing, "epilogue tile must fit the ring");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t full_bar[STAGES];
-  __shared__ __align__(8) uint64_t empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t full_bar[kWsMaxStages];
+  __shared__ __align__(8) uint64_t empty_bar[kWsMaxStages];
   __shared__ __align__(8) uint64_t accum_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  __shared__ int2 s_rows[128];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, S = gridDim.x;
   const int n_tile = blockIdx.y;
-  const int NT = p.NT;                       // tokens per MMA, multiple of 32, <= 256
+  const int NT = p.NT;  // tokens per MMA, multiple of 32, <= 256
+  const int STAGES = ws_stages(NACC, NT);
   const int X_BYTES = NT * 128;
   const int STAGE_BYTES = W_BYTES + X_BYTES;  // multiple of 1024
   const int KB = p.K / 64;
@@ -424,7 +503,6 @@ __global__ void __launch_bounds__(128, 1) tc_ws_kernel(const __grid_constant__ T
   int* err = p.ep.err;
 
   if (threadIdx.x == 0) {
-#pragma unroll
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
@@ -446,8 +524,7 @@ __global__ void __launch_bounds__(128, 1) tc_ws_kernel(const __grid_constant__ T
     tma_prefetch_desc(&p.tmX);
     for (int it = 0; it < nk; ++it) {
       const int s = it % STAGES;
-      if (it >= STAGES &&
-          !mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1, &abort_flag, err, 211))
+      if (it >= STAGES && !mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1, &abort_flag, err, 211))
         break;
       uint8_t* sw = smem + s * STAGE_BYTES;
       uint8_t* sx = sw + W_BYTES;
@@ -500,17 +577,18 @@ __global__ void __launch_bounds__(128, 1) tc_ws_kernel(const __grid_constant__ T
 
   float* tile = reinterpret_cast<float*>(smem);
   const int M = p.ep.M;
+  const int q4 = warp & 3, half = warp >> 2;
   for (int c0 = 0; c0 < NT; c0 += 128) {
     const int nt = min(128, NT - c0);
     if (good) {
-      const int f = warp * 32 + lane;
+      const int f = q4 * 32 + lane;
 #pragma unroll 1
       for (int a = 0; a < NACC; ++a) {
 #pragma unroll 1
-        for (int c = 0; c < nt; c += 32) {
+        for (int c = 32 * half; c < nt; c += 64) {
           float v[32];
           if (nk > 0) {
-            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(a * NT + c0 + c), v);
+            tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(a * NT + c0 + c), v);
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = 0.f;
@@ -521,30 +599,22 @@ __global__ void __launch_bounds__(128, 1) tc_ws_kernel(const __grid_constant__ T
       }
     }
     tc_fence_before();
+    int r0 = 0, r1 = nt;
     if (S > 1) {
       cluster_sync();
       const int q = (int)cluster_ctarank();
-      const int r0 = (q * nt) / S, r1 = ((q + 1) * nt) / S;
-      if (good) {
-        constexpr int C4 = FEAT / 4;
-        for (int it = threadIdx.x; it < (r1 - r0) * C4; it += 128) {
-          const int row = r0 + it / C4, c = (it % C4) * 4;
-          const uint32_t local = smem_u32(tile + row * LD + c);
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int src = 0; src < S; ++src) {
-            const float4 v = ld_dsmem_f4(mapa_shared(local, (uint32_t)src));
-            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-          }
-          *reinterpret_cast<float4*>(tile + row * LD + c) = acc;
-        }
-      }
+      r0 = (q * nt) / S;
+      r1 = ((q + 1) * nt) / S;
+      if (good) cluster_reduce_rows<FEAT>(tile, LD, r0, r1, S, threadIdx.x, kThreads);
       cluster_sync();
-      if (good && c0 + r0 < M)
-        run_epilogue<MODE, FEAT, __nv_bfloat16>(tile, LD, r0, r1, c0, n_tile, p.ep, threadIdx.x, 128);
     } else {
       __syncthreads();
-      if (good && c0 < M)
-        run_epilogue<MODE, FEAT, __nv_bfloat16>(tile, LD, 0, nt, c0, n_tile, p.ep, threadIdx.x, 128);
+    }
+    if (good && c0 + r0 < M) {
+      stage_rows(p.ep, c0, r0, r1, s_rows, threadIdx.x, kThreads);
+      __syncthreads();
+      run_epilogue<MODE, FEAT, __nv_bfloat16>(tile, LD, r0, r1, c0, n_tile, p.ep, s_rows,
+                                              threadIdx.x, kThreads);
     }
     __syncthreads();
   }
@@ -556,17 +626,16 @@ template <int MODE, int NACC>
 static cudaError_t launch_ws_typed(const TcWsParams& p, int n_tiles, int splits,
                                    cudaStream_t stream) {
   auto kern = tc_ws_kernel<MODE, NACC>;
-  const int smem = ws_smem_bytes(NACC);
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kWsSmem);
     if (e != cudaSuccess) return e;
     configured = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(splits, n_tiles, 1);
-  cfg.blockDim = dim3(128, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kWsSmem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -584,15 +653,14 @@ static int ws_max_clusters(int splits) {
   if (splits < 1 || splits > 8) return 0;
   if (cache[splits] == 0) {
     auto kern = tc_ws_kernel<MODE, NACC>;
-    const int smem = ws_smem_bytes(NACC);
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kWsSmem) != cudaSuccess) {
       cudaGetLastError();
       return 0;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(splits, 1, 1);
-    cfg.blockDim = dim3(128, 1, 1);
-    cfg.dynamicSmemBytes = smem;
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kWsSmem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = splits;
@@ -628,8 +696,8 @@ cudaError_t launch_tc_ws(int mode, int nacc, const TcWsParams& p, int n_tiles, i
 }
 
 // Split-K plan for the weight-stationary GEMM: estimated time ~ waves x
-// (k-blocks per CTA + fixed per-CTA cost), waves from how many clusters of
-// `splits` CTAs the GPU holds at once.
+// (k-blocks per CTA + fixed per-CTA cost in k-block units), waves from how
+// many clusters of `splits` CTAs the GPU holds at once.
 int plan_ws_splits(int mode, int nacc, int n_tiles, int KB) {
   int best = 1;
   double best_cost = 1e30;
@@ -642,7 +710,7 @@ int plan_ws_splits(int mode, int nacc, int n_tiles, int KB) {
 #undef SPA_WS_FIT
     if (fit <= 0) continue;
     const int waves = (n_tiles + fit - 1) / fit;
-    const double cost = waves * ((KB + s - 1) / s + 6.0);
+    const double cost = waves * ((KB + s - 1) / s + 12.0);
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best = s;
@@ -726,8 +794,10 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtGemmParams p) 
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) tile[(ty * 4 + i) * LD + tx * 8 + j] = acc[i][j];
+  __shared__ int2 s_rows[kSBM];
+  stage_rows(p.ep, m_tile * kSBM, 0, kSBM, s_rows, tid, 256);
   __syncthreads();
-  run_epilogue<MODE, kSBN, float>(tile, LD, 0, kSBM, m_tile * kSBM, n_tile, p.ep, tid, 256);
+  run_epilogue<MODE, kSBN, float>(tile, LD, 0, kSBM, m_tile * kSBM, n_tile, p.ep, s_rows, tid, 256);
 }
 
 cudaError_t launch_simt_gemm(int mode, const SimtGemmParams& p, int m_tiles, int n_tiles,

@@ -10,13 +10,54 @@ namespace spa {
 
 // ---------------------------------------------------------------------------
 // RMSNorm of gathered rows: X[t] = src[row(t)] / sqrt(mean(src^2) + eps) * gamma
-// One CTA of 128 threads per row; two passes over the row (the second from L1).
+// One CTA of 128 threads per row; every 16-byte chunk of the row (and of
+// gamma) is loaded up front into registers, so a row costs one round trip.
+// d must be a multiple of 16 bytes' worth of elements and <= 1024 chunks.
 // ---------------------------------------------------------------------------
+constexpr int kNormMaxChunks = 8;  // per thread: d <= 8 * 128 * 8 bf16 (8192) / 4096 f32
+
+template <typename T>
+__device__ __forceinline__ void unpack16(const uint4& u, float* f);
+template <>
+__device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4& u, float* f) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
+    const float2 t = __bfloat1622float2(b);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+template <>
+__device__ __forceinline__ void unpack16<float>(const uint4& u, float* f) {
+  f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+  f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+}
+template <typename T>
+__device__ __forceinline__ uint4 pack16(const float* f);
+template <>
+__device__ __forceinline__ uint4 pack16<__nv_bfloat16>(const float* f) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t*>(&b);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+template <>
+__device__ __forceinline__ uint4 pack16<float>(const float* f) {
+  return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                    __float_as_uint(f[3]));
+}
+
 template <typename T>
 __global__ void __launch_bounds__(128) rmsnorm_rows_kernel(const T* src, int src_is_cache,
                                                            const int32_t* idx, int tps, int N,
                                                            int M, int d, const T* gamma, float eps,
                                                            T* X, int* err) {
+  constexpr int VEC = 16 / sizeof(T);
   const int t = blockIdx.x;
   if (t >= M) return;
   size_t row;
@@ -31,11 +72,27 @@ __global__ void __launch_bounds__(128) rmsnorm_rows_kernel(const T* src, int src
   } else {
     row = (size_t)t;
   }
-  const T* x = src + row * d;
+  const uint4* x = reinterpret_cast<const uint4*>(src + row * d);
+  const uint4* g = reinterpret_cast<const uint4*>(gamma);
+  const int nch = d / VEC;
+  uint4 xv[kNormMaxChunks], gv[kNormMaxChunks];
+#pragma unroll
+  for (int i = 0; i < kNormMaxChunks; ++i) {
+    const int c = threadIdx.x + 128 * i;
+    if (c < nch) {
+      xv[i] = x[c];
+      gv[i] = g[c];
+    }
+  }
   float ss = 0.f;
-  for (int c = threadIdx.x * 4; c < d; c += 128 * 4) {
-    const float4 v = load4(x + c);
-    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+#pragma unroll
+  for (int i = 0; i < kNormMaxChunks; ++i) {
+    if (threadIdx.x + 128 * i < nch) {
+      float f[VEC];
+      unpack16<T>(xv[i], f);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) ss += f[e] * f[e];
+    }
   }
   __shared__ float red[4];
   ss = warp_sum(ss);
@@ -43,11 +100,18 @@ __global__ void __launch_bounds__(128) rmsnorm_rows_kernel(const T* src, int src
   __syncthreads();
   const float tot = (red[0] + red[1]) + (red[2] + red[3]);
   const float inv = 1.0f / sqrtf(tot / (float)d + eps);
-  T* out = X + (size_t)t * d;
-  for (int c = threadIdx.x * 4; c < d; c += 128 * 4) {
-    const float4 v = load4(x + c);
-    const float4 g = load4(gamma + c);
-    store4(out + c, make_float4(v.x * inv * g.x, v.y * inv * g.y, v.z * inv * g.z, v.w * inv * g.w));
+  uint4* out = reinterpret_cast<uint4*>(X + (size_t)t * d);
+#pragma unroll
+  for (int i = 0; i < kNormMaxChunks; ++i) {
+    const int c = threadIdx.x + 128 * i;
+    if (c < nch) {
+      float f[VEC], gg[VEC];
+      unpack16<T>(xv[i], f);
+      unpack16<T>(gv[i], gg);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) f[e] = f[e] * inv * gg[e];
+      out[c] = pack16<T>(f);
+    }
   }
 }
 
@@ -55,6 +119,8 @@ cudaError_t launch_rmsnorm_rows(int dtype, const void* src, int src_is_cache, co
                                 int tps, int N, int M, int d, const void* gamma, float eps, void* X,
                                 int* err, cudaStream_t stream) {
   if (M <= 0) return cudaSuccess;
+  const int vec = dtype == 1 ? 8 : 4;
+  if (d % vec != 0 || d / vec > 128 * kNormMaxChunks) return cudaErrorInvalidValue;
   if (dtype == 1)
     rmsnorm_rows_kernel<__nv_bfloat16><<<M, 128, 0, stream>>>(
         (const __nv_bfloat16*)src, src_is_cache, idx, tps, N, M, d, (const __nv_bfloat16*)gamma,
@@ -75,7 +141,8 @@ cudaError_t launch_rmsnorm_rows(int dtype, const void* src, int src_is_cache, co
 // token is selected if its key is > T, or == T and fewer than `need` equal
 // keys precede it by index (ties to the lowest index).  Block-wide exclusive
 // scans in index order then give each selected token its slot, so the index
-// set comes out ascending.  Finally P^c[I] <- a_hat[I], one warp per row.
+// set comes out ascending.  Finally P^c[I] <- a_hat[I], flattened over
+// (row, column) with several copies per thread in flight.
 // ---------------------------------------------------------------------------
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkPerThread = 8;  // N <= 8192
@@ -127,7 +194,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_select_kernel(const float* 
 #pragma unroll
   for (int j = 0; j < kTopkPerThread; ++j) {
     const int i = i0 + j;
-    key[j] = (j < E && i < N) ? __float_as_uint(fmaxf(s[i], 0.0f)) : 0u;
+    const uint32_t bits = (j < E && i < N) ? __float_as_uint(s[i]) : 0u;
+    key[j] = (bits & 0x80000000u) ? 0u : bits;  // s >= 0; -0 and negatives order as 0
   }
 
   uint32_t prefix = 0, mask = 0;
@@ -136,10 +204,18 @@ __global__ void __launch_bounds__(kTopkThreads) topk_select_kernel(const float* 
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0;
     __syncthreads();
+    // one shared-memory atomic per distinct digit per warp (scores cluster in
+    // a few top-byte values, so per-thread atomics would serialise)
 #pragma unroll
     for (int j = 0; j < kTopkPerThread; ++j) {
       const int i = i0 + j;
-      if (j < E && i < N && (key[j] & mask) == prefix) atomicAdd(&hist[(key[j] >> shift) & 255], 1);
+      const bool act = j < E && i < N && (key[j] & mask) == prefix;
+      const unsigned am = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const unsigned dig = (key[j] >> shift) & 255u;
+        const unsigned peers = __match_any_sync(am, dig);
+        if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[dig], __popc(peers));
+      }
     }
     __syncthreads();
     if (tid < 32) {
@@ -210,10 +286,20 @@ __global__ void __launch_bounds__(kTopkThreads) topk_select_kernel(const float* 
   __syncthreads();
   // P^c[b, I] <- a_hat[b, I]
   if (p_cache != nullptr) {
-    const int lane = tid & 31, wid = tid >> 5;
-    for (int j = wid; j < k; j += kTopkThreads / 32) {
-      const size_t rowoff = ((size_t)b * N + list[j]) * r;
-      for (int c = lane; c < r; c += 32) p_cache[rowoff + c] = a_hat[rowoff + c];
+    // flattened over (selected row, column): 4 independent copies per thread in flight
+    const int total = k * r;
+    for (int base = tid; base < total; base += kTopkThreads * 4) {
+      float v[4];
+      size_t off[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int it = base + u * kTopkThreads;
+        off[u] = it < total ? ((size_t)b * N + list[it / r]) * r + (it % r) : 0;
+        if (it < total) v[u] = a_hat[off[u]];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (base + u * kTopkThreads < total) p_cache[off[u]] = v[u];
     }
   }
 }
