@@ -585,7 +585,7 @@ static int run_proxy(spa_layer* L, const void* H, const spa_layer_cache* c, floa
     p.b_rows_per_src = r;
     p.ep = ep;
     // split count depends on d only, so a row's proxy bits never depend on B or N
-    const int splits = std::max(1, std::min(8, (d / 64) / 4));
+    const int splits = std::max(1, std::min(16, (d / 64) / 4));
     return run_tc(EPI_PROXY, r <= 128 ? 128 : 256, p, M, 1, splits, s, &L->ws->prof, w);
   }
   SimtGemmParams p;

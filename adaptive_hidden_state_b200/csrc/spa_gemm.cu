@@ -117,18 +117,19 @@ __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_e
       store4(reinterpret_cast<T*>(ep.out) + (size_t)t * ep.n_out + f, a);
     }
   } else if constexpr (MODE == EPI_QKV) {
+    constexpr int kUnrollQ = 2;  // four float4 operands per item
     // Item = 4 rotary pairs (j..j+3, j+hd/2..j+hd/2+3) of one head of one row.
     const int hd = ep.head_dim, hh = hd / 2;
     const int items_per_head = hh / 4;
     const int items = (BN / hd) * items_per_head;
     const int gn0 = n_tile * BN;
     const int total = nrows * items;
-    for (int base = tid; base < total; base += nthr * kUnroll) {
-      float4 x1[kUnroll], x2[kUnroll], cs[kUnroll], sn[kUnroll];
-      int row[kUnroll], c1[kUnroll], j[kUnroll];
-      bool ok[kUnroll];
+    for (int base = tid; base < total; base += nthr * kUnrollQ) {
+      float4 x1[kUnrollQ], x2[kUnrollQ], cs[kUnrollQ], sn[kUnrollQ];
+      int row[kUnrollQ], c1[kUnrollQ], j[kUnrollQ];
+      bool ok[kUnrollQ];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < kUnrollQ; ++u) {
         const int it = base + u * nthr;
         row[u] = row_begin + it / items;
         const int w = it % items;
@@ -148,7 +149,7 @@ __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_e
         }
       }
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < kUnrollQ; ++u) {
         if (!ok[u]) continue;
         const int g1 = gn0 + c1[u];
         const int part = g1 / ep.d, col1 = g1 % ep.d, col2 = col1 + hh;
@@ -245,14 +246,18 @@ __device__ void cluster_reduce_rows(float* tile, int ld, int r0, int r1, int S, 
   for (int it = tid; it < (r1 - r0) * C4; it += nthr) {
     const int row = r0 + it / C4, c = (it % C4) * 4;
     const uint32_t local = smem_u32(tile + row * ld + c);
-    float4 v[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      if (q < S) v[q] = ld_dsmem_f4(mapa_shared(local, (uint32_t)q));
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int q = 0; q < 8; ++q)
-      if (q < S) { acc.x += v[q].x; acc.y += v[q].y; acc.z += v[q].z; acc.w += v[q].w; }
+    for (int q0 = 0; q0 < 16; q0 += 8) {  // eight loads in flight, summed in order
+      if (q0 >= S) break;
+      float4 v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (q0 + q < S) v[q] = ld_dsmem_f4(mapa_shared(local, (uint32_t)(q0 + q)));
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (q0 + q < S) { acc.x += v[q].x; acc.y += v[q].y; acc.z += v[q].z; acc.w += v[q].w; }
+    }
     *reinterpret_cast<float4*>(tile + row * ld + c) = acc;
   }
 }
@@ -279,13 +284,13 @@ __device__ __forceinline__ void b_source(const TcGemmParams& p, int n_tile, int 
 constexpr int kTcABytes = 128 * 128;  // 128 rows x 64 bf16
 constexpr int kThreads = 256;         // 8 warps: producer, MMA issuer, all 8 in the epilogue
 
-__host__ __device__ constexpr int tc_stages(int BN) { return BN == 256 ? 4 : 6; }
+__host__ __device__ constexpr int tc_stages(int BN) { return BN == 256 ? 4 : 3; }
 __host__ __device__ constexpr int tc_smem_bytes(int BN) {
   return tc_stages(BN) * (kTcABytes + BN * 128) + 1024;
 }
 
 template <int MODE, int BN>
-__global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
+__global__ void __launch_bounds__(kThreads, BN == 128 ? 2 : 1) tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
   constexpr int STAGES = tc_stages(BN);
   constexpr int B_BYTES = BN * 128;
   constexpr int STAGE_BYTES = kTcABytes + B_BYTES;
@@ -418,6 +423,8 @@ static cudaError_t launch_tc_typed(const TcGemmParams& p, int m_tiles, int n_til
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
     configured = true;
   }
   cudaLaunchConfig_t cfg = {};
@@ -465,9 +472,12 @@ cudaError_t launch_tc_gemm(int mode, int BN, const TcGemmParams& p, int m_tiles,
 // (tile[token][feature]) and reuses run_epilogue.
 // ---------------------------------------------------------------------------
 constexpr int kWsW = 128 * 128;          // one 128-row x 64-column weight tile (bytes)
-constexpr int kWsRing = 200 * 1024;      // bytes of the TMA ring
+constexpr int kWsRing = 104 * 1024;      // bytes of the TMA ring: two CTAs fit on an SM
 constexpr int kWsMaxStages = 8;
 constexpr int kWsSmem = kWsRing + 1024;
+
+// Tokens per epilogue chunk: the fp32 chunk tile [tokens][FEAT + 4] reuses the ring.
+__host__ __device__ constexpr int ws_chunk(int nacc) { return nacc == 1 ? 128 : 64; }
 
 __host__ __device__ inline int ws_stages(int nacc, int NT) {
   const int st = kWsRing / (nacc * kWsW + NT * 128);
@@ -475,11 +485,12 @@ __host__ __device__ inline int ws_stages(int nacc, int NT) {
 }
 
 template <int MODE, int NACC>
-__global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constant__ TcWsParams p) {
+__global__ void __launch_bounds__(kThreads, 2) tc_ws_kernel(const __grid_constant__ TcWsParams p) {
   constexpr int W_BYTES = NACC * kWsW;
   constexpr int FEAT = NACC * 128;
   constexpr int LD = FEAT + 4;
-  static_assert(128 * LD * 4 <= kWsRing, "epilogue tile must fit the ring");
+  constexpr int CHUNK = ws_chunk(NACC);
+  static_assert(CHUNK * LD * 4 <= kWsRing, "epilogue tile must fit the ring");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -500,6 +511,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
   const int KB = p.K / 64;
   const int kb0 = (split * KB) / S, kb1 = ((split + 1) * KB) / S;
   const int nk = kb1 - kb0;
+  // CTAs start their k-loop at staggered blocks so they do not all read the
+  // same token tile at once (the sum order stays fixed per tile)
+  const int rot = nk > 0 ? (n_tile * 5) % nk : 0;
   int* err = p.ep.err;
 
   if (threadIdx.x == 0) {
@@ -529,7 +543,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
       uint8_t* sw = smem + s * STAGE_BYTES;
       uint8_t* sx = sw + W_BYTES;
       mbar_arrive_expect_tx(&full_bar[s], (uint32_t)STAGE_BYTES);
-      const int kx = (kb0 + it) * 64;
+      int kit = it + rot;
+      if (kit >= nk) kit -= nk;
+      const int kx = (kb0 + kit) * 64;
 #pragma unroll
       for (int a = 0; a < NACC; ++a) {
         int src, row;
@@ -578,8 +594,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
   float* tile = reinterpret_cast<float*>(smem);
   const int M = p.ep.M;
   const int q4 = warp & 3, half = warp >> 2;
-  for (int c0 = 0; c0 < NT; c0 += 128) {
-    const int nt = min(128, NT - c0);
+  for (int c0 = 0; c0 < NT; c0 += CHUNK) {
+    const int nt = min(CHUNK, NT - c0);
     if (good) {
       const int f = q4 * 32 + lane;
 #pragma unroll 1
