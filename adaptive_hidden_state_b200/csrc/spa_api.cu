@@ -515,12 +515,31 @@ static int run_tc(int mode, int BN, TcGemmParams& p, int M, int n_tiles, int spl
 }
 
 // Weight-stationary tcgen05 GEMM for M <= 256 tokens: X is the [M, K] bf16
-// token operand (row-major, 16-byte aligned).
-static int run_ws(int mode, int nacc, TcWsParams& p, const void* X, int M, int K, int n_tiles,
+// token operand (row-major, 16-byte aligned); `rows` weight rows (for
+// gate/up: features, each with a W_gate and a W_up row).  Each CTA keeps NACC
+// accumulators of 128 rows so one token tile feeds up to 512 weight rows
+// (NACC * NT <= 512 TMEM columns); NACC is the largest that still leaves at
+// least 16 tiles to spread over the SMs.
+static int run_ws(int mode, bool gateup, TcWsParams& p, const void* X, int M, int K, int rows,
                   cudaStream_t s, Profiler* prof, Work w) {
   if (M <= 0) return SPA_OK;
   if (M > 256) return fail(SPA_ERR_SHAPE, "weight-stationary GEMM takes at most 256 tokens");
   const int NT = ((M + 31) / 32) * 32;
+  const int min_nacc = gateup ? 2 : 1;
+  int nacc = min_nacc;
+  for (int n = 4; n > min_nacc; n /= 2) {
+    const int feat = gateup ? n / 2 * 128 : n * 128;
+    if (n * NT <= 512 && (rows + feat - 1) / feat >= 16) {
+      nacc = n;
+      break;
+    }
+  }
+  if (const char* env = std::getenv("SPA_WS_NACC")) {  // tuning override
+    const int v = std::atoi(env);
+    if ((v == 1 || v == 2 || v == 4) && v >= min_nacc && v * NT <= 512) nacc = v;
+  }
+  const int feat = gateup ? nacc / 2 * 128 : nacc * 128;
+  const int n_tiles = (rows + feat - 1) / feat;
   if (encode_bf16_map_box(&p.tmX, X, (uint64_t)M, (uint64_t)K, (uint32_t)NT))
     return fail(SPA_ERR_CUDA, "tensor map for the token operand failed");
   int cols = 32;
@@ -528,6 +547,7 @@ static int run_ws(int mode, int nacc, TcWsParams& p, const void* X, int M, int K
   p.NT = NT;
   p.tmem_cols = cols;
   p.K = K;
+  if (mode == EPI_ARGMAX) p.ep.n_tiles = n_tiles;
   int splits = plan_ws_splits(mode, nacc, n_tiles, K / 64);
   if (const char* env = std::getenv("SPA_WS_SPLITS")) {  // tuning override, 1..8
     const int v = std::atoi(env);
@@ -627,7 +647,7 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
       std::memset(&p, 0, sizeof(p));
       p.tmW[0] = L->tm_wq; p.tmW[1] = L->tm_wk; p.tmW[2] = L->tm_wv;
       p.b_mode = B_CONCAT3; p.b_rows_per_src = d; p.ep = ep;
-      SPA_TRY(run_ws(EPI_QKV, 1, p, ws->X, M, d, 3 * d / 128, s, prof,
+      SPA_TRY(run_ws(EPI_QKV, false, p, ws->X, M, d, 3 * d, s, prof,
                      Work{SPA_PROF_QKV, 3.0 * d * d * es + Md * es + 3.0 * Md * es, 6.0 * Md * d}));
     } else if (bf) {
       TcGemmParams p;
@@ -665,7 +685,7 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
       TcWsParams p;
       std::memset(&p, 0, sizeof(p));
       p.tmW[0] = L->tm_wo; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
-      SPA_TRY(run_ws(EPI_RESID, 1, p, ws->O, M, d, d / 128, s, prof,
+      SPA_TRY(run_ws(EPI_RESID, false, p, ws->O, M, d, d, s, prof,
                      Work{SPA_PROF_OPROJ, (double)d * d * es + 3.0 * Md * es, 2.0 * Md * d}));
     } else if (bf) {
       TcGemmParams p;
@@ -699,7 +719,7 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
       TcWsParams p;
       std::memset(&p, 0, sizeof(p));
       p.tmW[0] = L->tm_wg; p.tmW[1] = L->tm_wu; p.b_mode = B_GATEUP; p.b_rows_per_src = F; p.ep = ep;
-      SPA_TRY(run_ws(EPI_SWIGLU, 2, p, ws->X2, M, d, F / 128, s, prof,
+      SPA_TRY(run_ws(EPI_SWIGLU, true, p, ws->X2, M, d, F, s, prof,
                      Work{SPA_PROF_GATEUP, 2.0 * F * d * es + Md * es + (double)M * F * es, 4.0 * Md * F}));
     } else if (bf) {
       TcGemmParams p;
@@ -728,7 +748,7 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
       TcWsParams p;
       std::memset(&p, 0, sizeof(p));
       p.tmW[0] = L->tm_wd; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
-      SPA_TRY(run_ws(EPI_RESID_SCATTER, 1, p, ws->A, M, F, d / 128, s, prof,
+      SPA_TRY(run_ws(EPI_RESID_SCATTER, false, p, ws->A, M, F, d, s, prof,
                      Work{SPA_PROF_DOWN, (double)d * F * es + (double)M * F * es + 2.0 * Md * es, 2.0 * Md * F}));
     } else if (bf) {
       TcGemmParams p;
@@ -924,11 +944,11 @@ extern "C" int spa_decode_step(spa_model* m, const int32_t* pos, const int32_t* 
   ep.err = ws->err;
   int tiles = m->lm_tiles;
   if (D.dtype == SPA_BF16 && M <= 256) {
-    ep.n_tiles = tiles;
     TcWsParams p;
     std::memset(&p, 0, sizeof(p));
     p.tmW[0] = m->tm_lm; p.b_mode = B_SINGLE; p.b_rows_per_src = m->desc.vocab; p.ep = ep;
-    SPA_TRY(run_ws(EPI_ARGMAX, 1, p, ws->X, M, d, tiles, s, &ws->prof, wl));
+    SPA_TRY(run_ws(EPI_ARGMAX, false, p, ws->X, M, d, m->desc.vocab, s, &ws->prof, wl));
+    tiles = p.ep.n_tiles;
   } else if (D.dtype == SPA_BF16) {
     tiles = (m->desc.vocab + 255) / 256;
     ep.n_tiles = tiles;

@@ -472,12 +472,15 @@ cudaError_t launch_tc_gemm(int mode, int BN, const TcGemmParams& p, int m_tiles,
 // (tile[token][feature]) and reuses run_epilogue.
 // ---------------------------------------------------------------------------
 constexpr int kWsW = 128 * 128;          // one 128-row x 64-column weight tile (bytes)
-constexpr int kWsRing = 104 * 1024;      // bytes of the TMA ring: two CTAs fit on an SM
+constexpr int kWsRing = 200 * 1024;      // bytes of the TMA ring (one CTA per SM)
 constexpr int kWsMaxStages = 8;
 constexpr int kWsSmem = kWsRing + 1024;
 
 // Tokens per epilogue chunk: the fp32 chunk tile [tokens][FEAT + 4] reuses the ring.
-__host__ __device__ constexpr int ws_chunk(int nacc) { return nacc == 1 ? 128 : 64; }
+__host__ __device__ constexpr int ws_chunk(int nacc) {
+  return (kWsRing / ((nacc * 128 + 4) * 4)) / 32 * 32 < 128 ? (kWsRing / ((nacc * 128 + 4) * 4)) / 32 * 32
+                                                            : 128;
+}
 
 __host__ __device__ inline int ws_stages(int nacc, int NT) {
   const int st = kWsRing / (nacc * kWsW + NT * 128);
@@ -485,7 +488,7 @@ __host__ __device__ inline int ws_stages(int nacc, int NT) {
 }
 
 template <int MODE, int NACC>
-__global__ void __launch_bounds__(kThreads, 2) tc_ws_kernel(const __grid_constant__ TcWsParams p) {
+__global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constant__ TcWsParams p) {
   constexpr int W_BYTES = NACC * kWsW;
   constexpr int FEAT = NACC * 128;
   constexpr int LD = FEAT + 4;
@@ -548,14 +551,21 @@ __global__ void __launch_bounds__(kThreads, 2) tc_ws_kernel(const __grid_constan
       const int kx = (kb0 + kit) * 64;
 #pragma unroll
       for (int a = 0; a < NACC; ++a) {
+        // accumulator a holds weight rows: GATEUP -> the first NACC/2 from
+        // W_gate, the rest the same rows of W_up; otherwise 128 consecutive rows
         int src, row;
         if (p.b_mode == B_GATEUP) {
-          src = a;
-          row = n_tile * 128;
+          const int hal = NACC / 2;
+          src = a < hal ? 0 : 1;
+          row = n_tile * (FEAT / 2) + (a % hal) * 128;
         } else if (p.b_mode == B_CONCAT3) {
-          const int g = n_tile * 128;
+          const int g = n_tile * FEAT + a * 128;
           src = g / p.b_rows_per_src;
           row = g % p.b_rows_per_src;
+          if (src > 2) {  // past the last matrix: a box wholly out of range reads zeros
+            src = 2;
+            row = p.b_rows_per_src;
+          }
         } else {
           src = 0;
           row = n_tile * FEAT + a * 128;
@@ -694,13 +704,13 @@ static int ws_max_clusters(int splits) {
   return cache[splits] > 0 ? cache[splits] : 0;
 }
 
-#define SPA_WS_MODES(X)            \
-  X(EPI_STORE, 1)                  \
-  X(EPI_QKV, 1)                    \
-  X(EPI_RESID, 1)                  \
-  X(EPI_SWIGLU, 2)                 \
-  X(EPI_RESID_SCATTER, 1)          \
-  X(EPI_ARGMAX, 1)
+#define SPA_WS_MODES(X)                                                   \
+  X(EPI_STORE, 1) X(EPI_STORE, 2) X(EPI_STORE, 4)                         \
+  X(EPI_QKV, 1) X(EPI_QKV, 2) X(EPI_QKV, 4)                               \
+  X(EPI_RESID, 1) X(EPI_RESID, 2) X(EPI_RESID, 4)                         \
+  X(EPI_SWIGLU, 2) X(EPI_SWIGLU, 4)                                       \
+  X(EPI_RESID_SCATTER, 1) X(EPI_RESID_SCATTER, 2) X(EPI_RESID_SCATTER, 4) \
+  X(EPI_ARGMAX, 1) X(EPI_ARGMAX, 2) X(EPI_ARGMAX, 4)
 
 cudaError_t launch_tc_ws(int mode, int nacc, const TcWsParams& p, int n_tiles, int splits,
                          cudaStream_t stream) {

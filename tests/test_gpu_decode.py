@@ -100,3 +100,59 @@ def test_tiny_decode_full_k_matches_vanilla():
         spa.spa_decode_step(model, pos, forced, u, 2, tok_out)
         assert_close(caches[-1].h, np64(out_cached[t]), False, f"vanilla step {t}")
     lps[0].ws.check()
+
+
+SMALL_BF16 = synth.LayerShape(d=256, n_heads=2, head_dim=128, ffn=384, r=16)
+
+
+def test_bf16_decode_loop_and_graph_replay():
+    """bf16 model (2 layers of d=256, vocab 8192 so the LM head uses wide
+    weight tiles): teacher-forced steps against the oracle, then the same
+    steps replayed from a captured CUDA graph must reproduce the directly
+    launched steps bit for bit."""
+    B, N, vocab, steps, u = 2, 96, 8192, 4, 2
+    model, om, lps, caches, h0, keep = _tiny_model(spa.SPA_BF16, SMALL_BF16, 2, vocab, B, N,
+                                                   0.3, seed=50)
+    job = synth.decode_inputs(B=B, N=N, n_prompt=32, vocab=vocab, steps=steps, u=u, seed=51)
+    toks = torch.from_numpy(job.tokens.astype(np.int32)).cuda()
+    model.embed_tokens(toks)
+    state = O.init_decode_state(om, job.tokens)
+    tok_out = torch.empty((steps, B, u), dtype=torch.int32, device="cuda")
+    direct_h = []
+    for t in range(steps):
+        pos = torch.from_numpy(job.positions[t].astype(np.int32)).cuda()
+        forced = torch.from_numpy(job.forced[t].astype(np.int32)).cuda()
+        spa.spa_decode_step(model, pos, forced, u, 1 if t == 0 else 0, tok_out[t])
+        lps[0].ws.check()
+        ref = O.decode_step(om, state, job.positions[t], model.k, full=(t == 0),
+                            forced=job.forced[t])
+        got = tok_out[t].cpu().numpy()
+        lg = ref["logits"]
+        for b in range(B):
+            for j in range(u):
+                top2 = np.sort(lg[b, j])[-2:]
+                if top2[1] - top2[0] > 2e-2 * max(1.0, abs(top2[1])):
+                    assert got[b, j] == ref["argmax"][b, j]
+        for l in range(2):
+            assert_close(caches[l].h, np.stack([state.caches[l][b].H_c for b in range(B)]), True,
+                         f"bf16 step {t} layer {l} H^c")
+        direct_h.append(caches[-1].h.clone())
+    # replay steps 1.. from a captured graph after redoing step 0 directly
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        pos_buf = torch.empty((B, u), dtype=torch.int32, device="cuda")
+        tin_buf = torch.empty((B, u), dtype=torch.int32, device="cuda")
+        tout_buf = torch.empty((B, u), dtype=torch.int32, device="cuda")
+        model.embed_tokens(toks)
+        pos0 = torch.from_numpy(job.positions[0].astype(np.int32)).cuda()
+        f0 = torch.from_numpy(job.forced[0].astype(np.int32)).cuda()
+        spa.spa_decode_step(model, pos0, f0, u, 1, tout_buf)
+        spa.spa_decode_graph_capture(model, pos_buf, tin_buf, u, tout_buf)
+        for t in range(1, steps):
+            pos_buf.copy_(torch.from_numpy(job.positions[t].astype(np.int32)).cuda())
+            tin_buf.copy_(torch.from_numpy(job.forced[t].astype(np.int32)).cuda())
+            spa.spa_decode_graph_launch(model)
+            assert torch.equal(caches[-1].h, direct_h[t])
+            assert torch.equal(tout_buf, tok_out[t])
+    stream.synchronize()
+    lps[0].ws.check()

@@ -117,6 +117,19 @@ def test_bf16_small_layer_shapes(B, N, k):
     _step(lp, cache, ocs, H2, k)
 
 
+@pytest.mark.parametrize("nacc", ["2", "4"])
+@pytest.mark.parametrize("B,N,k", [(1, 200, 96), (2, 160, 33)])
+def test_bf16_wide_weight_tiles(monkeypatch, nacc, B, N, k):
+    # more weight rows per CTA than the planner would pick at this width,
+    # including tiles that run past the last weight matrix
+    monkeypatch.setenv("SPA_WS_NACC", nacc)
+    lp = LayerPair(spa, SMALL_BF16, seed=40 + k, dtype=spa.SPA_BF16, max_B=2, max_N=200, std=0.05)
+    H = synth.hidden_states(B, N, 256, seed=k, bf16=True)
+    cache, ocs = _run_fill(lp, H)
+    H2, _ = synth.drift_rows(H, 0.2, 0.5, seed=k + 1, bf16=True)
+    _step(lp, cache, ocs, H2, k)
+
+
 def test_bf16_zero_drift_selects_lowest_indices():
     lp = LayerPair(spa, SMALL_BF16, seed=21, dtype=spa.SPA_BF16, max_B=1, max_N=200, std=0.05)
     H = synth.hidden_states(1, 200, 256, seed=22, bf16=True)
