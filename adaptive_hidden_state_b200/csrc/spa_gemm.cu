@@ -32,7 +32,9 @@ namespace spa {
 // ---------------------------------------------------------------------------
 constexpr int kUnroll = 4;
 
-__device__ __forceinline__ float silu(float g) { return g / (1.0f + expf(-g)); }
+// silu(g) = g / (1 + e^-g) with the fast exponential and reciprocal
+// intrinsics: relative error ~1e-6, far below the bf16 rounding of the result.
+__device__ __forceinline__ float silu(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
 
 // s_rows[row] = (sequence b, cache row) of token t = gm0 + row; (0, -1) when
 // t >= M or the index is out of range (the latter is reported).
