@@ -125,6 +125,8 @@ extern "C" const char* spa_status_string(int status) {
 }
 
 extern "C" const char* spa_last_error(void) { return g_last_error; }
+
+int spa::set_last_error(int status, const char* msg) { return fail(status, "%s", msg); }
 extern "C" int spa_version(void) { return 100; }
 
 // ---------------------------------------------------------------------------

@@ -105,6 +105,10 @@ cudaError_t launch_simt_gemm(int mode, const SimtGemmParams& p, int m_tiles, int
 // Encodes a 2D bf16 tensor map (rows x cols, row-major) with a 64 x 128 box.
 int encode_bf16_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols);
 
+// Records `msg` as this host thread's last error (read by spa_last_error)
+// and returns `status`.
+int set_last_error(int status, const char* msg);
+
 // ---- small kernels (spa_kernels.cu) ----
 // X[t] = RMSNorm(src[row(t)]) * gamma, row(t) = b * N + (idx ? idx[t] : t % tps) when
 // src_is_cache, else t.

@@ -35,6 +35,7 @@ EXPORTS = [
     "spa_proxy_select", "spa_partial_block", "spa_layer_step", "spa_full_block",
     "spa_model_create", "spa_model_free", "spa_model_layer_k", "spa_model_embed",
     "spa_decode_step", "spa_decode_graph_capture", "spa_decode_graph_launch",
+    "spa_attention_noalloc",
 ]
 
 
@@ -116,6 +117,8 @@ _sig("spa_model_embed", c_int, c_void_p, c_void_p, c_void_p)
 _sig("spa_decode_step", c_int, c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p)
 _sig("spa_decode_graph_capture", c_int, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p)
 _sig("spa_decode_graph_launch", c_int, c_void_p, c_void_p)
+_sig("spa_attention_noalloc", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
+     c_int, c_int, c_void_p)
 
 
 def _check(status: int, where: str):
@@ -340,3 +343,11 @@ def spa_decode_graph_capture(model: Model, pos, tok_in, u: int, tok_out, stream=
 
 def spa_decode_graph_launch(model: Model, stream=None):
     _check(lib.spa_decode_graph_launch(model.handle, _stream(stream)), "spa_decode_graph_launch")
+
+
+def spa_attention_noalloc(Q, k_cache, v_cache, O, B: int, k: int, N: int, n_heads: int,
+                          head_dim: int, stream=None):
+    """Attention of the selected queries against the whole cache, with the
+    library's fixed scratch instead of allocated memory (see include/spa.h)."""
+    _check(lib.spa_attention_noalloc(_ptr(Q), _ptr(k_cache), _ptr(v_cache), _ptr(O), B, k, N,
+                                     n_heads, head_dim, _stream(stream)), "spa_attention_noalloc")

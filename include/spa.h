@@ -239,6 +239,31 @@ int spa_decode_graph_capture(spa_model *model, const int32_t *pos, const int32_t
                              int32_t *tok_out, void *stream);
 int spa_decode_graph_launch(spa_model *model, void *stream);
 
+/* ------------------------------------------------- allocation-free variant --
+ * No counterpart on the pages: an engineering addition for callers that may
+ * not allocate device memory (custom memory managers and allocator hooks that
+ * must not re-enter the CUDA allocator, hosts that give the library a fixed
+ * memory budget up front, loops where an allocation's implicit device
+ * synchronisation is not allowed).
+ *
+ * The sparse-query attention of spa_partial_block on its own, bf16, head_dim
+ * 128: O = softmax(Q K^cT / sqrt(head_dim)) V^c per head over all N cached
+ * rows.  Q [B, k, n_heads * 128] (the compact selected queries, post-RoPE),
+ * k_cache, v_cache [B, N, n_heads * 128], O [B, k, n_heads * 128]: device,
+ * bf16, row-major, caller-owned.  It allocates nothing: the split-over-keys
+ * partials live in one fixed 8 MiB array inside the library (held on every
+ * GPU that loads it until the process exits), so B * k * (n_heads * 130)
+ * fp32 values must fit in 2 Mi floats; larger calls return SPA_ERR_SHAPE and
+ * launch nothing.  The first call on each device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.  Every call on a device shares the array:
+ * calls whose work overlaps on the GPU (other streams, other host threads)
+ * race, so order them on one stream.  Errors: SPA_ERR_INVALID (null
+ * pointer), SPA_ERR_SHAPE, SPA_ERR_UNSUPPORTED (head_dim != 128),
+ * SPA_ERR_CUDA; details in spa_last_error(). */
+int spa_attention_noalloc(const void *Q, const void *k_cache, const void *v_cache, void *O, int B,
+                          int k, int N, int n_heads, int head_dim, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
