@@ -185,6 +185,8 @@ struct spa_workspace {
   float* part_o = nullptr;  // attention split partials
   float* part_ml = nullptr;
   int part_rows = 0;
+  int* attn_sync = nullptr;  // per query tile: attention key splits finished
+  int attn_sync_len = 0;
   int* err = nullptr;       // [2]
   float* rope_cos = nullptr;  // [max_N, hd/2]
   float* rope_sin = nullptr;
@@ -293,6 +295,8 @@ extern "C" int spa_workspace_create(const spa_layer_desc* desc, int max_B, int m
   WS_ALLOC(A, cap * F * e)
   WS_ALLOC(part_o, (size_t)ws->part_rows * d * 4)
   WS_ALLOC(part_ml, (size_t)ws->part_rows * desc->n_heads * 2 * 4)
+  ws->attn_sync_len = max_B * desc->n_heads * ((max_N + 127) / 128);
+  WS_ALLOC(attn_sync, (size_t)ws->attn_sync_len * sizeof(int))
   WS_ALLOC(err, 2 * sizeof(int))
   WS_ALLOC(rope_cos, (size_t)max_N * (desc->head_dim / 2) * 4)
   WS_ALLOC(rope_sin, (size_t)max_N * (desc->head_dim / 2) * 4)
@@ -313,7 +317,8 @@ extern "C" int spa_workspace_create(const spa_layer_desc* desc, int max_B, int m
     }
   if (cudaMemcpy(ws->rope_cos, cs.data(), cs.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
       cudaMemcpy(ws->rope_sin, sn.data(), sn.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
-      cudaMemset(ws->err, 0, 2 * sizeof(int)) != cudaSuccess) {
+      cudaMemset(ws->err, 0, 2 * sizeof(int)) != cudaSuccess ||
+      cudaMemset(ws->attn_sync, 0, (size_t)ws->attn_sync_len * sizeof(int)) != cudaSuccess) {
     spa_workspace_free(ws);
     return fail(SPA_ERR_CUDA, "workspace initialisation copy failed");
   }
@@ -674,7 +679,8 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
   {
     ProfScope ps(prof, SPA_PROF_ATTN, 2.0 * Md * es + 2.0 * Bn * d * es, 4.0 * Md * N, s);
     e = launch_attention(D.dtype, ws->Q, c->k_cache, c->v_cache, ws->O, c->B, tps, N, D.n_heads,
-                         D.head_dim, ws->part_o, ws->part_ml, ws->part_rows, ws->err, s);
+                         D.head_dim, ws->part_o, ws->part_ml, ws->part_rows, ws->attn_sync,
+                         ws->attn_sync_len, ws->err, s);
   }
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
   // H1 = H[I] + O W_o^T

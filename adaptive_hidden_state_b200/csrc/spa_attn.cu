@@ -2,17 +2,14 @@
 // queries of each sequence attend to all N cached keys and values (the
 // bidirectional cache K^c, V^c, already holding this step's fresh rows).
 //
-// attn_mma_kernel (bf16, head_dim 128): flash-style, 64 queries x 1 head per
-// CTA (16 per warp), key/value tiles of 64 rows double-buffered in shared
-// memory with cp.async, S = Q K^T and O += P V on the tensor cores
-// (mma.sync m16n8k16, fp32 accumulate), online softmax in fp32 registers.
-// Keys are split across CTAs when the grid would not fill the GPU; each split
-// writes (O_s / l_s, m_s, l_s) and attn_combine_kernel merges them in a fixed
-// order.
+// attn_tc_kernel (bf16, head_dim 128): tcgen05 tensor cores with TMEM
+// accumulators, described below.
 //
 // attn_simt_kernel: one warp per (query, head), online softmax over chunks of
 // 32 keys (one key per lane), fp32 throughout.  Used for the fp32
 // configurations and for head sizes the tensor-core kernel does not cover.
+#include <cstring>
+
 #include "spa_device.cuh"
 #include "spa_internal.h"
 
@@ -23,6 +20,8 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(const T* Q, const T* Kc,
                                                         int k, int N, int n_heads, int hd,
                                                         float scale) {
   __shared__ float qs[4][128];
+  griddep_launch_dependents();
+  griddep_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int i = blockIdx.x * 4 + warp;  // query within the sequence
   const int h = blockIdx.y, b = blockIdx.z;
@@ -71,293 +70,439 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(const T* Q, const T* Kc,
 }
 
 // ---------------------------------------------------------------------------
-// tensor-core attention, head_dim = 128
+// tensor-core attention (tcgen05, TMEM), bf16, head_dim 128
+//
+// One CTA = one head of one sequence, one tile of 128 selected queries, one
+// contiguous range of the N cached keys (split-KV).  Q (128 x 128) is loaded
+// once; K and V tiles of 128 keys stream through a 2-stage TMA ring.
+//   warp 0      TMA producer
+//   warp 1      one thread issues tcgen05.mma: S_j = Q K_j^T into one of two
+//               TMEM score buffers, then O += P_{j-1} V_{j-1} (P from shared
+//               memory, V as an MN-major operand), so the tensor core works on
+//               the next scores while the softmax warps work on these
+//   warps 4-7   softmax: thread i owns query row i (TMEM lane i).  It reads
+//               its 128 scores, keeps the running max m and sum l in
+//               registers, writes P = 2^(s*log2e/sqrt(d_h) - m) as bf16 into
+//               the 128-byte-swizzled K-major layout the MMA reads, and
+//               rescales O in TMEM only when the max grows by more than 2^8
+//               (the result is exact for any reference max: the final
+//               division by l uses the same one).
+// With several key splits each CTA writes (O, m, l) to scratch; the last CTA
+// of the query tile to finish (an atomic counter) combines them in split
+// order 0..S-1, so the result does not depend on timing, and resets the
+// counter.
 // ---------------------------------------------------------------------------
-constexpr int kBQ = 64, kBK = 64, kHD = 128;
+constexpr int kAT = 128;                 // queries per CTA and keys per tile
+constexpr int kAQBytes = 2 * 16384;      // Q: two 64-column boxes of 128 rows
+constexpr int kAKVBytes = 4 * 16384;     // K and V tiles, two boxes each
+constexpr int kAPBytes = 2 * 16384;      // P: 128 x 128 bf16
+constexpr int kAStages = 2;
+constexpr int kASmem = kAQBytes + kAStages * kAKVBytes + kAPBytes + 1024;
+constexpr int kAThreads = 256;
+constexpr float kARescale = 8.0f;        // rescale O when the max grows by > 2^8
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(valid ? 16 : 0)
-               : "memory");
+struct alignas(64) AttnTcParams {
+  CUtensorMap tmQ;  // compact Q [B*k, d], box 64 x 128
+  CUtensorMap tmK;  // K^c [B*N, d], box 64 x 128
+  CUtensorMap tmV;  // V^c [B*N, d], box 64 x 128
+  __nv_bfloat16* O; // [B*k, d]
+  float* part_o;    // split partials: slot -> [128][128] fp32
+  float* part_ml;   // slot -> m[128], l[128]
+  int* sync;        // per query tile: splits finished (zero between launches)
+  int* err;
+  int B, k, N, n_heads, q_tiles, splits;
+  float scale_log2;  // log2(e) / sqrt(head_dim)
+};
+
+// Shared-memory descriptor of an MN-major operand tile with 128-byte
+// swizzling: 64 contiguous MN elements (128 B) per K row, 8-row atoms of
+// 1024 B (stride byte offset), the next 64 MN elements `lbo` bytes further
+// (leading byte offset).
+__device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr, uint32_t lbo) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)64 << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                        uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                          uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
-      "{%8, %9}, {%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
 }
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
+// 128 consecutive TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float (&v)[128]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) tmem_ld32(taddr + (uint32_t)(32 * q), *reinterpret_cast<float(*)[32]>(&v[32 * q]));
 }
-
-// Byte offset of 16-byte chunk c of row `row` in a [rows][128] bf16 tile whose
-// chunks are XOR-swizzled by (row & 7) so ldmatrix reads are conflict-free.
-__device__ __forceinline__ uint32_t swz(int row, int c) {
-  return (uint32_t)(row * 256 + ((c ^ (row & 7)) << 4));
-}
-
-// Loads rows [row0, row0 + 64) (head h) of a [., n_rows, d] bf16 matrix into a
-// swizzled 64 x 128 tile; rows >= n_rows are zero-filled.
-__device__ __forceinline__ void load_tile64(uint32_t sbase, const __nv_bfloat16* g, int row0,
-                                            int n_rows, int d, int tid) {
-#pragma unroll
-  for (int i = 0; i < (kBK * 16) / 128; ++i) {
-    const int id = tid + i * 128;
-    const int row = id >> 4, c = id & 15;
-    const int gr = row0 + row;
-    const bool ok = gr < n_rows;
-    const __nv_bfloat16* src = g + (size_t)(ok ? gr : 0) * d + c * 8;
-    cp_async16(sbase + swz(row, c), src, ok);
-  }
-}
-
-__global__ void __launch_bounds__(128) attn_mma_kernel(const __nv_bfloat16* __restrict__ Q,
-                                                       const __nv_bfloat16* __restrict__ Kc,
-                                                       const __nv_bfloat16* __restrict__ Vc,
-                                                       __nv_bfloat16* __restrict__ O, float* part_o,
-                                                       float* part_ml, int k, int N, int n_heads,
-                                                       int splits, float scale_log2) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const uint32_t sQ = smem_u32(smem);
-  const uint32_t sK0 = sQ + kBQ * 256;
-  const uint32_t sV0 = sK0 + 2 * kBK * 256;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qt = blockIdx.x, h = blockIdx.y;
-  const int b = blockIdx.z / splits, split = blockIdx.z % splits;
-  const int d = n_heads * kHD;
-  const int n_kt = (N + kBK - 1) / kBK;
-  const int kt0 = (split * n_kt) / splits, kt1 = ((split + 1) * n_kt) / splits;
-
-  const __nv_bfloat16* Qg = Q + ((size_t)b * k) * d + (size_t)h * kHD;
-  const __nv_bfloat16* Kg = Kc + ((size_t)b * N) * d + (size_t)h * kHD;
-  const __nv_bfloat16* Vg = Vc + ((size_t)b * N) * d + (size_t)h * kHD;
-
-  load_tile64(sQ, Qg, qt * kBQ, k, d, tid);
-  if (kt0 < kt1) {
-    load_tile64(sK0, Kg, kt0 * kBK, N, d, tid);
-    load_tile64(sV0, Vg, kt0 * kBK, N, d, tid);
-  }
-  cp_async_commit();
-
-  float o[16][4];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
-  uint32_t qf[8][4];
-
-  for (int kt = kt0; kt < kt1; ++kt) {
-    const int stage = (kt - kt0) & 1;
-    if (kt + 1 < kt1) {
-      const int ns = stage ^ 1;
-      load_tile64(sK0 + ns * kBK * 256, Kg, (kt + 1) * kBK, N, d, tid);
-      load_tile64(sV0 + ns * kBK * 256, Vg, (kt + 1) * kBK, N, d, tid);
-    }
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    if (kt == kt0) {
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const int row = warp * 16 + (lane & 15), c = 2 * kk + (lane >> 4);
-        ldsm_x4(sQ + swz(row, c), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
-      }
-    }
-    const uint32_t sK = sK0 + stage * kBK * 256, sV = sV0 + stage * kBK * 256;
-    // S = Q K^T  (16 x 64 per warp)
-    float s[8][4];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-      for (int j = 0; j < 8; j += 2) {
-        const int key = j * 8 + ((lane >> 4) << 3) + (lane & 7);
-        const int c = 2 * kk + ((lane >> 3) & 1);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(sK + swz(key, c), b0, b1, b2, b3);
-        mma_bf16(s[j], qf[kk], b0, b1);
-        mma_bf16(s[j + 1], qf[kk], b2, b3);
-      }
-    }
-    // scale, mask keys >= N, online softmax (rows lane/4 and lane/4 + 8)
-    const int key_base = kt * kBK + 2 * (lane & 3);
-    float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = key_base + j * 8 + (e & 1);
-        float v = s[j][e] * scale_log2;
-        if (key >= N) v = -INFINITY;
-        s[j][e] = v;
-        mx[e >> 1] = fmaxf(mx[e >> 1], v);
-      }
-    }
-    float corr[2];
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 1));
-      mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 2));
-      const float mn = fmaxf(m_r[rr], mx[rr]);
-      corr[rr] = exp2f(m_r[rr] - mn);
-      m_r[rr] = mn;
-    }
-    float rs[2] = {0.f, 0.f};
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float p = exp2f(s[j][e] - m_r[e >> 1]);
-        s[j][e] = p;
-        rs[e >> 1] += p;
-      }
-    }
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      rs[rr] += __shfl_xor_sync(0xffffffffu, rs[rr], 1);
-      rs[rr] += __shfl_xor_sync(0xffffffffu, rs[rr], 2);
-      l_r[rr] = l_r[rr] * corr[rr] + rs[rr];
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      o[i][0] *= corr[0]; o[i][1] *= corr[0];
-      o[i][2] *= corr[1]; o[i][3] *= corr[1];
-    }
-    // O += P V
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t pa[4];
-      pa[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-      pa[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-      pa[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-      pa[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
-#pragma unroll
-      for (int c = 0; c < 16; c += 2) {
-        const int key = kk * 16 + (((lane >> 3) & 1) << 3) + (lane & 7);
-        const int ch = c + (lane >> 4);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(sV + swz(key, ch), b0, b1, b2, b3);
-        mma_bf16(o[c], pa, b0, b1);
-        mma_bf16(o[c + 1], pa, b2, b3);
-      }
-    }
-    __syncthreads();
-  }
-  cp_async_wait<0>();
-
-  // write: rows r = lane/4 (+8) of this warp's 16 queries
-#pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const int qi = qt * kBQ + warp * 16 + (lane >> 2) + rr * 8;
-    if (qi >= k) continue;
-    const float inv = l_r[rr] > 0.f ? 1.0f / l_r[rr] : 0.f;
-    const size_t t = (size_t)b * k + qi;
-    if (splits == 1) {
-      __nv_bfloat16* dst = O + t * d + (size_t)h * kHD + 2 * (lane & 3);
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        *reinterpret_cast<uint32_t*>(dst + c * 8) =
-            pack_bf16(o[c][2 * rr] * inv, o[c][2 * rr + 1] * inv);
-      }
-    } else {
-      const size_t rows = gridDim.z / splits * (size_t)k;  // B * k
-      float* dst = part_o + ((size_t)split * rows + t) * d + (size_t)h * kHD + 2 * (lane & 3);
-#pragma unroll
-      for (int c = 0; c < 16; ++c)
-        *reinterpret_cast<float2*>(dst + c * 8) = make_float2(o[c][2 * rr] * inv, o[c][2 * rr + 1] * inv);
-      if ((lane & 3) == 0) {
-        float* ml = part_ml + (((size_t)split * rows + t) * n_heads + h) * 2;
-        ml[0] = m_r[rr];
-        ml[1] = l_r[rr];
-      }
+// Bounded wait that ignores the abort flag (copies/MMAs in flight after an abort).
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, int* err, int site) {
+  const uint32_t a = smem_u32(bar);
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      report_error(err, DEVERR_TIMEOUT, site);
+      return;
     }
   }
 }
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive1(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void named_bar(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 
-// O[t, h] = sum_s w_s O_s / sum_s w_s with w_s = l_s 2^(m_s - max m), in order s = 0..S-1.
-__global__ void attn_combine_kernel(const float* part_o, const float* part_ml,
-                                    __nv_bfloat16* O, int rows, int n_heads, int splits) {
-  const int t = blockIdx.x, h = blockIdx.y, c = threadIdx.x;  // 128 threads = head_dim
-  const int d = n_heads * kHD;
-  float mmax = -INFINITY;
-  for (int s = 0; s < splits; ++s)
-    mmax = fmaxf(mmax, part_ml[(((size_t)s * rows + t) * n_heads + h) * 2]);
-  float num = 0.f, den = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float* ml = part_ml + (((size_t)s * rows + t) * n_heads + h) * 2;
-    const float w = ml[1] * exp2f(ml[0] - mmax);
-    num += w * part_o[((size_t)s * rows + t) * d + (size_t)h * kHD + c];
-    den += w;
+__global__ void __launch_bounds__(kAThreads, 1) attn_tc_kernel(const __grid_constant__ AttnTcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = sQ + kAQBytes;
+  uint8_t* sP = sKV + kAStages * kAKVBytes;
+  __shared__ __align__(8) uint64_t q_full, kv_full[kAStages], kv_empty[kAStages];
+  __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full, pv_done, o_done;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag, last_flag;
+  __shared__ int kv_issued, kv_consumed, tile_ok;
+
+  griddep_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = p.splits;
+  const int qt = blockIdx.x / S, sp = blockIdx.x % S, h = blockIdx.y, b = blockIdx.z;
+  const int n_kt = (p.N + kAT - 1) / kAT;
+  const int kt0 = (sp * n_kt) / S, kt1 = ((sp + 1) * n_kt) / S;
+  const int nkt = kt1 - kt0;
+  int* err = p.err;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&q_full, 1);
+    for (int s = 0; s < kAStages; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_empty[s], 128);
+    }
+    mbar_init(&p_full, 128);
+    mbar_init(&pv_done, 1);
+    mbar_init(&o_done, 1);
+    abort_flag = 0;
+    last_flag = 0;
+    kv_issued = kv_consumed = 0;
+    tile_ok = 1;
+    fence_mbar_init();
   }
-  O[(size_t)t * d + (size_t)h * kHD + c] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;  // S buffers at columns 0 and 128, O at 256
+  griddep_wait();  // Q, K^c and V^c come from the previous kernel
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tmK);
+    tma_prefetch_desc(&p.tmV);
+    const int qrow = b * p.k + qt * kAT, col = h * kAT;
+    mbar_arrive_expect_tx(&q_full, kAQBytes);
+    tma_load_2d(sQ, &p.tmQ, &q_full, col, qrow);
+    tma_load_2d(sQ + 16384, &p.tmQ, &q_full, col + 64, qrow);
+    for (int j = 0; j < nkt; ++j) {
+      const int s = j % kAStages;
+      if (j >= kAStages && !mbar_wait(&kv_empty[s], ((j / kAStages) - 1) & 1, &abort_flag, err, 601)) break;
+      uint8_t* kv = sKV + s * kAKVBytes;
+      const int krow = b * p.N + (kt0 + j) * kAT;
+      mbar_arrive_expect_tx(&kv_full[s], kAKVBytes);
+      tma_load_2d(kv, &p.tmK, &kv_full[s], col, krow);
+      tma_load_2d(kv + 16384, &p.tmK, &kv_full[s], col + 64, krow);
+      tma_load_2d(kv + 32768, &p.tmV, &kv_full[s], col, krow);
+      tma_load_2d(kv + 49152, &p.tmV, &kv_full[s], col + 64, krow);
+      kv_issued = j + 1;
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128);                 // both K-major
+    constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128) | (1u << 16);    // B (V) MN-major
+    const uint64_t dq = smem_desc_sw128(smem_u32(sQ));
+    const uint64_t dp = smem_desc_sw128(smem_u32(sP));
+    bool ok = mbar_wait(&q_full, 0, &abort_flag, err, 602);
+    for (int j = 0; ok && j <= nkt; ++j) {
+      if (j < nkt) {
+        // S_j = Q K_j^T into score buffer j % 2
+        const int s = j % kAStages, sb = j & 1;
+        if (!mbar_wait(&kv_full[s], (j / kAStages) & 1, &abort_flag, err, 603)) break;
+        kv_consumed = j + 1;
+        if (j >= 2 && !mbar_wait(&s_empty[sb], ((j / 2) - 1) & 1, &abort_flag, err, 604)) break;
+        tc_fence_after();
+        const uint64_t dk = smem_desc_sw128(smem_u32(sKV + s * kAKVBytes));
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t off = (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2);
+          umma_bf16(tmem + (uint32_t)(sb * 128), dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[sb]);
+      }
+      if (j >= 1) {
+        // O += P_{j-1} V_{j-1}
+        const int jj = j - 1, s = jj % kAStages;
+        if (!mbar_wait(&p_full, jj & 1, &abort_flag, err, 605)) break;
+        tc_fence_after();
+        const uint64_t dv = smem_desc_sw128_mn(smem_u32(sKV + s * kAKVBytes + 32768), 16384);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t offp = (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2);
+          umma_bf16(tmem + 256u, dp + offp, dv + (uint64_t)(kk * 128), idesc_pv,
+                    (jj > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&pv_done);
+        umma_commit(&kv_empty[s]);
+      }
+    }
+    umma_commit(&o_done);
+  } else if (warp >= 4) {
+    const int q4 = warp - 4, row = q4 * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(q4 * 32) << 16);
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkt; ++j) {
+      const int sb = j & 1;
+      // every lane waits, then the warp reconverges before the warp-wide
+      // (.sync.aligned) TMEM instructions
+      const bool got = mbar_wait(&s_full[sb], (j / 2) & 1, &abort_flag, err, 606);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      tc_fence_after();
+      float x[128];
+      tmem_ld128(lane_base + (uint32_t)(sb * 128), x);
+      tc_fence_before();
+      mbar_arrive1(&s_empty[sb]);
+      const int key0 = (kt0 + j) * kAT;
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        x[c] = (key0 + c < p.N) ? x[c] * p.scale_log2 : -INFINITY;
+        tmax = fmaxf(tmax, x[c]);
+      }
+      // O and P may be rewritten only once the previous PV product is done
+      const bool pv_ok = j == 0 || mbar_wait(&pv_done, (j - 1) & 1, &abort_flag, err, 607);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, pv_ok)) { ok = false; break; }
+      if (j == 0) {
+        m_used = tmax;
+      } else if (__any_sync(0xffffffffu, tmax > m_used + kARescale)) {
+        // some row's max grew by more than 2^8: the whole warp rescales (the
+        // TMEM instructions are warp-wide), each row to its own new max
+        const float m_new = fmaxf(m_used, tmax);
+        const float f = exp2f(m_used - m_new);
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          float o[32];
+          tmem_ld32(lane_base + 256u + (uint32_t)c, o);
+#pragma unroll
+          for (int q = 0; q < 32; ++q) o[q] *= f;
+          tmem_st32(lane_base + 256u + (uint32_t)c, o);
+        }
+        tmem_st_wait();
+        l *= f;
+        m_used = m_new;
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 128; c += 8) {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float a = exp2f(x[c + 2 * q] - m_used), bb = exp2f(x[c + 2 * q + 1] - m_used);
+          sum += a + bb;
+          __nv_bfloat162 v2 = __floats2bfloat162_rn(a, bb);
+          w[q] = *reinterpret_cast<uint32_t*>(&v2);
+        }
+        // 16-byte chunk c/8 of row `row`, 128-byte swizzle, two 64-key halves
+        const int chunk = c >> 3, half = chunk >> 3, cc = chunk & 7;
+        uint8_t* dst = sP + half * 16384 + row * 128 + ((cc ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      l += sum;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive1(&p_full);
+    }
+    // final O row
+    const bool fin = ok && mbar_wait(&o_done, 0, &abort_flag, err, 608);
+    __syncwarp();
+    const bool warp_ok = __all_sync(0xffffffffu, fin);
+    // the four softmax warps agree on whether the tile is usable, so the
+    // named barriers below are reached by all 128 threads or by none
+    if (lane == 0) atomicAnd(&tile_ok, warp_ok ? 1 : 0);
+    named_bar(1, 128);
+    if (tile_ok) {
+      tc_fence_after();
+      const int d = p.n_heads * kAT;
+      const int qi = qt * kAT + row;  // query within the sequence
+      if (S == 1) {
+        const float inv = l > 0.f ? 1.0f / l : 0.f;
+        __nv_bfloat16* dst = p.O + ((size_t)b * p.k + qi) * d + (size_t)h * kAT;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          float o[32];
+          tmem_ld32(lane_base + 256u + (uint32_t)c0, o);
+          if (qi < p.k) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 8) {
+              uint32_t w[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                __nv_bfloat162 v2 = __floats2bfloat162_rn(o[c + 2 * q] * inv, o[c + 2 * q + 1] * inv);
+                w[q] = *reinterpret_cast<uint32_t*>(&v2);
+              }
+              *reinterpret_cast<uint4*>(dst + c0 + c) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
+        }
+      } else {
+        const size_t grp = ((size_t)b * p.n_heads + h) * p.q_tiles + qt;
+        const size_t slot = grp * S + sp;
+        float* po = p.part_o + slot * (kAT * kAT) + (size_t)row * kAT;
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          float o[32];
+          tmem_ld32(lane_base + 256u + (uint32_t)c0, o);
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            *reinterpret_cast<float4*>(po + c0 + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+        }
+        p.part_ml[slot * 256 + row] = m_used;
+        p.part_ml[slot * 256 + 128 + row] = l;
+        __threadfence();
+        named_bar(1, 128);
+        if (row == 0) last_flag = (atomicAdd(p.sync + grp, 1) == S - 1) ? 1 : 0;
+        named_bar(1, 128);
+        if (last_flag) {
+          __threadfence();
+          // combine the S splits of this row in split order 0..S-1
+          float mm = -INFINITY;
+          for (int q = 0; q < S; ++q) mm = fmaxf(mm, __ldcg(p.part_ml + (grp * S + q) * 256 + row));
+          float wsum = 0.f;
+          for (int q = 0; q < S; ++q) {
+            const size_t sl = grp * S + q;
+            wsum += __ldcg(p.part_ml + sl * 256 + 128 + row) * exp2f(__ldcg(p.part_ml + sl * 256 + row) - mm);
+          }
+          const float inv = wsum > 0.f ? 1.0f / wsum : 0.f;
+          // all 128 columns of one split per round: 32 independent loads in flight
+          float acc[128];
+#pragma unroll
+          for (int c = 0; c < 128; ++c) acc[c] = 0.f;
+#pragma unroll 1
+          for (int q = 0; q < S; ++q) {
+            const size_t sl = grp * S + q;
+            const float pw = exp2f(__ldcg(p.part_ml + sl * 256 + row) - mm);
+            const float4* src = reinterpret_cast<const float4*>(p.part_o + sl * (kAT * kAT) + (size_t)row * kAT);
+            float4 v[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) v[c] = __ldcg(src + c);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              acc[4 * c] += pw * v[c].x; acc[4 * c + 1] += pw * v[c].y;
+              acc[4 * c + 2] += pw * v[c].z; acc[4 * c + 3] += pw * v[c].w;
+            }
+          }
+          if (qi < p.k) {
+            __nv_bfloat16* dst = p.O + ((size_t)b * p.k + qi) * d + (size_t)h * kAT;
+#pragma unroll
+            for (int c = 0; c < 128; c += 8) {
+              uint32_t w4[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                __nv_bfloat162 v2 = __floats2bfloat162_rn(acc[c + 2 * q] * inv, acc[c + 2 * q + 1] * inv);
+                w4[q] = *reinterpret_cast<uint32_t*>(&v2);
+              }
+              *reinterpret_cast<uint4*>(dst + c) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+          }
+          if (row == 0) p.sync[grp] = 0;  // ready for the next launch
+        }
+      }
+    }
+  }
+  __syncwarp();
+  __syncthreads();
+  if (abort_flag != 0 && threadIdx.x == 0) {
+    // after a bounded wait gave up: MMAs and copies in flight must finish
+    // before TMEM and shared memory are released
+    mbar_drain(&o_done, 0, err, 609);
+    mbar_drain(&q_full, 0, err, 610);
+    for (int j = kv_consumed; j < kv_issued; ++j) mbar_drain(&kv_full[j % kAStages], (j / kAStages) & 1, err, 611);
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 cudaError_t launch_attention(int dtype, const void* Q, const void* Kc, const void* Vc, void* O,
                              int B, int k, int N, int n_heads, int head_dim, float* part_o,
-                             float* part_ml, int max_rows, int* err, cudaStream_t stream) {
-  (void)err;
+                             float* part_ml, int max_rows, int* sync, int sync_len, int* err,
+                             cudaStream_t stream) {
   if (head_dim > 128) return cudaErrorInvalidValue;
   const float scale = 1.0f / sqrtf((float)head_dim);
-  if (dtype == 1 && head_dim == kHD) {
-    const int q_tiles = (k + kBQ - 1) / kBQ;
-    const int n_kt = (N + kBK - 1) / kBK;
-    const int base = q_tiles * n_heads * B;
+  if (dtype == 1 && head_dim == kAT) {
+    const int q_tiles = (k + kAT - 1) / kAT;
+    const int n_kt = (N + kAT - 1) / kAT;
+    const long long groups = (long long)B * n_heads * q_tiles;
+    // capacity of the scratch in (128-row, one-head) partial slots
+    const long long slots = (long long)max_rows * n_heads / kAT;
     int splits = 1;
-    // split the keys until about two CTAs per SM are busy, >= 2 key tiles per split
-    while (splits < 16 && base * splits < 2 * 148 && n_kt / (splits * 2) >= 2 &&
-           (long long)(splits * 2) * B * k <= max_rows)
+    // split the keys while the grid is small, each split keeps >= 2 key tiles
+    while (splits < 8 && groups * splits * 2 <= 160 && n_kt >= splits * 4 &&
+           groups * splits * 2 <= slots && groups <= sync_len)
       splits *= 2;
-    const int smem = (kBQ + 4 * kBK) * 256;
+    AttnTcParams p;
+    std::memset(&p, 0, sizeof(p));
+    if (encode_bf16_map(&p.tmQ, Q, (uint64_t)B * k, (uint64_t)n_heads * kAT) ||
+        encode_bf16_map(&p.tmK, Kc, (uint64_t)B * N, (uint64_t)n_heads * kAT) ||
+        encode_bf16_map(&p.tmV, Vc, (uint64_t)B * N, (uint64_t)n_heads * kAT))
+      return cudaErrorInvalidValue;
+    p.O = (__nv_bfloat16*)O;
+    p.part_o = part_o;
+    p.part_ml = part_ml;
+    p.sync = sync;
+    p.err = err;
+    p.B = B; p.k = k; p.N = N; p.n_heads = n_heads; p.q_tiles = q_tiles; p.splits = splits;
+    p.scale_log2 = scale * 1.4426950408889634f;
     static bool configured = false;
     if (!configured) {
-      cudaError_t e = cudaFuncSetAttribute(attn_mma_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kASmem);
       if (e != cudaSuccess) return e;
       configured = true;
     }
-    dim3 grid(q_tiles, n_heads, B * splits);
-    attn_mma_kernel<<<grid, 128, smem, stream>>>(
-        (const __nv_bfloat16*)Q, (const __nv_bfloat16*)Kc, (const __nv_bfloat16*)Vc,
-        (__nv_bfloat16*)O, part_o, part_ml, k, N, n_heads, splits, scale * 1.4426950408889634f);
-    if (splits > 1) {
-      cudaError_t e = cudaPeekAtLastError();
-      if (e != cudaSuccess) return e;
-      attn_combine_kernel<<<dim3(B * k, n_heads), kHD, 0, stream>>>(part_o, part_ml,
-                                                                   (__nv_bfloat16*)O, B * k,
-                                                                   n_heads, splits);
-    }
-    return cudaPeekAtLastError();
+    dim3 grid(q_tiles * splits, n_heads, B);
+    return launch_k(attn_tc_kernel, grid, dim3(kAThreads), kASmem, stream, p);
   }
   dim3 grid((k + 3) / 4, n_heads, B), block(128);
   if (dtype == 1)
-    attn_simt_kernel<__nv_bfloat16><<<grid, block, 0, stream>>>(
-        (const __nv_bfloat16*)Q, (const __nv_bfloat16*)Kc, (const __nv_bfloat16*)Vc,
-        (__nv_bfloat16*)O, k, N, n_heads, head_dim, scale);
-  else
-    attn_simt_kernel<float><<<grid, block, 0, stream>>>((const float*)Q, (const float*)Kc,
-                                                        (const float*)Vc, (float*)O, k, N, n_heads,
-                                                        head_dim, scale);
-  return cudaPeekAtLastError();
+    return launch_k(attn_simt_kernel<__nv_bfloat16>, grid, block, 0, stream, (const __nv_bfloat16*)Q,
+                    (const __nv_bfloat16*)Kc, (const __nv_bfloat16*)Vc, (__nv_bfloat16*)O, k, N,
+                    n_heads, head_dim, scale);
+  return launch_k(attn_simt_kernel<float>, grid, block, 0, stream, (const float*)Q, (const float*)Kc,
+                  (const float*)Vc, (float*)O, k, N, n_heads, head_dim, scale);
 }
 
 }  // namespace spa

@@ -7,6 +7,8 @@
 // and reports failure, so kernels can release what they hold and return.
 #pragma once
 #include <cstdint>
+#include <cstdlib>
+#include <utility>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -116,6 +118,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       return false;
     }
   }
+}
+
+// ---- programmatic dependent launch ---------------------------------------------
+// Every library kernel is launched with the programmatic-serialization
+// attribute (launch_k below) so that it can be scheduled while the previous
+// kernel of the stream is finishing.  It calls griddep_launch_dependents early
+// (the next kernel may then be scheduled once all its CTAs have) and
+// griddep_wait (all threads, on every path) before its first access to
+// global memory that an earlier kernel writes or reads, so a kernel's
+// completion still implies the completion of every kernel before it.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---- TMA (tiled, 2D, no multicast) -----------------------------------------
@@ -245,6 +260,32 @@ __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
+}
+
+// Host: programmatic dependent launch is on unless the environment sets SPA_PDL=0.
+inline bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("SPA_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+// Host: launches `kern` on `stream` with the programmatic-serialization attribute.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 }  // namespace spa

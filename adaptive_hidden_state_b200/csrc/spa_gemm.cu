@@ -308,6 +308,7 @@ __global__ void __launch_bounds__(kThreads, BN == 128 ? 2 : 1) tc_gemm_kernel(co
   __shared__ int abort_flag;
   __shared__ int2 s_rows[128];
 
+  griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, S = gridDim.x;
   const int n_tile = blockIdx.y, m_tile = blockIdx.z;
@@ -334,6 +335,7 @@ __global__ void __launch_bounds__(kThreads, BN == 128 ? 2 : 1) tc_gemm_kernel(co
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  griddep_wait();  // the token rows and the epilogue operands come from earlier kernels
 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&p.tmA);
@@ -434,13 +436,15 @@ static cudaError_t launch_tc_typed(const TcGemmParams& p, int m_tiles, int n_til
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = splits;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
@@ -489,6 +493,36 @@ __host__ __device__ inline int ws_stages(int nacc, int NT) {
   return st < kWsMaxStages ? st : kWsMaxStages;
 }
 
+// The NACC weight boxes (128 rows x 64 columns each) of one k-block of
+// column tile n_tile: GATEUP -> the first NACC/2 from W_gate, the rest the
+// same rows of W_up; otherwise 128 consecutive rows per accumulator.
+template <int NACC>
+__device__ __forceinline__ void ws_load_weights(const TcWsParams& p, int n_tile, uint8_t* sw,
+                                                uint64_t* bar, int kx) {
+  constexpr int FEAT = NACC * 128;
+#pragma unroll
+  for (int a = 0; a < NACC; ++a) {
+    int src, row;
+    if (p.b_mode == B_GATEUP) {
+      const int hal = NACC / 2;
+      src = a < hal ? 0 : 1;
+      row = n_tile * (FEAT / 2) + (a % hal) * 128;
+    } else if (p.b_mode == B_CONCAT3) {
+      const int g = n_tile * FEAT + a * 128;
+      src = g / p.b_rows_per_src;
+      row = g % p.b_rows_per_src;
+      if (src > 2) {  // past the last matrix: a box wholly out of range reads zeros
+        src = 2;
+        row = p.b_rows_per_src;
+      }
+    } else {
+      src = 0;
+      row = n_tile * FEAT + a * 128;
+    }
+    tma_load_2d(sw + a * kWsW, &p.tmW[src], bar, kx, row);
+  }
+}
+
 template <int MODE, int NACC>
 __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constant__ TcWsParams p) {
   constexpr int W_BYTES = NACC * kWsW;
@@ -506,6 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
   __shared__ int abort_flag;
   __shared__ int2 s_rows[128];
 
+  griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, S = gridDim.x;
   const int n_tile = blockIdx.y;
@@ -541,7 +576,25 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&p.tmX);
-    for (int it = 0; it < nk; ++it) {
+    // The weights do not depend on earlier kernels: the weight boxes of the
+    // first stages are requested before griddepcontrol.wait, so they stream
+    // while the previous kernel finishes; the token tiles follow the wait.
+    const int pre = nk < STAGES ? nk : STAGES;
+    for (int it = 0; it < pre; ++it) {
+      uint8_t* sw = smem + it * STAGE_BYTES;
+      mbar_arrive_expect_tx(&full_bar[it], (uint32_t)STAGE_BYTES);
+      int kit = it + rot;
+      if (kit >= nk) kit -= nk;
+      const int kx = (kb0 + kit) * 64;
+      ws_load_weights<NACC>(p, n_tile, sw, &full_bar[it], kx);
+    }
+    griddep_wait();
+    for (int it = 0; it < pre; ++it) {
+      int kit = it + rot;
+      if (kit >= nk) kit -= nk;
+      tma_load_2d(smem + it * STAGE_BYTES + W_BYTES, &p.tmX, &full_bar[it], (kb0 + kit) * 64, 0);
+    }
+    for (int it = pre; it < nk; ++it) {
       const int s = it % STAGES;
       if (it >= STAGES && !mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1, &abort_flag, err, 211))
         break;
@@ -551,29 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
       int kit = it + rot;
       if (kit >= nk) kit -= nk;
       const int kx = (kb0 + kit) * 64;
-#pragma unroll
-      for (int a = 0; a < NACC; ++a) {
-        // accumulator a holds weight rows: GATEUP -> the first NACC/2 from
-        // W_gate, the rest the same rows of W_up; otherwise 128 consecutive rows
-        int src, row;
-        if (p.b_mode == B_GATEUP) {
-          const int hal = NACC / 2;
-          src = a < hal ? 0 : 1;
-          row = n_tile * (FEAT / 2) + (a % hal) * 128;
-        } else if (p.b_mode == B_CONCAT3) {
-          const int g = n_tile * FEAT + a * 128;
-          src = g / p.b_rows_per_src;
-          row = g % p.b_rows_per_src;
-          if (src > 2) {  // past the last matrix: a box wholly out of range reads zeros
-            src = 2;
-            row = p.b_rows_per_src;
-          }
-        } else {
-          src = 0;
-          row = n_tile * FEAT + a * 128;
-        }
-        tma_load_2d(sw + a * kWsW, &p.tmW[src], &full_bar[s], kx, row);
-      }
+      ws_load_weights<NACC>(p, n_tile, sw, &full_bar[s], kx);
       tma_load_2d(sx, &p.tmX, &full_bar[s], kx, 0);
     }
   } else if (warp == 1 && lane == 0) {
@@ -601,6 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
   mbar_wait(&accum_bar, 0, &abort_flag, err, 213);
   __syncthreads();
   const bool good = (abort_flag == 0);
+  griddep_wait();  // the epilogue reads and writes rows that earlier kernels use
   tc_fence_after();
 
   float* tile = reinterpret_cast<float*>(smem);
@@ -665,13 +697,15 @@ static cudaError_t launch_ws_typed(const TcWsParams& p, int n_tiles, int splits,
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kWsSmem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = splits;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
@@ -775,6 +809,8 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtGemmParams p) 
   __shared__ __align__(16) float As[kSBK][kSBM + 4];
   __shared__ __align__(16) float Bs[kSBK][kSBN + 4];
   __shared__ __align__(16) float tile[kSBM * (kSBN + 4)];
+  griddep_launch_dependents();
+  griddep_wait();
   const int tid = threadIdx.x;
   const int n_tile = blockIdx.x, m_tile = blockIdx.y;
   const int ty = tid / 16, tx = tid % 16;
@@ -832,16 +868,15 @@ cudaError_t launch_simt_gemm(int mode, const SimtGemmParams& p, int m_tiles, int
                              cudaStream_t stream) {
   dim3 grid(n_tiles, m_tiles), block(256);
   switch (mode) {
-    case EPI_STORE: simt_gemm_kernel<EPI_STORE><<<grid, block, 0, stream>>>(p); break;
-    case EPI_QKV: simt_gemm_kernel<EPI_QKV><<<grid, block, 0, stream>>>(p); break;
-    case EPI_RESID: simt_gemm_kernel<EPI_RESID><<<grid, block, 0, stream>>>(p); break;
-    case EPI_SWIGLU: simt_gemm_kernel<EPI_SWIGLU><<<grid, block, 0, stream>>>(p); break;
-    case EPI_RESID_SCATTER: simt_gemm_kernel<EPI_RESID_SCATTER><<<grid, block, 0, stream>>>(p); break;
-    case EPI_PROXY: simt_gemm_kernel<EPI_PROXY><<<grid, block, 0, stream>>>(p); break;
-    case EPI_ARGMAX: simt_gemm_kernel<EPI_ARGMAX><<<grid, block, 0, stream>>>(p); break;
+    case EPI_STORE: return launch_k(simt_gemm_kernel<EPI_STORE>, grid, block, 0, stream, p);
+    case EPI_QKV: return launch_k(simt_gemm_kernel<EPI_QKV>, grid, block, 0, stream, p);
+    case EPI_RESID: return launch_k(simt_gemm_kernel<EPI_RESID>, grid, block, 0, stream, p);
+    case EPI_SWIGLU: return launch_k(simt_gemm_kernel<EPI_SWIGLU>, grid, block, 0, stream, p);
+    case EPI_RESID_SCATTER: return launch_k(simt_gemm_kernel<EPI_RESID_SCATTER>, grid, block, 0, stream, p);
+    case EPI_PROXY: return launch_k(simt_gemm_kernel<EPI_PROXY>, grid, block, 0, stream, p);
+    case EPI_ARGMAX: return launch_k(simt_gemm_kernel<EPI_ARGMAX>, grid, block, 0, stream, p);
     default: return cudaErrorInvalidValue;
   }
-  return cudaPeekAtLastError();
 }
 
 // ---------------------------------------------------------------------------

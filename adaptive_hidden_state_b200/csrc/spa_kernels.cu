@@ -58,6 +58,8 @@ __global__ void __launch_bounds__(128) rmsnorm_rows_kernel(const T* src, int src
                                                            int M, int d, const T* gamma, float eps,
                                                            T* X, int* err) {
   constexpr int VEC = 16 / sizeof(T);
+  griddep_launch_dependents();
+  griddep_wait();
   const int t = blockIdx.x;
   if (t >= M) return;
   size_t row;
@@ -122,14 +124,11 @@ cudaError_t launch_rmsnorm_rows(int dtype, const void* src, int src_is_cache, co
   const int vec = dtype == 1 ? 8 : 4;
   if (d % vec != 0 || d / vec > 128 * kNormMaxChunks) return cudaErrorInvalidValue;
   if (dtype == 1)
-    rmsnorm_rows_kernel<__nv_bfloat16><<<M, 128, 0, stream>>>(
-        (const __nv_bfloat16*)src, src_is_cache, idx, tps, N, M, d, (const __nv_bfloat16*)gamma,
-        eps, (__nv_bfloat16*)X, err);
-  else
-    rmsnorm_rows_kernel<float><<<M, 128, 0, stream>>>((const float*)src, src_is_cache, idx, tps, N,
-                                                      M, d, (const float*)gamma, eps, (float*)X,
-                                                      err);
-  return cudaPeekAtLastError();
+    return launch_k(rmsnorm_rows_kernel<__nv_bfloat16>, dim3(M), dim3(128), 0, stream,
+                    (const __nv_bfloat16*)src, src_is_cache, idx, tps, N, M, d,
+                    (const __nv_bfloat16*)gamma, eps, (__nv_bfloat16*)X, err);
+  return launch_k(rmsnorm_rows_kernel<float>, dim3(M), dim3(128), 0, stream, (const float*)src,
+                  src_is_cache, idx, tps, N, M, d, (const float*)gamma, eps, (float*)X, err);
 }
 
 // ---------------------------------------------------------------------------
@@ -184,6 +183,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_select_kernel(const float* 
   __shared__ int warp_tot[33];
   __shared__ int sel_digit, sel_above;
   __shared__ int32_t list[kTopkPerThread * kTopkThreads];
+  griddep_launch_dependents();
+  griddep_wait();
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
   const float* s = score + (size_t)b * N;
@@ -284,22 +285,42 @@ __global__ void __launch_bounds__(kTopkThreads) topk_select_kernel(const float* 
     }
   }
   __syncthreads();
-  // P^c[b, I] <- a_hat[b, I]
+  // P^c[b, I] <- a_hat[b, I], flattened over (selected row, 16-byte chunk):
+  // up to kScatterBatch loads per thread in flight before any store
   if (p_cache != nullptr) {
-    // flattened over (selected row, column): 4 independent copies per thread in flight
-    const int total = k * r;
-    for (int base = tid; base < total; base += kTopkThreads * 4) {
-      float v[4];
-      size_t off[4];
+    constexpr int kScatterBatch = 8;
+    if ((r & 3) == 0) {
+      const int r4 = r / 4, total = k * r4;
+      const float4* src = reinterpret_cast<const float4*>(a_hat);
+      float4* dst = reinterpret_cast<float4*>(p_cache);
+      for (int base = tid; base < total; base += kTopkThreads * kScatterBatch) {
+        float4 v[kScatterBatch];
+        size_t off[kScatterBatch];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int it = base + u * kTopkThreads;
-        off[u] = it < total ? ((size_t)b * N + list[it / r]) * r + (it % r) : 0;
-        if (it < total) v[u] = a_hat[off[u]];
+        for (int u = 0; u < kScatterBatch; ++u) {
+          const int it = base + u * kTopkThreads;
+          off[u] = it < total ? ((size_t)b * N + list[it / r4]) * r4 + (it % r4) : 0;
+          if (it < total) v[u] = src[off[u]];
+        }
+#pragma unroll
+        for (int u = 0; u < kScatterBatch; ++u)
+          if (base + u * kTopkThreads < total) dst[off[u]] = v[u];
       }
+    } else {
+      const int total = k * r;
+      for (int base = tid; base < total; base += kTopkThreads * kScatterBatch) {
+        float v[kScatterBatch];
+        size_t off[kScatterBatch];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (base + u * kTopkThreads < total) p_cache[off[u]] = v[u];
+        for (int u = 0; u < kScatterBatch; ++u) {
+          const int it = base + u * kTopkThreads;
+          off[u] = it < total ? ((size_t)b * N + list[it / r]) * r + (it % r) : 0;
+          if (it < total) v[u] = a_hat[off[u]];
+        }
+#pragma unroll
+        for (int u = 0; u < kScatterBatch; ++u)
+          if (base + u * kTopkThreads < total) p_cache[off[u]] = v[u];
+      }
     }
   }
 }
@@ -308,8 +329,8 @@ cudaError_t launch_topk_select(const float* score, int B, int N, int k, int32_t*
                                const float* a_hat, float* p_cache, int r, int* err,
                                cudaStream_t stream) {
   if (N > kTopkThreads * kTopkPerThread || k < 1 || k > N) return cudaErrorInvalidValue;
-  topk_select_kernel<<<B, kTopkThreads, 0, stream>>>(score, N, k, idx, a_hat, p_cache, r, err);
-  return cudaPeekAtLastError();
+  return launch_k(topk_select_kernel, dim3(B), dim3(kTopkThreads), 0, stream, score, N, k, idx,
+                  a_hat, p_cache, r, err);
 }
 
 // ---------------------------------------------------------------------------
@@ -318,6 +339,8 @@ cudaError_t launch_topk_select(const float* score, int B, int N, int k, int32_t*
 template <typename T>
 __global__ void embed_rows_kernel(const T* embed, const int32_t* tokens, const int32_t* pos, int u,
                                   int N, int d, int vocab, T* h0, int* err) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int j = blockIdx.x;  // row among B*u (or B*N when pos is null)
   const int b = j / u;
   const int p = pos ? pos[j] : (j % u);
@@ -337,12 +360,10 @@ cudaError_t launch_embed_rows(int dtype, const void* embed, const int32_t* token
   const int rows = B * u;
   if (rows <= 0) return cudaSuccess;
   if (dtype == 1)
-    embed_rows_kernel<__nv_bfloat16><<<rows, 128, 0, stream>>>(
-        (const __nv_bfloat16*)embed, tokens, pos, u, N, d, vocab, (__nv_bfloat16*)h0, err);
-  else
-    embed_rows_kernel<float><<<rows, 128, 0, stream>>>((const float*)embed, tokens, pos, u, N, d,
-                                                       vocab, (float*)h0, err);
-  return cudaPeekAtLastError();
+    return launch_k(embed_rows_kernel<__nv_bfloat16>, dim3(rows), dim3(128), 0, stream,
+                    (const __nv_bfloat16*)embed, tokens, pos, u, N, d, vocab, (__nv_bfloat16*)h0, err);
+  return launch_k(embed_rows_kernel<float>, dim3(rows), dim3(128), 0, stream, (const float*)embed,
+                  tokens, pos, u, N, d, vocab, (float*)h0, err);
 }
 
 cudaError_t launch_gather_final(int dtype, const void* hc, const int32_t* pos, int B, int u, int N,
@@ -353,6 +374,8 @@ cudaError_t launch_gather_final(int dtype, const void* hc, const int32_t* pos, i
 
 __global__ void argmax_reduce_kernel(const float* val, const int32_t* idx, int rows, int n_tiles,
                                      int32_t* out) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int row = blockIdx.x;
   const int lane = threadIdx.x;
   float best = -INFINITY;
@@ -374,19 +397,19 @@ __global__ void argmax_reduce_kernel(const float* val, const int32_t* idx, int r
 cudaError_t launch_argmax_reduce(const float* val, const int32_t* idx, int rows, int n_tiles,
                                  int32_t* out, cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
-  argmax_reduce_kernel<<<rows, 32, 0, stream>>>(val, idx, rows, n_tiles, out);
-  return cudaPeekAtLastError();
+  return launch_k(argmax_reduce_kernel, dim3(rows), dim3(32), 0, stream, val, idx, rows, n_tiles, out);
 }
 
 __global__ void copy_i32_kernel(const int32_t* src, int32_t* dst, int n) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) dst[i] = src[i];
 }
 
 cudaError_t launch_copy_i32(const int32_t* src, int32_t* dst, int n, cudaStream_t stream) {
   if (n <= 0) return cudaSuccess;
-  copy_i32_kernel<<<(n + 255) / 256, 256, 0, stream>>>(src, dst, n);
-  return cudaPeekAtLastError();
+  return launch_k(copy_i32_kernel, dim3((n + 255) / 256), dim3(256), 0, stream, src, dst, n);
 }
 
 }  // namespace spa

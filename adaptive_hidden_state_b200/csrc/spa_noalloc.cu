@@ -23,8 +23,11 @@
 
 namespace {
 
-// 8 MiB of fp32 split-KV partials: B * k * (d + 2 * n_heads) floats at most.
+// 8 MiB: fp32 split-KV partials, B * k * (d + 2 * n_heads) floats at most,
+// then kNoAllocSyncInts counters (per query tile: splits finished).
 constexpr size_t kNoAllocScratchFloats = (size_t)2 << 20;
+constexpr int kNoAllocSyncInts = 4096;
+constexpr size_t kNoAllocPartialFloats = kNoAllocScratchFloats - kNoAllocSyncInts;
 
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
 
@@ -47,10 +50,11 @@ extern "C" int spa_attention_noalloc(const void* Q, const void* k_cache, const v
   const long long d = (long long)n_heads * head_dim;
   const long long row_floats = d + 2LL * n_heads;  // one partial output row + its (m, l) pairs
   const long long rows = (long long)B * k;
-  if (rows * row_floats > (long long)kNoAllocScratchFloats)
+  const long long tiles = (long long)B * n_heads * ((k + 127) / 128);
+  if (rows * row_floats > (long long)kNoAllocPartialFloats || tiles > kNoAllocSyncInts)
     return fail(SPA_ERR_SHAPE,
                 "B * k * (n_heads * head_dim + 2 * n_heads) exceeds the fixed scratch "
-                "(2 Mi floats = 8 MiB)");
+                "(2 Mi floats = 8 MiB), or B * n_heads * ceil(k / 128) exceeds 4096");
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     cudaGetLastError();
@@ -73,12 +77,18 @@ extern "C" int spa_attention_noalloc(const void* Q, const void* k_cache, const v
   }
   // split partials first, then their (m, l) pairs; the launcher splits the
   // keys only as far as max_rows partial rows fit
-  const int max_rows = (int)(kNoAllocScratchFloats / row_floats);
+  const int max_rows = (int)(kNoAllocPartialFloats / row_floats);
   float* part_o = scratch;
   float* part_ml = scratch + (size_t)max_rows * d;
+  int* sync = reinterpret_cast<int*>(scratch + kNoAllocPartialFloats);
+  // the split counters must start at zero (a completed call leaves them so)
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(sync, 0, (size_t)tiles * sizeof(int), s) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(SPA_ERR_CUDA, "clearing the split counters failed");
+  }
   const cudaError_t e = spa::launch_attention(1, Q, k_cache, v_cache, O, B, k, N, n_heads, head_dim,
-                                              part_o, part_ml, max_rows, nullptr,
-                                              static_cast<cudaStream_t>(stream));
+                                              part_o, part_ml, max_rows, sync, (int)tiles, nullptr, s);
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, cudaGetErrorString(e));
   return SPA_OK;
 }
