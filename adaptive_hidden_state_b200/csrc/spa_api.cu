@@ -168,6 +168,9 @@ extern "C" int spa_singular_proxy_host(const float* w_v, int d, int r, float* w_
 // ---------------------------------------------------------------------------
 // handles
 // ---------------------------------------------------------------------------
+// SMs of the device, recorded when a workspace is created (GEMM planning).
+static int ws_num_sms_hint = 148;
+
 struct spa_workspace {
   spa_layer_desc desc;
   int device = 0;
@@ -278,6 +281,7 @@ extern "C" int spa_workspace_create(const spa_layer_desc* desc, int max_B, int m
   ws->elem = desc->dtype == SPA_BF16 ? 2 : 4;
   cudaGetDevice(&ws->device);
   cudaDeviceGetAttribute(&ws->num_sms, cudaDevAttrMultiProcessorCount, ws->device);
+  if (ws->num_sms > 0) ws_num_sms_hint = ws->num_sms;
   const size_t cap = ws->cap, d = desc->d, F = desc->ffn, r = desc->r, e = ws->elem;
   ws->part_rows = (int)std::min<size_t>(cap, 4096) * 4;
   int st = SPA_OK;
@@ -532,15 +536,20 @@ static int run_ws(int mode, bool gateup, TcWsParams& p, const void* X, int M, in
   if (M <= 0) return SPA_OK;
   if (M > 256) return fail(SPA_ERR_SHAPE, "weight-stationary GEMM takes at most 256 tokens");
   const int NT = ((M + 31) / 32) * 32;
+  // The layer GEMMs stream faster with one 128-row block per CTA (two for
+  // gate/up): smaller TMA ring stages, more of them in flight.  Only a GEMM
+  // with many more weight rows than the SMs can cover (the LM head) takes
+  // larger blocks, which need fewer TMA boxes per weight byte.
   const int min_nacc = gateup ? 2 : 1;
   int nacc = min_nacc;
-  for (int n = 4; n > min_nacc; n /= 2) {
-    const int feat = gateup ? n / 2 * 128 : n * 128;
-    if (n * NT <= 512 && (rows + feat - 1) / feat >= 16) {
-      nacc = n;
-      break;
+  if (rows / 128 > 4 * ws_num_sms_hint)
+    for (int n = 4; n > min_nacc; n /= 2) {
+      const int feat = gateup ? n / 2 * 128 : n * 128;
+      if (n * NT <= 512 && (rows + feat - 1) / feat >= 16) {
+        nacc = n;
+        break;
+      }
     }
-  }
   if (const char* env = std::getenv("SPA_WS_NACC")) {  // tuning override
     const int v = std::atoi(env);
     if ((v == 1 || v == 2 || v == 4) && v >= min_nacc && v * NT <= 512) nacc = v;
@@ -612,7 +621,11 @@ static int run_proxy(spa_layer* L, const void* H, const spa_layer_cache* c, floa
     p.b_rows_per_src = r;
     p.ep = ep;
     // split count depends on d only, so a row's proxy bits never depend on B or N
-    const int splits = std::max(1, std::min(16, (d / 64) / 4));
+    int splits = std::max(1, std::min(16, (d / 64) / 4));
+    if (const char* env = std::getenv("SPA_PROXY_SPLITS")) {  // tuning override (depends on d only)
+      const int v = std::atoi(env);
+      if (v >= 1 && v <= 16 && (d / 64) / v >= 1) splits = v;
+    }
     return run_tc(EPI_PROXY, r <= 128 ? 128 : 256, p, M, 1, splits, s, &L->ws->prof, w);
   }
   SimtGemmParams p;
