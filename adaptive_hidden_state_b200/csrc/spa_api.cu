@@ -693,7 +693,7 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
     ProfScope ps(prof, SPA_PROF_ATTN, 2.0 * Md * es + 2.0 * Bn * d * es, 4.0 * Md * N, s);
     e = launch_attention(D.dtype, ws->Q, c->k_cache, c->v_cache, ws->O, c->B, tps, N, D.n_heads,
                          D.head_dim, ws->part_o, ws->part_ml, ws->part_rows, ws->attn_sync,
-                         ws->attn_sync_len, ws->err, s);
+                         ws->attn_sync_len, ws->err, 1, s);
   }
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
   // H1 = H[I] + O W_o^T

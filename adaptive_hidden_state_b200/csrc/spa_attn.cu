@@ -87,10 +87,14 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(const T* Q, const T* Kc,
 //               rescales O in TMEM only when the max grows by more than 2^8
 //               (the result is exact for any reference max: the final
 //               division by l uses the same one).
-// With several key splits each CTA writes (O, m, l) to scratch; the last CTA
-// of the query tile to finish (an atomic counter) combines them in split
-// order 0..S-1, so the result does not depend on timing, and resets the
-// counter.
+// With several key splits the S CTAs of a query tile form a thread-block
+// cluster: each leaves its unnormalised O rows, m and l in its own shared
+// memory, and after a cluster barrier CTA q combines rows [q*128/S,
+// (q+1)*128/S) of all S splits through distributed shared memory, in split
+// order 0..S-1, so the result does not depend on timing.  Where clusters are
+// not allowed (the allocation-free entry point) each CTA writes (O, m, l) to
+// scratch instead and the last CTA of the query tile to finish (an atomic
+// counter) combines them in the same order and resets the counter.
 // ---------------------------------------------------------------------------
 constexpr int kAT = 128;                 // queries per CTA and keys per tile
 constexpr int kAQBytes = 2 * 16384;      // Q: two 64-column boxes of 128 rows
@@ -111,6 +115,7 @@ struct alignas(64) AttnTcParams {
   int* sync;        // per query tile: splits finished (zero between launches)
   int* err;
   int B, k, N, n_heads, q_tiles, splits;
+  int cluster;       // splits > 1: 1 = combine in distributed shared memory
   float scale_log2;  // log2(e) / sqrt(head_dim)
 };
 
@@ -180,6 +185,8 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_tc_kernel(const __grid_cons
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag, last_flag;
   __shared__ int kv_issued, kv_consumed, tile_ok;
+  __shared__ float s_m[kAT], s_l[kAT];  // this split's row max and sum (cluster combine)
+  __shared__ float s_w[kAT / 2][8];     // combine weights of this CTA's rows, per split
 
   griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -378,6 +385,23 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_tc_kernel(const __grid_cons
             }
           }
         }
+      } else if (p.cluster) {
+        // unnormalised O row into the (now idle) K/V ring, 16-byte chunk c
+        // of row r at chunk position c ^ (r % 32)
+        float* sO = reinterpret_cast<float*>(sKV);
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          float o[32];
+          tmem_ld32(lane_base + 256u + (uint32_t)c0, o);
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            const int ch = (c0 + c) >> 2;
+            *reinterpret_cast<float4*>(sO + row * 128 + ((ch ^ (row & 31)) << 2)) =
+                make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+          }
+        }
+        s_m[row] = m_used;
+        s_l[row] = l;
       } else {
         const size_t grp = ((size_t)b * p.n_heads + h) * p.q_tiles + qt;
         const size_t slot = grp * S + sp;
@@ -453,14 +477,95 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_tc_kernel(const __grid_cons
     for (int j = kv_consumed; j < kv_issued; ++j) mbar_drain(&kv_full[j % kAStages], (j / kAStages) & 1, err, 611);
   }
   __syncthreads();
+  if (S > 1 && p.cluster) {
+    // every thread of every CTA of the cluster passes both cluster barriers,
+    // whatever happened before, so none waits for a CTA that left
+    cluster_sync();
+    const bool good = abort_flag == 0 && tile_ok;
+    const int RS = kAT / S, r0 = sp * RS;
+    if (good) {
+      if ((int)threadIdx.x < RS) {
+        const int row = r0 + threadIdx.x;
+        const uint32_t am = smem_u32(&s_m[row]), al = smem_u32(&s_l[row]);
+        float mq[8], lq[8], mm = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q < S) {
+            mq[q] = ld_dsmem_f32(mapa_shared(am, (uint32_t)q));
+            lq[q] = ld_dsmem_f32(mapa_shared(al, (uint32_t)q));
+            mm = fmaxf(mm, mq[q]);
+          }
+        float w[8], L = 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q < S) {
+            w[q] = mq[q] == -INFINITY ? 0.f : exp2f(mq[q] - mm);
+            L += w[q] * lq[q];
+          }
+        const float inv = L > 0.f ? 1.0f / L : 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q < S) s_w[threadIdx.x][q] = w[q] * inv;
+      }
+      __syncthreads();
+      // one warp per row: 32 lanes x 4 columns, S remote loads in flight each
+      const float* sO = reinterpret_cast<const float*>(sKV);
+      const int d = p.n_heads * kAT;
+      for (int task = threadIdx.x; task < RS * 32; task += kAThreads) {
+        const int rl = task >> 5, ch = task & 31, row = r0 + rl;
+        const int qi = qt * kAT + row;
+        if (qi >= p.k) continue;
+        const uint32_t la = smem_u32(sO + row * 128 + ((ch ^ (row & 31)) << 2));
+        float4 v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q < S) v[q] = ld_dsmem_f4(mapa_shared(la, (uint32_t)q));
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q < S) {
+            const float wq = s_w[rl][q];
+            acc.x += wq * v[q].x; acc.y += wq * v[q].y; acc.z += wq * v[q].z; acc.w += wq * v[q].w;
+          }
+        store4(p.O + ((size_t)b * p.k + qi) * d + (size_t)h * kAT + ch * 4, acc);
+      }
+    }
+    cluster_sync();
+  }
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// How many clusters of `splits` attention CTAs the GPU holds at once (0: none).
+static int attn_max_clusters(int splits) {
+  static int cache[9] = {0};
+  if (splits < 2 || splits > 8) return 0;
+  if (cache[splits] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(splits, 1, 1);
+    cfg.blockDim = dim3(kAThreads, 1, 1);
+    cfg.dynamicSmemBytes = kASmem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    cache[splits] = n > 0 ? n : -1;
+  }
+  return cache[splits] > 0 ? cache[splits] : 0;
 }
 
 cudaError_t launch_attention(int dtype, const void* Q, const void* Kc, const void* Vc, void* O,
                              int B, int k, int N, int n_heads, int head_dim, float* part_o,
                              float* part_ml, int max_rows, int* sync, int sync_len, int* err,
-                             cudaStream_t stream) {
+                             int allow_cluster, cudaStream_t stream) {
   if (head_dim > 128) return cudaErrorInvalidValue;
   const float scale = 1.0f / sqrtf((float)head_dim);
   if (dtype == 1 && head_dim == kAT) {
@@ -469,11 +574,23 @@ cudaError_t launch_attention(int dtype, const void* Q, const void* Kc, const voi
     const long long groups = (long long)B * n_heads * q_tiles;
     // capacity of the scratch in (128-row, one-head) partial slots
     const long long slots = (long long)max_rows * n_heads / kAT;
+    static bool configured = false;
+    if (!configured) {
+      cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kASmem);
+      if (e != cudaSuccess) return e;
+      configured = true;
+    }
     int splits = 1;
-    // split the keys while the grid is small, each split keeps >= 2 key tiles
-    while (splits < 8 && groups * splits * 2 <= 160 && n_kt >= splits * 4 &&
-           groups * splits * 2 <= slots && groups <= sync_len)
-      splits *= 2;
+    if (allow_cluster) {
+      // split the keys while every cluster of the grid is resident at once and
+      // each split keeps >= 2 key tiles
+      while (splits < 8 && n_kt >= splits * 4 && groups <= attn_max_clusters(splits * 2)) splits *= 2;
+    } else {
+      // split the keys while the grid is small, each split keeps >= 2 key tiles
+      while (splits < 8 && groups * splits * 2 <= 160 && n_kt >= splits * 4 &&
+             groups * splits * 2 <= slots && groups <= sync_len)
+        splits *= 2;
+    }
     AttnTcParams p;
     std::memset(&p, 0, sizeof(p));
     if (encode_bf16_map(&p.tmQ, Q, (uint64_t)B * k, (uint64_t)n_heads * kAT) ||
@@ -486,15 +603,25 @@ cudaError_t launch_attention(int dtype, const void* Q, const void* Kc, const voi
     p.sync = sync;
     p.err = err;
     p.B = B; p.k = k; p.N = N; p.n_heads = n_heads; p.q_tiles = q_tiles; p.splits = splits;
+    p.cluster = allow_cluster && splits > 1;
     p.scale_log2 = scale * 1.4426950408889634f;
-    static bool configured = false;
-    if (!configured) {
-      cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kASmem);
-      if (e != cudaSuccess) return e;
-      configured = true;
-    }
     dim3 grid(q_tiles * splits, n_heads, B);
-    return launch_k(attn_tc_kernel, grid, dim3(kAThreads), kASmem, stream, p);
+    if (!p.cluster) return launch_k(attn_tc_kernel, grid, dim3(kAThreads), kASmem, stream, p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kAThreads, 1, 1);
+    cfg.dynamicSmemBytes = kASmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, attn_tc_kernel, p);
   }
   dim3 grid((k + 3) / 4, n_heads, B), block(128);
   if (dtype == 1)

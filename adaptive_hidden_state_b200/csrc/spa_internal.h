@@ -121,12 +121,14 @@ cudaError_t launch_topk_select(const float* score, int B, int N, int k, int32_t*
                                const float* a_hat, float* p_cache, int r, int* err,
                                cudaStream_t stream);
 // Sparse-query attention: O[t] = softmax(Q_t K^cT / sqrt(hd)) V^c per head.
-// Key splits use part_o / part_ml (max_rows partial rows of n_heads * hd and
+// allow_cluster = 1: key splits run as thread-block clusters and combine in
+// distributed shared memory (the scratch arguments are unused).  Otherwise
+// key splits use part_o / part_ml (max_rows partial rows of n_heads * hd and
 // of 2 * n_heads floats) and `sync` (sync_len ints, zero between launches).
 cudaError_t launch_attention(int dtype, const void* Q, const void* Kc, const void* Vc, void* O,
                              int B, int k, int N, int n_heads, int head_dim, float* part_o,
                              float* part_ml, int max_rows, int* sync, int sync_len, int* err,
-                             cudaStream_t stream);
+                             int allow_cluster, cudaStream_t stream);
 // h0[b, pos] <- embed[tok] for the listed (or all) positions.
 cudaError_t launch_embed_rows(int dtype, const void* embed, const int32_t* tokens,
                               const int32_t* pos, int B, int u, int N, int d, int vocab,

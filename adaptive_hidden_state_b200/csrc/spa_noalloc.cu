@@ -88,7 +88,7 @@ extern "C" int spa_attention_noalloc(const void* Q, const void* k_cache, const v
     return fail(SPA_ERR_CUDA, "clearing the split counters failed");
   }
   const cudaError_t e = spa::launch_attention(1, Q, k_cache, v_cache, O, B, k, N, n_heads, head_dim,
-                                              part_o, part_ml, max_rows, sync, (int)tiles, nullptr, s);
+                                              part_o, part_ml, max_rows, sync, (int)tiles, nullptr, 0, s);
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, cudaGetErrorString(e));
   return SPA_OK;
 }

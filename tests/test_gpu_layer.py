@@ -130,6 +130,18 @@ def test_bf16_wide_weight_tiles(monkeypatch, nacc, B, N, k):
     _step(lp, cache, ocs, H2, k)
 
 
+@pytest.mark.parametrize("B,N,k", [(1, 2048, 200), (2, 1000, 62), (1, 1536, 129)])
+def test_bf16_split_key_attention(B, N, k):
+    # long caches: the keys of each query tile are split over a cluster of 8,
+    # 4 and 4 CTAs (2, 2 and 3 key tiles each; N=1000 ends in a partial key
+    # tile), with one or two query tiles, the second holding 72 or 1 rows
+    lp = LayerPair(spa, SMALL_BF16, seed=50 + k, dtype=spa.SPA_BF16, max_B=B, max_N=N, std=0.05)
+    H = synth.hidden_states(B, N, 256, seed=k + 7, bf16=True)
+    cache, ocs = _run_fill(lp, H)
+    H2, _ = synth.drift_rows(H, 0.05, 0.5, seed=k + 8, bf16=True)  # fewer drifted rows than k
+    _step(lp, cache, ocs, H2, k)
+
+
 def test_bf16_zero_drift_selects_lowest_indices():
     lp = LayerPair(spa, SMALL_BF16, seed=21, dtype=spa.SPA_BF16, max_B=1, max_N=200, std=0.05)
     H = synth.hidden_states(1, 200, 256, seed=22, bf16=True)
