@@ -641,7 +641,7 @@ static int run_proxy(spa_layer* L, const void* H, const spa_layer_cache* c, floa
 
 // Phases 2 and 3 for M = B * tps tokens; idx == null means every row (rho = 1).
 static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
-                     const spa_layer_cache* c, cudaStream_t s) {
+                     const spa_layer_cache* c, cudaStream_t s, bool x_ready = false) {
   spa_workspace* ws = L->ws;
   const spa_layer_desc& D = L->desc;
   const int d = D.d, F = D.ffn, M = c->B * tps, N = c->N;
@@ -649,12 +649,14 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
   const double es = bf ? 2.0 : 4.0, Md = (double)M * d, Bn = (double)c->B * N;
   Profiler* prof = &ws->prof;
   cudaError_t e;
-  // x = RMSNorm(H[I])
-  {
-    ProfScope ps(prof, SPA_PROF_NORM, 2.0 * Md * es + d * es, 4.0 * Md, s);
-    e = launch_rmsnorm_rows(D.dtype, H, 1, idx, tps, N, M, d, L->w.attn_norm, D.rms_eps, ws->X, ws->err, s);
+  // x = RMSNorm(H[I]) (already in ws->X when the select wrote it)
+  if (!x_ready) {
+    {
+      ProfScope ps(prof, SPA_PROF_NORM, 2.0 * Md * es + d * es, 4.0 * Md, s);
+      e = launch_rmsnorm_rows(D.dtype, H, 1, idx, tps, N, M, d, L->w.attn_norm, D.rms_eps, ws->X, ws->err, s);
+    }
+    if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "rmsnorm launch: %s", cudaGetErrorString(e));
   }
-  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "rmsnorm launch: %s", cudaGetErrorString(e));
   // Q, K, V with RoPE; K, V scattered into the caches
   {
     EpiParams ep = base_epi(L, M, tps, N, idx);
@@ -829,8 +831,30 @@ extern "C" int spa_partial_block(spa_layer* L, const void* H, const int32_t* idx
 
 extern "C" int spa_layer_step(spa_layer* L, const void* H, const spa_layer_cache* c, int k,
                               int32_t* idx, void* stream) {
-  SPA_TRY(spa_proxy_select(L, H, c, k, idx, nullptr, stream));
-  return run_block(L, H, idx, k, c, (cudaStream_t)stream);
+  if (!L) return fail(SPA_ERR_INVALID, "null layer");
+  SPA_TRY(check_H(H));
+  SPA_TRY(check_cache(L, c));
+  const spa_layer_desc& D = L->desc;
+  if (!select_norm_supported(D.dtype, c->N, D.d)) {
+    SPA_TRY(spa_proxy_select(L, H, c, k, idx, nullptr, stream));
+    return run_block(L, H, idx, k, c, (cudaStream_t)stream);
+  }
+  // proxy, then one launch for the select, the P^c scatter and RMSNorm(H[I])
+  if (!idx) return fail(SPA_ERR_INVALID, "null idx");
+  if (k < 1 || k > c->N) return fail(SPA_ERR_SHAPE, "k=%d outside [1, N=%d]", k, c->N);
+  cudaStream_t s = (cudaStream_t)stream;
+  spa_workspace* ws = L->ws;
+  SPA_TRY(run_proxy(L, H, c, ws->score, 0, s));
+  cudaError_t e;
+  {
+    const double Bn = (double)c->B * c->N, Bk = (double)c->B * k;
+    const double es = D.dtype == SPA_BF16 ? 2.0 : 4.0;
+    ProfScope ps(&ws->prof, SPA_PROF_TOPK, 4.0 * Bn + 8.0 * Bk * D.r + 4.0 * Bk + 2.0 * Bk * D.d * es, 0.0, s);
+    e = launch_select_norm(D.dtype, ws->score, c->B, c->N, k, idx, ws->a_hat, c->p_cache, D.r, H,
+                           L->w.attn_norm, D.rms_eps, D.d, ws->X, ws->err, s);
+  }
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "select + norm launch: %s", cudaGetErrorString(e));
+  return run_block(L, H, idx, k, c, s, true);
 }
 
 extern "C" int spa_full_block(spa_layer* L, const void* H, const spa_layer_cache* c, int fill_proxy,

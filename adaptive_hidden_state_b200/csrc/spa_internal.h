@@ -120,6 +120,15 @@ cudaError_t launch_rmsnorm_rows(int dtype, const void* src, int src_is_cache, co
 cudaError_t launch_topk_select(const float* score, int B, int N, int k, int32_t* idx,
                                const float* a_hat, float* p_cache, int r, int* err,
                                cudaStream_t stream);
+// The top-k above fused with the gathered RMSNorm of the selected rows
+// (X[b*k + j] = RMSNorm(H[b, idx[b, j]]) * gamma), bit-identical to running
+// launch_topk_select then launch_rmsnorm_rows; for N <= 2048 and rows of at
+// most 512 16-byte chunks (select_norm_supported).
+bool select_norm_supported(int dtype, int N, int d);
+cudaError_t launch_select_norm(int dtype, const float* score, int B, int N, int k, int32_t* idx,
+                               const float* a_hat, float* p_cache, int r, const void* H,
+                               const void* gamma, float eps, int d, void* X, int* err,
+                               cudaStream_t stream);
 // Sparse-query attention: O[t] = softmax(Q_t K^cT / sqrt(hd)) V^c per head.
 // allow_cluster = 1: key splits run as thread-block clusters and combine in
 // distributed shared memory (the scratch arguments are unused).  Otherwise

@@ -52,12 +52,61 @@ __device__ __forceinline__ uint4 pack16<float>(const float* f) {
                     __float_as_uint(f[3]));
 }
 
+// One row, 128 threads (gt = thread index within the group, red = 4 floats
+// of shared memory for the group, bar = the group's barrier).  The sum of
+// squares is taken in the same order by every caller, so a row's output bits
+// do not depend on the kernel that normalises it.
+template <typename T, int MAXC, typename Bar>
+__device__ __forceinline__ void rmsnorm_one_row(const T* src_row, const T* gamma, int d, float eps,
+                                                T* out_row, int gt, float* red, Bar bar) {
+  constexpr int VEC = 16 / sizeof(T);
+  const uint4* x = reinterpret_cast<const uint4*>(src_row);
+  const uint4* g = reinterpret_cast<const uint4*>(gamma);
+  const int nch = d / VEC;
+  uint4 xv[MAXC], gv[MAXC];  // the row and gamma, all loads issued up front
+#pragma unroll
+  for (int i = 0; i < MAXC; ++i) {
+    const int c = gt + 128 * i;
+    if (c < nch) {
+      xv[i] = x[c];
+      gv[i] = g[c];
+    }
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXC; ++i) {
+    if (gt + 128 * i < nch) {
+      float f[VEC];
+      unpack16<T>(xv[i], f);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) ss += f[e] * f[e];
+    }
+  }
+  ss = warp_sum(ss);
+  if ((gt & 31) == 0) red[gt >> 5] = ss;
+  bar();
+  const float tot = (red[0] + red[1]) + (red[2] + red[3]);
+  const float inv = 1.0f / sqrtf(tot / (float)d + eps);
+  uint4* out = reinterpret_cast<uint4*>(out_row);
+#pragma unroll
+  for (int i = 0; i < MAXC; ++i) {
+    const int c = gt + 128 * i;
+    if (c < nch) {
+      float f[VEC], gg[VEC];
+      unpack16<T>(xv[i], f);
+      unpack16<T>(gv[i], gg);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) f[e] = f[e] * inv * gg[e];
+      out[c] = pack16<T>(f);
+    }
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(128) rmsnorm_rows_kernel(const T* src, int src_is_cache,
                                                            const int32_t* idx, int tps, int N,
                                                            int M, int d, const T* gamma, float eps,
                                                            T* X, int* err) {
-  constexpr int VEC = 16 / sizeof(T);
   griddep_launch_dependents();
   griddep_wait();
   const int t = blockIdx.x;
@@ -74,47 +123,9 @@ __global__ void __launch_bounds__(128) rmsnorm_rows_kernel(const T* src, int src
   } else {
     row = (size_t)t;
   }
-  const uint4* x = reinterpret_cast<const uint4*>(src + row * d);
-  const uint4* g = reinterpret_cast<const uint4*>(gamma);
-  const int nch = d / VEC;
-  uint4 xv[kNormMaxChunks], gv[kNormMaxChunks];
-#pragma unroll
-  for (int i = 0; i < kNormMaxChunks; ++i) {
-    const int c = threadIdx.x + 128 * i;
-    if (c < nch) {
-      xv[i] = x[c];
-      gv[i] = g[c];
-    }
-  }
-  float ss = 0.f;
-#pragma unroll
-  for (int i = 0; i < kNormMaxChunks; ++i) {
-    if (threadIdx.x + 128 * i < nch) {
-      float f[VEC];
-      unpack16<T>(xv[i], f);
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) ss += f[e] * f[e];
-    }
-  }
   __shared__ float red[4];
-  ss = warp_sum(ss);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  const float tot = (red[0] + red[1]) + (red[2] + red[3]);
-  const float inv = 1.0f / sqrtf(tot / (float)d + eps);
-  uint4* out = reinterpret_cast<uint4*>(X + (size_t)t * d);
-#pragma unroll
-  for (int i = 0; i < kNormMaxChunks; ++i) {
-    const int c = threadIdx.x + 128 * i;
-    if (c < nch) {
-      float f[VEC], gg[VEC];
-      unpack16<T>(xv[i], f);
-      unpack16<T>(gv[i], gg);
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) f[e] = f[e] * inv * gg[e];
-      out[c] = pack16<T>(f);
-    }
-  }
+  rmsnorm_one_row<T, kNormMaxChunks>(src + row * d, gamma, d, eps, X + (size_t)t * d, threadIdx.x, red,
+                                     []() { __syncthreads(); });
 }
 
 cudaError_t launch_rmsnorm_rows(int dtype, const void* src, int src_is_cache, const int32_t* idx,
@@ -132,22 +143,36 @@ cudaError_t launch_rmsnorm_rows(int dtype, const void* src, int src_is_cache, co
 }
 
 // ---------------------------------------------------------------------------
-// Top-k select, one CTA of 1024 threads per sequence (N <= 8192).
+// Top-k select (per sequence; ties to the lowest index; indices ascending).
 //
 // Scores are non-negative floats, so their bit patterns order like the
-// values.  A 4-pass MSB-first radix select (8 bits per pass) finds the k-th
-// largest key T and how many keys equal to T are still needed (`need`).  A
-// token is selected if its key is > T, or == T and fewer than `need` equal
-// keys precede it by index (ties to the lowest index).  Block-wide exclusive
-// scans in index order then give each selected token its slot, so the index
-// set comes out ascending.  Finally P^c[I] <- a_hat[I], flattened over
-// (row, column) with several copies per thread in flight.
+// values (-0 and negatives are taken as 0).  Thread t of an NT-thread block
+// holds keys [t*E, t*E + E) in registers (E = ceil(N / NT) <= 8).  The k-th
+// largest key T, the largest value with #{key >= T} >= k, is found two bits
+// per round from the top: a round counts the keys >= each of the three
+// candidates T | d << b (d = 1, 2, 3) with warp reductions and one block
+// barrier, and keeps the largest candidate that still has k keys at or above
+// it.  One block-wide exclusive scan of each thread's counts of keys > T and
+// == T (packed into one int) then places every selected key: with
+// need = k - #{key > T}, a key == T is taken while fewer than `need` equal
+// keys precede it, and a taken key's slot is (#keys > T before it) +
+// min(#keys == T before it, need), so the list comes out ascending without a
+// sort.  Per-thread key counts stay below 2^16, so the packed sums cannot
+// carry.
 // ---------------------------------------------------------------------------
 constexpr int kTopkThreads = 1024;
-constexpr int kTopkPerThread = 8;  // N <= 8192
+constexpr int kSelMaxPerThread = 8;  // N <= 8 * block size
 
-// Exclusive scan of one int per thread across the block; returns the total.
+__device__ __forceinline__ uint32_t score_key(float v) {
+  const uint32_t bits = __float_as_uint(v);
+  return (bits & 0x80000000u) ? 0u : bits;
+}
+
+// Exclusive scan of one int per thread across an NT-thread block; `total`
+// gets the block sum.  warp_tot holds 33 ints.
+template <int NT>
 __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& total) {
+  constexpr int NW = NT / 32;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   int incl = v;
 #pragma unroll
@@ -158,7 +183,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& t
   if (lane == 31) warp_tot[wid] = incl;
   __syncthreads();
   if (wid == 0) {
-    int w = warp_tot[lane];
+    const int w = lane < NW ? warp_tot[lane] : 0;
     int wi = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -175,115 +200,97 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& t
   return res;
 }
 
+// Shared memory of block_select.
+template <int NT>
+struct SelectSmem {
+  unsigned cnt[2][NT / 32][3];
+  int warp_tot[33];
+};
+
+// list[0..k) (and idx_out, when not null) <- the selected indices, ascending.
+template <int NT>
+__device__ void block_select(const float* s, int N, int k, int32_t* list, int32_t* idx_out,
+                             SelectSmem<NT>& sm, int* err) {
+  constexpr int NW = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int E = (N + NT - 1) / NT;
+  const int i0 = tid * E;
+  uint32_t key[kSelMaxPerThread];
+#pragma unroll
+  for (int j = 0; j < kSelMaxPerThread; ++j)
+    key[j] = (j < E && i0 + j < N) ? score_key(s[i0 + j]) : 0u;  // 0 is below every candidate
+  uint32_t t = 0;
+#pragma unroll 1
+  for (int r = 0; r < 16; ++r) {
+    const int shift = 30 - 2 * r;  // bits (31, 30), (29, 28), ..., (1, 0)
+    const uint32_t c1 = t | (1u << shift), c2 = t | (2u << shift), c3 = t | (3u << shift);
+    unsigned n1 = 0, n2 = 0, n3 = 0;
+#pragma unroll
+    for (int j = 0; j < kSelMaxPerThread; ++j) {
+      n1 += key[j] >= c1 ? 1u : 0u;
+      n2 += key[j] >= c2 ? 1u : 0u;
+      n3 += key[j] >= c3 ? 1u : 0u;
+    }
+    n1 = __reduce_add_sync(0xffffffffu, n1);
+    n2 = __reduce_add_sync(0xffffffffu, n2);
+    n3 = __reduce_add_sync(0xffffffffu, n3);
+    if (lane == 0) {
+      sm.cnt[r & 1][wid][0] = n1;
+      sm.cnt[r & 1][wid][1] = n2;
+      sm.cnt[r & 1][wid][2] = n3;
+    }
+    __syncthreads();  // double-buffered counts: one barrier per round
+    unsigned s1 = 0, s2 = 0, s3 = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      s1 += sm.cnt[r & 1][w][0];
+      s2 += sm.cnt[r & 1][w][1];
+      s3 += sm.cnt[r & 1][w][2];
+    }
+    const unsigned kk = (unsigned)k;
+    t = s3 >= kk ? c3 : s2 >= kk ? c2 : s1 >= kk ? c1 : t;
+  }
+  int n_gt = 0, n_eq = 0;
+#pragma unroll
+  for (int j = 0; j < kSelMaxPerThread; ++j) {
+    const bool v = j < E && i0 + j < N;
+    n_gt += (v && key[j] > t) ? 1 : 0;
+    n_eq += (v && key[j] == t) ? 1 : 0;
+  }
+  int tot;
+  const int pre = block_exclusive_scan<NT>((n_gt << 16) | n_eq, sm.warp_tot, tot);
+  const int need = k - (tot >> 16);
+  if (tid == 0 && (tot >> 16) + min(tot & 0xffff, need) != k) report_error(err, DEVERR_SHAPE, 401);
+  int gb = pre >> 16, eb = pre & 0xffff;
+#pragma unroll
+  for (int j = 0; j < kSelMaxPerThread; ++j) {
+    if (!(j < E && i0 + j < N)) continue;
+    int slot = -1;
+    if (key[j] > t) {
+      slot = gb + min(eb, need);
+      ++gb;
+    } else if (key[j] == t) {
+      if (eb < need) slot = gb + eb;
+      ++eb;
+    }
+    if (slot >= 0 && slot < k) {
+      list[slot] = i0 + j;
+      if (idx_out) idx_out[slot] = i0 + j;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kTopkThreads) topk_select_kernel(const float* score, int N, int k,
                                                                    int32_t* idx_out,
                                                                    const float* a_hat,
                                                                    float* p_cache, int r, int* err) {
-  __shared__ int hist[256];
-  __shared__ int warp_tot[33];
-  __shared__ int sel_digit, sel_above;
-  __shared__ int32_t list[kTopkPerThread * kTopkThreads];
+  __shared__ SelectSmem<kTopkThreads> sm;
+  __shared__ int32_t list[kSelMaxPerThread * kTopkThreads];
   griddep_launch_dependents();
   griddep_wait();
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
-  const float* s = score + (size_t)b * N;
-  const int E = (N + kTopkThreads - 1) / kTopkThreads;
-  const int i0 = tid * E;
-
-  uint32_t key[kTopkPerThread];
-#pragma unroll
-  for (int j = 0; j < kTopkPerThread; ++j) {
-    const int i = i0 + j;
-    const uint32_t bits = (j < E && i < N) ? __float_as_uint(s[i]) : 0u;
-    key[j] = (bits & 0x80000000u) ? 0u : bits;  // s >= 0; -0 and negatives order as 0
-  }
-
-  uint32_t prefix = 0, mask = 0;
-  int need = k;
-#pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0;
-    __syncthreads();
-    // one shared-memory atomic per distinct digit per warp (scores cluster in
-    // a few top-byte values, so per-thread atomics would serialise)
-#pragma unroll
-    for (int j = 0; j < kTopkPerThread; ++j) {
-      const int i = i0 + j;
-      const bool act = j < E && i < N && (key[j] & mask) == prefix;
-      const unsigned am = __ballot_sync(0xffffffffu, act);
-      if (act) {
-        const unsigned dig = (key[j] >> shift) & 255u;
-        const unsigned peers = __match_any_sync(am, dig);
-        if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[dig], __popc(peers));
-      }
-    }
-    __syncthreads();
-    if (tid < 32) {
-      // lane l owns digits [8l, 8l+8); scan from the top digit downwards
-      int c[8], lsum = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) { c[j] = hist[tid * 8 + j]; lsum += c[j]; }
-      // suffix sum over lanes above this one (higher digits)
-      int suf = lsum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_down_sync(0xffffffffu, suf, o);
-        if (tid + o < 32) suf += n;
-      }
-      int above = suf - lsum;  // count in lanes with higher digits
-      // the lane whose range contains the boundary
-      if (above < need && need <= suf) {
-        int acc = above;
-#pragma unroll
-        for (int j = 7; j >= 0; --j) {
-          if (acc < need && need <= acc + c[j]) { sel_digit = tid * 8 + j; sel_above = acc; }
-          acc += c[j];
-        }
-      }
-    }
-    __syncthreads();
-    prefix |= (uint32_t)sel_digit << shift;
-    mask |= 255u << shift;
-    need -= sel_above;
-    __syncthreads();
-  }
-  const uint32_t T = prefix;
-
-  // selected = key > T, or key == T among the first `need` equal keys by index
-  int n_eq = 0;
-#pragma unroll
-  for (int j = 0; j < kTopkPerThread; ++j) {
-    const int i = i0 + j;
-    if (j < E && i < N && key[j] == T) ++n_eq;
-  }
-  int tot;
-  int eq_before = block_exclusive_scan(n_eq, warp_tot, tot);
-  int flags = 0, n_sel = 0;
-#pragma unroll
-  for (int j = 0; j < kTopkPerThread; ++j) {
-    const int i = i0 + j;
-    if (j < E && i < N) {
-      bool sel = key[j] > T;
-      if (key[j] == T) {
-        sel = eq_before < need;
-        ++eq_before;
-      }
-      if (sel) { flags |= 1 << j; ++n_sel; }
-    }
-  }
-  int slot = block_exclusive_scan(n_sel, warp_tot, tot);
-  if (tid == 0 && tot != k) report_error(err, DEVERR_SHAPE, 401);
-#pragma unroll
-  for (int j = 0; j < kTopkPerThread; ++j) {
-    if (flags & (1 << j)) {
-      if (slot < k) {
-        list[slot] = i0 + j;
-        idx_out[(size_t)b * k + slot] = i0 + j;
-      }
-      ++slot;
-    }
-  }
+  block_select<kTopkThreads>(score + (size_t)b * N, N, k, list, idx_out + (size_t)b * k, sm, err);
   __syncthreads();
   // P^c[b, I] <- a_hat[b, I], flattened over (selected row, 16-byte chunk):
   // up to kScatterBatch loads per thread in flight before any store
@@ -328,9 +335,71 @@ __global__ void __launch_bounds__(kTopkThreads) topk_select_kernel(const float* 
 cudaError_t launch_topk_select(const float* score, int B, int N, int k, int32_t* idx,
                                const float* a_hat, float* p_cache, int r, int* err,
                                cudaStream_t stream) {
-  if (N > kTopkThreads * kTopkPerThread || k < 1 || k > N) return cudaErrorInvalidValue;
+  if (N > kTopkThreads * kSelMaxPerThread || k < 1 || k > N) return cudaErrorInvalidValue;
   return launch_k(topk_select_kernel, dim3(B), dim3(kTopkThreads), 0, stream, score, N, k, idx,
                   a_hat, p_cache, r, err);
+}
+
+// ---------------------------------------------------------------------------
+// Select + gather + RMSNorm in one launch (the cached layer step): CTA (c, b)
+// runs the top-k of sequence b itself (its scores are a few KB, and every
+// CTA of the sequence computes the same index set), then each group
+// of 128 threads takes one selected row j = 2c + group: writes idx[b, j], copies the
+// proxy row a_hat -> P^c, and writes X[b*k + j] = RMSNorm(H[b, I_j]).  The
+// select and the row arithmetic are the ones of the two separate kernels, so
+// the results are bit-identical to theirs.
+// ---------------------------------------------------------------------------
+constexpr int kSelThreads = 256;
+constexpr int kSelRows = kSelThreads / 128;               // selected rows per CTA
+constexpr int kSelMaxChunks = 4;                          // d <= 512 16-byte chunks
+constexpr int kSelMaxN = kSelThreads * kSelMaxPerThread;  // 2048 scores
+
+template <typename T>
+__global__ void __launch_bounds__(kSelThreads, 2) select_norm_kernel(
+    const float* score, int N, int k, int32_t* idx_out, const float* a_hat, float* p_cache, int r,
+    const T* H, const T* gamma, float eps, int d, T* X, int* err) {
+  __shared__ SelectSmem<kSelThreads> sm;
+  __shared__ int32_t list[kSelMaxN];
+  __shared__ float red[kSelRows][4];
+  griddep_launch_dependents();
+  griddep_wait();
+  const int c = blockIdx.x, b = blockIdx.y;
+  block_select<kSelThreads>(score + (size_t)b * N, N, k, list, nullptr, sm, c == 0 ? err : nullptr);
+  __syncthreads();
+  const int g = threadIdx.x >> 7, gt = threadIdx.x & 127;
+  const int j = c * kSelRows + g;
+  if (j >= k) return;  // whole groups only: the row barriers below are per group
+  const int pos = list[j];
+  const size_t row = (size_t)b * N + pos;
+  if (gt == 0) idx_out[(size_t)b * k + j] = pos;
+  if ((r & 3) == 0) {
+    const float4* src = reinterpret_cast<const float4*>(a_hat) + row * (r / 4);
+    float4* dst = reinterpret_cast<float4*>(p_cache) + row * (r / 4);
+    for (int q = gt; q < r / 4; q += 128) dst[q] = src[q];
+  } else {
+    for (int q = gt; q < r; q += 128) p_cache[row * r + q] = a_hat[row * r + q];
+  }
+  rmsnorm_one_row<T, kSelMaxChunks>(H + row * d, gamma, d, eps, X + ((size_t)b * k + j) * d, gt, red[g],
+                                    [g]() { asm volatile("bar.sync %0, 128;" ::"r"(g + 1) : "memory"); });
+}
+
+bool select_norm_supported(int dtype, int N, int d) {
+  const int vec = dtype == 1 ? 8 : 4;
+  return N <= kSelMaxN && d % vec == 0 && d / vec <= 128 * kSelMaxChunks;
+}
+
+cudaError_t launch_select_norm(int dtype, const float* score, int B, int N, int k, int32_t* idx,
+                               const float* a_hat, float* p_cache, int r, const void* H,
+                               const void* gamma, float eps, int d, void* X, int* err,
+                               cudaStream_t stream) {
+  if (!select_norm_supported(dtype, N, d) || k < 1 || k > N || !p_cache) return cudaErrorInvalidValue;
+  const dim3 grid((k + kSelRows - 1) / kSelRows, B);
+  if (dtype == 1)
+    return launch_k(select_norm_kernel<__nv_bfloat16>, grid, dim3(kSelThreads), 0, stream, score, N, k,
+                    idx, a_hat, p_cache, r, (const __nv_bfloat16*)H, (const __nv_bfloat16*)gamma, eps, d,
+                    (__nv_bfloat16*)X, err);
+  return launch_k(select_norm_kernel<float>, grid, dim3(kSelThreads), 0, stream, score, N, k, idx, a_hat,
+                  p_cache, r, (const float*)H, (const float*)gamma, eps, d, (float*)X, err);
 }
 
 // ---------------------------------------------------------------------------

@@ -130,16 +130,44 @@ def test_bf16_wide_weight_tiles(monkeypatch, nacc, B, N, k):
     _step(lp, cache, ocs, H2, k)
 
 
-@pytest.mark.parametrize("B,N,k", [(1, 2048, 200), (2, 1000, 62), (1, 1536, 129)])
+@pytest.mark.parametrize("B,N,k", [(1, 2048, 200), (2, 1000, 62), (1, 1536, 129), (1, 3000, 200)])
 def test_bf16_split_key_attention(B, N, k):
     # long caches: the keys of each query tile are split over a cluster of 8,
-    # 4 and 4 CTAs (2, 2 and 3 key tiles each; N=1000 ends in a partial key
-    # tile), with one or two query tiles, the second holding 72 or 1 rows
+    # 4, 4 and 8 CTAs (2, 2, 3 and 3 key tiles each; N=1000 and N=3000 end in
+    # a partial key tile), with one or two query tiles, the second holding 72
+    # or 1 rows.  N=3000 also takes the radix top-k (more than 2048 scores).
     lp = LayerPair(spa, SMALL_BF16, seed=50 + k, dtype=spa.SPA_BF16, max_B=B, max_N=N, std=0.05)
     H = synth.hidden_states(B, N, 256, seed=k + 7, bf16=True)
     cache, ocs = _run_fill(lp, H)
     H2, _ = synth.drift_rows(H, 0.05, 0.5, seed=k + 8, bf16=True)  # fewer drifted rows than k
     _step(lp, cache, ocs, H2, k)
+
+
+@pytest.mark.parametrize("bf16,B,N,k", [(False, 2, 64, 16), (True, 2, 1000, 62), (True, 1, 300, 257)])
+def test_layer_step_equals_select_then_partial_block(bf16, B, N, k):
+    # spa_layer_step selects, gathers and normalises in one launch; its
+    # results must be bit-identical to spa_proxy_select + spa_partial_block
+    shape = SMALL_BF16 if bf16 else synth.TINY_LAYER
+    dtype = spa.SPA_BF16 if bf16 else spa.SPA_F32
+    lp = LayerPair(spa, shape, seed=60 + k, dtype=dtype, max_B=B, max_N=N, std=0.05)
+    H = synth.hidden_states(B, N, shape.d, seed=k + 9, bf16=bf16)
+    H2, _ = synth.drift_rows(H, 0.3, 0.5, seed=k + 10, bf16=bf16)
+    Hd, H2d = lp.to_dev(H), lp.to_dev(H2)
+    outs = []
+    for fused in (True, False):
+        cache = lp.cache(B, N)
+        spa.spa_full_block(lp.layer, Hd, cache, True)
+        idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
+        if fused:
+            spa.spa_layer_step(lp.layer, H2d, cache, k, idx)
+        else:
+            spa.spa_proxy_select(lp.layer, H2d, cache, k, idx)
+            spa.spa_partial_block(lp.layer, H2d, idx, k, cache)
+        lp.ws.check()
+        x = lp.ws.view("x", (B * k, shape.d), spa.torch_dtype(dtype)).clone()
+        outs.append((idx.clone(), x, cache.k.clone(), cache.v.clone(), cache.h.clone(), cache.p.clone()))
+    for name, a, b in zip(("idx", "X", "K^c", "V^c", "H^c", "P^c"), *outs):
+        assert torch.equal(a, b), name
 
 
 def test_bf16_zero_drift_selects_lowest_indices():
