@@ -146,11 +146,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
       : "memory");
 }
-// 128 consecutive TMEM columns of this thread's lane.
-__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float (&v)[128]) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) tmem_ld32(taddr + (uint32_t)(32 * q), *reinterpret_cast<float(*)[32]>(&v[32 * q]));
-}
 // Bounded wait that ignores the abort flag (copies/MMAs in flight after an abort).
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, int* err, int site) {
   const uint32_t a = smem_u32(bar);
@@ -171,6 +166,41 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Rows [r0, r0 + 128/S) of the cluster's S split partials (unnormalised O in
+// each CTA's shared memory, 16-byte chunk c of row r at chunk c ^ (r % 32)),
+// weighted by w[row][q] and summed in split order, to bf16 rows of O (query
+// q0 + row, skipped past k).  128/S rows x 32 chunks = 4096/S tasks over the
+// block's 256 threads: 16/S tasks and 16 remote loads per thread, all issued
+// before any is used.
+template <int S>
+__device__ __forceinline__ void attn_cluster_combine(const float* sO, const float (*w)[8], int r0, int q0,
+                                                     int k, int d, __nv_bfloat16* Ob) {
+  constexpr int T = 16 / S;
+  float4 v[T][S];
+#pragma unroll
+  for (int t = 0; t < T; ++t) {
+    const int task = threadIdx.x + kAThreads * t;
+    const int rl = task >> 5, ch = task & 31, row = r0 + rl;
+    const uint32_t la = smem_u32(sO + row * 128 + ((ch ^ (row & 31)) << 2));
+#pragma unroll
+    for (int q = 0; q < S; ++q)
+      v[t][q] = q0 + row < k ? ld_dsmem_f4(mapa_shared(la, (uint32_t)q)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int t = 0; t < T; ++t) {
+    const int task = threadIdx.x + kAThreads * t;
+    const int rl = task >> 5, ch = task & 31, row = r0 + rl;
+    if (q0 + row >= k) continue;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < S; ++q) {
+      const float wq = w[rl][q];
+      acc.x += wq * v[t][q].x; acc.y += wq * v[t][q].y; acc.z += wq * v[t][q].z; acc.w += wq * v[t][q].w;
+    }
+    store4(Ob + (size_t)(q0 + row) * d + ch * 4, acc);
+  }
 }
 
 __global__ void __launch_bounds__(kAThreads, 1) attn_tc_kernel(const __grid_constant__ AttnTcParams p) {
@@ -297,16 +327,19 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_tc_kernel(const __grid_cons
       __syncwarp();
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
-      float x[128];
-      tmem_ld128(lane_base + (uint32_t)(sb * 128), x);
-      tc_fence_before();
-      mbar_arrive1(&s_empty[sb]);
+      // two passes over the scores in TMEM, 32 columns at a time (compact
+      // code and 32 registers instead of a 128-wide unrolled row): the row
+      // max, then the probabilities
       const int key0 = (kt0 + j) * kAT;
+      const uint32_t s_base = lane_base + (uint32_t)(sb * 128);
       float tmax = -INFINITY;
+#pragma unroll 1
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        float x[32];
+        tmem_ld32(s_base + (uint32_t)c0, x);
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        x[c] = (key0 + c < p.N) ? x[c] * p.scale_log2 : -INFINITY;
-        tmax = fmaxf(tmax, x[c]);
+        for (int c = 0; c < 32; ++c)
+          tmax = fmaxf(tmax, (key0 + c0 + c < p.N) ? x[c] * p.scale_log2 : -INFINITY);
       }
       // O and P may be rewritten only once the previous PV product is done
       const bool pv_ok = j == 0 || mbar_wait(&pv_done, (j - 1) & 1, &abort_flag, err, 607);
@@ -333,21 +366,31 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_tc_kernel(const __grid_cons
         m_used = m_new;
       }
       float sum = 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        float x[32];
+        tmem_ld32(s_base + (uint32_t)c0, x);
 #pragma unroll
-      for (int c = 0; c < 128; c += 8) {
-        uint32_t w[4];
+        for (int c = 0; c < 32; ++c) x[c] = (key0 + c0 + c < p.N) ? x[c] * p.scale_log2 : -INFINITY;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float a = exp2f(x[c + 2 * q] - m_used), bb = exp2f(x[c + 2 * q + 1] - m_used);
-          sum += a + bb;
-          __nv_bfloat162 v2 = __floats2bfloat162_rn(a, bb);
-          w[q] = *reinterpret_cast<uint32_t*>(&v2);
+        for (int c = 0; c < 32; c += 8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float a = exp2f(x[c + 2 * q] - m_used), bb = exp2f(x[c + 2 * q + 1] - m_used);
+            sum += a + bb;
+            __nv_bfloat162 v2 = __floats2bfloat162_rn(a, bb);
+            w[q] = *reinterpret_cast<uint32_t*>(&v2);
+          }
+          // 16-byte chunk of row `row`, 128-byte swizzle, two 64-key halves
+          const int chunk = (c0 + c) >> 3, half = chunk >> 3, cc = chunk & 7;
+          uint8_t* dst = sP + half * 16384 + row * 128 + ((cc ^ (row & 7)) << 4);
+          *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        // 16-byte chunk c/8 of row `row`, 128-byte swizzle, two 64-key halves
-        const int chunk = c >> 3, half = chunk >> 3, cc = chunk & 7;
-        uint8_t* dst = sP + half * 16384 + row * 128 + ((cc ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
       }
+      // the score buffer is free once both passes have read it
+      tc_fence_before();
+      mbar_arrive1(&s_empty[sb]);
       l += sum;
       fence_proxy_async_smem();
       tc_fence_before();
@@ -431,35 +474,39 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_tc_kernel(const __grid_cons
             wsum += __ldcg(p.part_ml + sl * 256 + 128 + row) * exp2f(__ldcg(p.part_ml + sl * 256 + row) - mm);
           }
           const float inv = wsum > 0.f ? 1.0f / wsum : 0.f;
-          // all 128 columns of one split per round: 32 independent loads in flight
-          float acc[128];
-#pragma unroll
-          for (int c = 0; c < 128; ++c) acc[c] = 0.f;
+          // 32 columns at a time, splits in order (8 loads in flight per split)
+          __nv_bfloat16* dst = p.O + ((size_t)b * p.k + qi) * d + (size_t)h * kAT;
 #pragma unroll 1
-          for (int q = 0; q < S; ++q) {
-            const size_t sl = grp * S + q;
-            const float pw = exp2f(__ldcg(p.part_ml + sl * 256 + row) - mm);
-            const float4* src = reinterpret_cast<const float4*>(p.part_o + sl * (kAT * kAT) + (size_t)row * kAT);
-            float4 v[32];
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            float acc[32];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) v[c] = __ldcg(src + c);
+            for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+#pragma unroll 1
+            for (int q = 0; q < S; ++q) {
+              const size_t sl = grp * S + q;
+              const float pw = exp2f(__ldcg(p.part_ml + sl * 256 + row) - mm);
+              const float4* src =
+                  reinterpret_cast<const float4*>(p.part_o + sl * (kAT * kAT) + (size_t)row * kAT + c0);
+              float4 v[8];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              acc[4 * c] += pw * v[c].x; acc[4 * c + 1] += pw * v[c].y;
-              acc[4 * c + 2] += pw * v[c].z; acc[4 * c + 3] += pw * v[c].w;
-            }
-          }
-          if (qi < p.k) {
-            __nv_bfloat16* dst = p.O + ((size_t)b * p.k + qi) * d + (size_t)h * kAT;
+              for (int c = 0; c < 8; ++c) v[c] = __ldcg(src + c);
 #pragma unroll
-            for (int c = 0; c < 128; c += 8) {
-              uint32_t w4[4];
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                __nv_bfloat162 v2 = __floats2bfloat162_rn(acc[c + 2 * q] * inv, acc[c + 2 * q + 1] * inv);
-                w4[q] = *reinterpret_cast<uint32_t*>(&v2);
+              for (int c = 0; c < 8; ++c) {
+                acc[4 * c] += pw * v[c].x; acc[4 * c + 1] += pw * v[c].y;
+                acc[4 * c + 2] += pw * v[c].z; acc[4 * c + 3] += pw * v[c].w;
               }
-              *reinterpret_cast<uint4*>(dst + c) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+            if (qi < p.k) {
+#pragma unroll
+              for (int c = 0; c < 32; c += 8) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  __nv_bfloat162 v2 = __floats2bfloat162_rn(acc[c + 2 * q] * inv, acc[c + 2 * q + 1] * inv);
+                  w4[q] = *reinterpret_cast<uint32_t*>(&v2);
+                }
+                *reinterpret_cast<uint4*>(dst + c0 + c) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+              }
             }
           }
           if (row == 0) p.sync[grp] = 0;  // ready for the next launch
@@ -508,27 +555,13 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_tc_kernel(const __grid_cons
           if (q < S) s_w[threadIdx.x][q] = w[q] * inv;
       }
       __syncthreads();
-      // one warp per row: 32 lanes x 4 columns, S remote loads in flight each
+      // one warp per row, 32 lanes x 4 columns; each thread has all of its
+      // 16 remote loads in flight at once
       const float* sO = reinterpret_cast<const float*>(sKV);
-      const int d = p.n_heads * kAT;
-      for (int task = threadIdx.x; task < RS * 32; task += kAThreads) {
-        const int rl = task >> 5, ch = task & 31, row = r0 + rl;
-        const int qi = qt * kAT + row;
-        if (qi >= p.k) continue;
-        const uint32_t la = smem_u32(sO + row * 128 + ((ch ^ (row & 31)) << 2));
-        float4 v[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (q < S) v[q] = ld_dsmem_f4(mapa_shared(la, (uint32_t)q));
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (q < S) {
-            const float wq = s_w[rl][q];
-            acc.x += wq * v[q].x; acc.y += wq * v[q].y; acc.z += wq * v[q].z; acc.w += wq * v[q].w;
-          }
-        store4(p.O + ((size_t)b * p.k + qi) * d + (size_t)h * kAT + ch * 4, acc);
-      }
+      __nv_bfloat16* Ob = p.O + (size_t)b * p.k * (p.n_heads * kAT) + (size_t)h * kAT;
+      if (S == 2) attn_cluster_combine<2>(sO, s_w, r0, qt * kAT, p.k, p.n_heads * kAT, Ob);
+      else if (S == 4) attn_cluster_combine<4>(sO, s_w, r0, qt * kAT, p.k, p.n_heads * kAT, Ob);
+      else attn_cluster_combine<8>(sO, s_w, r0, qt * kAT, p.k, p.n_heads * kAT, Ob);
     }
     cluster_sync();
   }
