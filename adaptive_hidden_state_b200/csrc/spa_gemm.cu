@@ -119,7 +119,7 @@ __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_e
       store4(reinterpret_cast<T*>(ep.out) + (size_t)t * ep.n_out + f, a);
     }
   } else if constexpr (MODE == EPI_QKV) {
-    constexpr int kUnrollQ = 2;  // four float4 operands per item
+    constexpr int kUnrollQ = 4;  // four float4 operands per item, all loads of 4 items in flight
     // Item = 4 rotary pairs (j..j+3, j+hd/2..j+hd/2+3) of one head of one row.
     const int hd = ep.head_dim, hh = hd / 2;
     const int items_per_head = hh / 4;
@@ -504,7 +504,7 @@ __device__ __forceinline__ void ws_load_weights(const TcWsParams& p, int n_tile,
   for (int a = 0; a < NACC; ++a) {
     int src, row;
     if (p.b_mode == B_GATEUP) {
-      const int hal = NACC / 2;
+      const int hal = NACC / 2 > 0 ? NACC / 2 : 1;  // gate/up blocks come in pairs (NACC >= 2)
       src = a < hal ? 0 : 1;
       row = n_tile * (FEAT / 2) + (a % hal) * 128;
     } else if (p.b_mode == B_CONCAT3) {
@@ -626,6 +626,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
       umma_commit(&empty_bar[s]);
     }
     umma_commit(&accum_bar);
+  } else if (warp >= 2) {
+    // idle during the main loop: fetch the first chunk's row indices now
+    griddep_wait();
+    stage_rows(p.ep, 0, 0, min(CHUNK, NT), s_rows, threadIdx.x - 64, kThreads - 64);
   }
   __syncwarp();
 
@@ -671,8 +675,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
       __syncthreads();
     }
     if (good && c0 + r0 < M) {
-      stage_rows(p.ep, c0, r0, r1, s_rows, threadIdx.x, kThreads);
-      __syncthreads();
+      if (c0 > 0) {  // the first chunk's rows were staged during the main loop
+        stage_rows(p.ep, c0, r0, r1, s_rows, threadIdx.x, kThreads);
+        __syncthreads();
+      }
       run_epilogue<MODE, FEAT, __nv_bfloat16>(tile, LD, r0, r1, c0, n_tile, p.ep, s_rows,
                                               threadIdx.x, kThreads);
     }
