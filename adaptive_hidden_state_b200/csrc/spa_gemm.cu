@@ -241,11 +241,41 @@ __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_e
 }
 
 // Rows [r0, r1) of the cluster's S partial tiles summed in the fixed order
-// 0..S-1 into this CTA's tile (all S loads of an element issued first).
+// 0..S-1 into this CTA's tile.  With S <= 4 a thread takes four 16-byte
+// items at once and issues all of their remote loads (up to 16) before using
+// any; with more splits, eight loads of one item at a time.
 template <int W>
 __device__ void cluster_reduce_rows(float* tile, int ld, int r0, int r1, int S, int tid, int nthr) {
   constexpr int C4 = W / 4;
-  for (int it = tid; it < (r1 - r0) * C4; it += nthr) {
+  const int total = (r1 - r0) * C4;
+  if (S <= 4) {
+    for (int base = tid; base < total; base += 4 * nthr) {
+      float4 v[4][4];
+      uint32_t local[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int it = base + u * nthr;
+        const int row = r0 + it / C4, c = (it % C4) * 4;
+        local[u] = smem_u32(tile + row * ld + c);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (it < total && q < S) v[u][q] = ld_dsmem_f4(mapa_shared(local[u], (uint32_t)q));
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int it = base + u * nthr;
+        if (it >= total) continue;
+        float4 acc = v[u][0];  // split 0 first, then 1..S-1 in order
+#pragma unroll
+        for (int q = 1; q < 4; ++q)
+          if (q < S) { acc.x += v[u][q].x; acc.y += v[u][q].y; acc.z += v[u][q].z; acc.w += v[u][q].w; }
+        const int row = r0 + it / C4, c = (it % C4) * 4;
+        *reinterpret_cast<float4*>(tile + row * ld + c) = acc;
+      }
+    }
+    return;
+  }
+  for (int it = tid; it < total; it += nthr) {
     const int row = r0 + it / C4, c = (it % C4) * 4;
     const uint32_t local = smem_u32(tile + row * ld + c);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -484,8 +514,8 @@ constexpr int kWsSmem = kWsRing + 1024;
 
 // Tokens per epilogue chunk: the fp32 chunk tile [tokens][FEAT + 4] reuses the ring.
 __host__ __device__ constexpr int ws_chunk(int nacc) {
-  return (kWsRing / ((nacc * 128 + 4) * 4)) / 32 * 32 < 128 ? (kWsRing / ((nacc * 128 + 4) * 4)) / 32 * 32
-                                                            : 128;
+  return (kWsRing / ((nacc * 128 + 4) * 4)) / 32 * 32 < 256 ? (kWsRing / ((nacc * 128 + 4) * 4)) / 32 * 32
+                                                            : 256;
 }
 
 __host__ __device__ inline int ws_stages(int nacc, int NT) {
@@ -538,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
   __shared__ __align__(8) uint64_t accum_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
-  __shared__ int2 s_rows[128];
+  __shared__ int2 s_rows[256];  // >= CHUNK
 
   griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -642,6 +672,35 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
   float* tile = reinterpret_cast<float*>(smem);
   const int M = p.ep.M;
   const int q4 = warp & 3, half = warp >> 2;
+  if constexpr (MODE == EPI_SWIGLU && NACC == 2) {
+    if (S == 1) {
+      // no reduction: thread (quadrant, lane) owns feature f, whose gate and
+      // up accumulators sit in the same TMEM lane; silu(g) * u goes straight
+      // from registers to A, 32 tokens per TMEM load (64-byte rows of 32
+      // features per warp store), with no shared-memory pass
+      if (good && nk > 0) {
+        const int f = n_tile * 128 + q4 * 32 + lane;
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.ep.out);
+        const uint32_t row_base = tmem + ((uint32_t)(q4 * 32) << 16);
+#pragma unroll 1
+        for (int c = 32 * half; c < NT; c += 64) {
+          float g[32], u[32];
+          tmem_ld32(row_base + (uint32_t)c, g);
+          tmem_ld32(row_base + (uint32_t)(NT + c), u);
+          if (f < p.ep.n_out) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c + j < M) out[(size_t)(c + j) * p.ep.n_out + f] = __float2bfloat16_rn(silu(g[j]) * u[j]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      if (warp == 0) tmem_dealloc(tmem, (uint32_t)p.tmem_cols);
+      return;
+    }
+  }
   for (int c0 = 0; c0 < NT; c0 += CHUNK) {
     const int nt = min(CHUNK, NT - c0);
     if (good) {
