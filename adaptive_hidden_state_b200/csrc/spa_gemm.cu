@@ -30,7 +30,7 @@ namespace spa {
 // global loads issued before any result is used, and the cache row of every
 // tile row (b, position in I) is staged in shared memory once per tile.
 // ---------------------------------------------------------------------------
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 8;
 
 // silu(g) = g / (1 + e^-g) with the fast exponential and reciprocal
 // intrinsics: relative error ~1e-6, far below the bf16 rounding of the result.

@@ -427,7 +427,10 @@ def main():
     prof_ms_step = p0.elapsed_time(p1) / K
 
     layer_ms = sum(prof[k][1] for k in LAYER_CLASSES) / K
-    us_per_layer = layer_ms * 1e3 / c["L"]
+    # us per layer step from the graph-timed step: (step - LM head - embed/argmax) / L; the
+    # event-profiled per-kernel sum (no overlap between kernels) is reported beside it
+    us_per_layer = (ms_step - (prof["lmhead"][1] + prof["misc"][1]) / K) * 1e3 / c["L"]
+    us_per_layer_kernels = layer_ms * 1e3 / c["L"]
     dom = max(LAYER_CLASSES + ["lmhead"], key=lambda k: prof[k][1])
     n_l, ms_l, by_l, fl_l = prof[dom]
     hbm, tf_burst, tf_sus, peak_kind = load_peaks()
@@ -516,6 +519,7 @@ def main():
                            "launch": "one CUDA graph replay per decode step",
                            "budget_k": model.k},
                 "us_per_layer": us_per_layer,
+                "us_per_layer_kernel_sum": us_per_layer_kernels,
                 "step_roofline_ms": step_roof_ms,
                 "step_roofline_frac": step_roof_ms / ms_step,
                 "vanilla_rho1": {"tokens_per_s": world * B * u / (v_ms / 1e3), "ms_per_step": v_ms,
