@@ -1,0 +1,192 @@
+"""GPU parity at the workloads' full sizes, in the launch configuration the
+benchmark times: the 32-layer LLaDA-8B-shaped bf16 decode loop (d=4096,
+32x128 heads, F=12288, vocab 126464, r=128) at B=1, N=1024 (256 prompt ids,
+2 unmaskings per step) and at B=8, N=2048 (512 prompt ids, 4 unmaskings per
+step), piecewise-Gaussian budget rho_p=0.25, l_p=12, rho_1=rho_L=0.06, with
+seeded random weights of that shape (W_v with the i^-0.8 power-law spectrum).
+
+The oracle cannot run whole steps at these sizes, so the checks are sampled
+and by property:
+- one graph-replayed cached step equals the same step launched directly, bit
+  for bit (all 32 layers' caches and the unmasked ids);
+- at a few layers of a later step (the first, the widest k = 256 / 512, the
+  last) and a few sequences, the layer's input and caches are copied before
+  the layer runs, and the oracle's proxy scores, top-k and cached block on
+  them are compared with the GPU's: the index set (exact, or valid within the
+  score margin), Q, O, H1, A and the rewritten K^c, V^c, H^c, P^c rows, with
+  the bf16 tolerance; the rows outside I stay bit-identical.
+Layers run through spa_layer_step, the call spa_decode_step makes."""
+import gc
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from adaptive_hidden_state_b200 import synth
+from spa_testutil import assert_close, assert_index_set, np64
+
+pytestmark = pytest.mark.gpu
+
+spa = pytest.importorskip("adaptive_hidden_state_b200.spa")
+
+D, NH, HD, F, R, VOCAB, L = 4096, 32, 128, 12288, 128, 126464, 32
+RHO = dict(rho_p=0.25, l_p=12, rho_1=0.06, rho_L=0.06)
+NAMES = ["wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down", "attn_norm", "ffn_norm"]
+
+
+def _build(B, N, seed):
+    dev = "cuda"
+    g = torch.Generator(device=dev).manual_seed(seed)
+
+    def randn(shape, std):
+        return (torch.randn(shape, generator=g, device=dev, dtype=torch.float32) * std).to(torch.bfloat16)
+
+    def haar(n):
+        q, rr = torch.linalg.qr(torch.randn((n, n), generator=g, device=dev, dtype=torch.float32))
+        return q * torch.sign(torch.diagonal(rr))[None, :]
+
+    sigma = torch.arange(1, D + 1, device=dev, dtype=torch.float32) ** -0.8
+    desc = spa.LayerDesc(d=D, n_heads=NH, head_dim=HD, ffn=F, r=R, dtype=spa.SPA_BF16,
+                         rms_eps=1e-5, rope_theta=1e4)
+    ws = spa.Workspace(desc, B, N)
+    ones = torch.ones(D, device=dev, dtype=torch.bfloat16)
+    layers, caches, weights = [], [], []
+    for _ in range(L):
+        U, Vm = haar(D), haar(D)
+        wv = ((U * sigma[None, :]) @ Vm.T).to(torch.bfloat16)
+        w_r = (sigma[:R, None] * Vm[:, :R].T).float().cpu()
+        del U, Vm
+        w = {"wq": randn((D, D), .02), "wk": randn((D, D), .02), "wv": wv, "wo": randn((D, D), .02),
+             "w_gate": randn((F, D), .02), "w_up": randn((F, D), .02), "w_down": randn((D, F), .02),
+             "attn_norm": ones, "ffn_norm": ones}
+        layers.append(spa.Layer(desc, w, ws, w_r_host=w_r))
+        weights.append(w)
+        caches.append(spa.Cache(B, N, D, R, spa.SPA_BF16))
+    embed = randn((VOCAB, D), 1.0)
+    lm_head = randn((VOCAB, D), .02)
+    h0 = torch.zeros((B, N, D), device=dev, dtype=torch.bfloat16)
+    model = spa.Model(layers, caches, h0, embed, ones, lm_head, VOCAB, B, N, RHO["rho_p"], RHO["l_p"],
+                      RHO["rho_1"], RHO["rho_L"])
+    return model, ws, layers, caches, weights, (embed, lm_head, h0, ones)
+
+
+def _oracle_layer(layer, w):
+    host = {k: w[k].float().cpu().numpy() for k in NAMES}
+    W_r = layer.proxy_weights().numpy().astype(np.float64)  # the library's bf16-stored proxy
+    return O.OracleLayer.from_weights(host, W_r, NH, 1e-5, 1e4)
+
+
+def _snapshot(caches, l):
+    c = caches[l]
+    return [t.clone() for t in (c.k, c.v, c.h, c.p)]
+
+
+def _check_layer(lp_args, H_in, snap, caches, l, k, idx, ws, seqs):
+    layer, w = lp_args
+    ol = _oracle_layer(layer, w)
+    B = H_in.shape[0]
+    M = B * k
+    views = {name: ws.view(name, (M, width), torch.bfloat16).clone()
+             for name, width in (("q", D), ("o", D), ("h1", D), ("a", F))}
+    I_all = idx.cpu().numpy()
+    c = caches[l]
+    after = [np64(t) for t in (c.k, c.v, c.h)]
+    p_after = np64(c.p)
+    before = [np64(t) for t in snap[:3]]
+    p_before = np64(snap[3])
+    for b in seqs:
+        Hb = np64(H_in[b])
+        cache_b = O.LayerCache(before[0][b].copy(), before[1][b].copy(), before[2][b].copy(), p_before[b].copy())
+        a_hat, s = O.proxy_identify(Hb, ol.W_r, cache_b.P_c)
+        I_ref = O.select_topk(s, k)
+        I = I_all[b].astype(np.int64)
+        assert_index_set(I, s, k, I_ref, f"layer {l} seq {b} I")
+        cache_b.P_c[I] = a_hat[I]
+        out = O.partial_block(ol, Hb, I, cache_b)
+        rows = slice(b * k, (b + 1) * k)
+        for name, key in (("q", "Q"), ("o", "O"), ("h1", "H1"), ("a", "A")):
+            assert_close(views[name][rows], out[key], True, f"layer {l} seq {b} {key}")
+        for j, (name, ref) in enumerate((("K^c", cache_b.K_c), ("V^c", cache_b.V_c), ("H^c", cache_b.H_c))):
+            assert_close(after[j][b][I], ref[I], True, f"layer {l} seq {b} {name}[I]")
+            keep = np.ones(after[j].shape[1], bool)
+            keep[I] = False
+            assert np.array_equal(after[j][b][keep], before[j][b][keep]), f"layer {l} seq {b} {name} outside I"
+        assert np.max(np.abs(p_after[b][I] - cache_b.P_c[I])) < 2e-3, f"layer {l} seq {b} P^c[I]"
+
+
+def _run(B, N, n_prompt, u, sample_layers, seqs, check_graph):
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        _run_on_stream(B, N, n_prompt, u, sample_layers, seqs, check_graph)
+    stream.synchronize()
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def _run_on_stream(B, N, n_prompt, u, sample_layers, seqs, check_graph):
+    model, ws, layers, caches, weights, keep = _build(B, N, seed=1234 + B)
+    steps = 4
+    job = synth.decode_inputs(B=B, N=N, n_prompt=n_prompt, vocab=VOCAB, steps=steps, u=u, seed=77 + B)
+    toks = torch.from_numpy(job.tokens.astype(np.int32)).cuda()
+    pos = [torch.from_numpy(p.astype(np.int32)).cuda() for p in job.positions]
+    tok_out = torch.empty((steps, B, u), dtype=torch.int32, device="cuda")
+    model.embed_tokens(toks)
+    spa.spa_decode_step(model, pos[0], None, u, 1, tok_out[0])
+    spa.spa_decode_step(model, pos[1], None, u, 0, tok_out[1])
+    ws.check()
+    h0 = keep[2]
+
+    if check_graph:
+        # the graph-replayed step against the same step launched directly
+        state = [h0.clone()] + [t.clone() for c in caches for t in (c.k, c.v, c.h, c.p)]
+        pos_buf = torch.empty((B, u), dtype=torch.int32, device="cuda")
+        tok_buf = torch.empty((B, u), dtype=torch.int32, device="cuda")
+        spa.spa_decode_graph_capture(model, pos_buf, None, u, tok_buf)
+        pos_buf.copy_(pos[2])
+        spa.spa_decode_graph_launch(model)
+        torch.cuda.synchronize()
+        ws.check()
+        graph_out = [tok_buf.clone(), h0.clone()] + [t.clone() for c in caches for t in (c.k, c.v, c.h, c.p)]
+        h0.copy_(state[0])
+        for i, c in enumerate(caches):
+            for j, t in enumerate((c.k, c.v, c.h, c.p)):
+                t.copy_(state[1 + 4 * i + j])
+        del state
+        spa.spa_decode_step(model, pos[2], None, u, 0, tok_out[2])
+        ws.check()
+        direct = [tok_out[2], h0] + [t for c in caches for t in (c.k, c.v, c.h, c.p)]
+        for i, (a, b) in enumerate(zip(graph_out, direct)):
+            assert torch.equal(a, b), f"graph replay differs from direct launch (tensor {i})"
+        del graph_out
+    else:
+        spa.spa_decode_step(model, pos[2], None, u, 0, tok_out[2])
+        ws.check()
+    torch.cuda.synchronize()
+
+    # step 3, layer by layer, with sampled oracle checks
+    for l in range(L):
+        H = h0 if l == 0 else caches[l - 1].h
+        k = model.k[l]
+        Ik = torch.empty((B, k), dtype=torch.int32, device="cuda")
+        if l in sample_layers:
+            H_in = H.clone()
+            snap = _snapshot(caches, l)
+            spa.spa_layer_step(layers[l], H, caches[l], k, Ik)
+            ws.check()
+            torch.cuda.synchronize()
+            _check_layer((layers[l], weights[l]), H_in, snap, caches, l, k, Ik, ws, seqs)
+            del H_in, snap
+            gc.collect()
+        else:
+            spa.spa_layer_step(layers[l], H, caches[l], k, Ik)
+    ws.check()
+
+
+def test_llada_decode_full_size_b1_n1024():
+    _run(B=1, N=1024, n_prompt=256, u=2, sample_layers=(0, 11, 31), seqs=(0,), check_graph=True)
+
+
+def test_llada_decode_full_size_b8_n2048():
+    # B*k reaches 4096 tokens at the widest layers: the tiled GEMM path
+    _run(B=8, N=2048, n_prompt=512, u=4, sample_layers=(0, 11), seqs=(0, 5), check_graph=False)
