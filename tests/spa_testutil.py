@@ -101,3 +101,49 @@ class LayerPair:
 
     def to_dev(self, H: np.ndarray) -> torch.Tensor:
         return torch.from_numpy(np.ascontiguousarray(H)).to("cuda", self.spa.torch_dtype(self.dtype))
+
+
+def snapshot_cache(c) -> list:
+    """Device copies of one layer cache's K^c, V^c, H^c, P^c."""
+    return [t.clone() for t in (c.k, c.v, c.h, c.p)]
+
+
+def check_layer_step(spa, layer, w: dict, H_in, snap, cache, k, idx, ws, seqs, what):
+    """A cached layer step the GPU has just run, checked for the sequences in
+    `seqs` against the oracle on the same inputs: H_in (device copy of the
+    step's input), snap (snapshot_cache before the step), the layer's weights
+    w (device tensors) and its stored proxy.  Index set (exact or valid within
+    the score margin), Q, O, H1, A, the rewritten K^c/V^c/H^c/P^c rows, and the
+    other rows bit-identical to the snapshot."""
+    host = {n: w[n].float().cpu().numpy() for n in NAMES}
+    d, F, nh = layer.desc.d, layer.desc.ffn, layer.desc.n_heads
+    W_r = layer.proxy_weights().numpy().astype(np.float64)
+    ol = O.OracleLayer.from_weights(host, W_r, nh, layer.desc.rms_eps, layer.desc.rope_theta)
+    B = H_in.shape[0]
+    M = B * k
+    views = {name: ws.view(name, (M, width), torch.bfloat16).clone()
+             for name, width in (("q", d), ("o", d), ("h1", d), ("a", F))}
+    I_all = idx.cpu().numpy()
+    after = [np64(t) for t in (cache.k, cache.v, cache.h)]
+    p_after = np64(cache.p)
+    before = [np64(t) for t in snap[:3]]
+    p_before = np64(snap[3])
+    for b in seqs:
+        Hb = np64(H_in[b])
+        cache_b = O.LayerCache(before[0][b].copy(), before[1][b].copy(), before[2][b].copy(),
+                               p_before[b].copy())
+        a_hat, s = O.proxy_identify(Hb, ol.W_r, cache_b.P_c)
+        I_ref = O.select_topk(s, k)
+        I = I_all[b].astype(np.int64)
+        assert_index_set(I, s, k, I_ref, f"{what} seq {b} I")
+        cache_b.P_c[I] = a_hat[I]
+        out = O.partial_block(ol, Hb, I, cache_b)
+        rows = slice(b * k, (b + 1) * k)
+        for name, key in (("q", "Q"), ("o", "O"), ("h1", "H1"), ("a", "A")):
+            assert_close(views[name][rows], out[key], True, f"{what} seq {b} {key}")
+        for j, (name, ref) in enumerate((("K^c", cache_b.K_c), ("V^c", cache_b.V_c), ("H^c", cache_b.H_c))):
+            assert_close(after[j][b][I], ref[I], True, f"{what} seq {b} {name}[I]")
+            keep = np.ones(after[j].shape[1], bool)
+            keep[I] = False
+            assert np.array_equal(after[j][b][keep], before[j][b][keep]), f"{what} seq {b} {name} outside I"
+        assert np.max(np.abs(p_after[b][I] - cache_b.P_c[I])) < 2e-3, f"{what} seq {b} P^c[I]"

@@ -24,7 +24,7 @@ import torch
 
 import oracle as O
 from adaptive_hidden_state_b200 import synth
-from spa_testutil import assert_close, assert_index_set, np64
+from spa_testutil import check_layer_step, snapshot_cache
 
 pytestmark = pytest.mark.gpu
 
@@ -32,7 +32,6 @@ spa = pytest.importorskip("adaptive_hidden_state_b200.spa")
 
 D, NH, HD, F, R, VOCAB, L = 4096, 32, 128, 12288, 128, 126464, 32
 RHO = dict(rho_p=0.25, l_p=12, rho_1=0.06, rho_L=0.06)
-NAMES = ["wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down", "attn_norm", "ffn_norm"]
 
 
 def _build(B, N, seed):
@@ -69,50 +68,6 @@ def _build(B, N, seed):
     model = spa.Model(layers, caches, h0, embed, ones, lm_head, VOCAB, B, N, RHO["rho_p"], RHO["l_p"],
                       RHO["rho_1"], RHO["rho_L"])
     return model, ws, layers, caches, weights, (embed, lm_head, h0, ones)
-
-
-def _oracle_layer(layer, w):
-    host = {k: w[k].float().cpu().numpy() for k in NAMES}
-    W_r = layer.proxy_weights().numpy().astype(np.float64)  # the library's bf16-stored proxy
-    return O.OracleLayer.from_weights(host, W_r, NH, 1e-5, 1e4)
-
-
-def _snapshot(caches, l):
-    c = caches[l]
-    return [t.clone() for t in (c.k, c.v, c.h, c.p)]
-
-
-def _check_layer(lp_args, H_in, snap, caches, l, k, idx, ws, seqs):
-    layer, w = lp_args
-    ol = _oracle_layer(layer, w)
-    B = H_in.shape[0]
-    M = B * k
-    views = {name: ws.view(name, (M, width), torch.bfloat16).clone()
-             for name, width in (("q", D), ("o", D), ("h1", D), ("a", F))}
-    I_all = idx.cpu().numpy()
-    c = caches[l]
-    after = [np64(t) for t in (c.k, c.v, c.h)]
-    p_after = np64(c.p)
-    before = [np64(t) for t in snap[:3]]
-    p_before = np64(snap[3])
-    for b in seqs:
-        Hb = np64(H_in[b])
-        cache_b = O.LayerCache(before[0][b].copy(), before[1][b].copy(), before[2][b].copy(), p_before[b].copy())
-        a_hat, s = O.proxy_identify(Hb, ol.W_r, cache_b.P_c)
-        I_ref = O.select_topk(s, k)
-        I = I_all[b].astype(np.int64)
-        assert_index_set(I, s, k, I_ref, f"layer {l} seq {b} I")
-        cache_b.P_c[I] = a_hat[I]
-        out = O.partial_block(ol, Hb, I, cache_b)
-        rows = slice(b * k, (b + 1) * k)
-        for name, key in (("q", "Q"), ("o", "O"), ("h1", "H1"), ("a", "A")):
-            assert_close(views[name][rows], out[key], True, f"layer {l} seq {b} {key}")
-        for j, (name, ref) in enumerate((("K^c", cache_b.K_c), ("V^c", cache_b.V_c), ("H^c", cache_b.H_c))):
-            assert_close(after[j][b][I], ref[I], True, f"layer {l} seq {b} {name}[I]")
-            keep = np.ones(after[j].shape[1], bool)
-            keep[I] = False
-            assert np.array_equal(after[j][b][keep], before[j][b][keep]), f"layer {l} seq {b} {name} outside I"
-        assert np.max(np.abs(p_after[b][I] - cache_b.P_c[I])) < 2e-3, f"layer {l} seq {b} P^c[I]"
 
 
 def _run(B, N, n_prompt, u, sample_layers, seqs, check_graph):
@@ -171,11 +126,11 @@ def _run_on_stream(B, N, n_prompt, u, sample_layers, seqs, check_graph):
         Ik = torch.empty((B, k), dtype=torch.int32, device="cuda")
         if l in sample_layers:
             H_in = H.clone()
-            snap = _snapshot(caches, l)
+            snap = snapshot_cache(caches[l])
             spa.spa_layer_step(layers[l], H, caches[l], k, Ik)
             ws.check()
             torch.cuda.synchronize()
-            _check_layer((layers[l], weights[l]), H_in, snap, caches, l, k, Ik, ws, seqs)
+            check_layer_step(spa, layers[l], weights[l], H_in, snap, caches[l], k, Ik, ws, seqs, f"layer {l}")
             del H_in, snap
             gc.collect()
         else:
