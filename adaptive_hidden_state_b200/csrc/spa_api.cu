@@ -223,6 +223,18 @@ struct spa_model {
   CUtensorMap tm_lm;
   cudaGraphExec_t graph = nullptr;  // a captured cached decode step
   int graph_u = 0;
+  // incremental proxy: per layer, the unit proxy of every row's current input
+  // and its drift score, kept across steps; only rows whose input changed are
+  // projected again (the previous layer's index set, or the unmasked rows at
+  // layer 0), whose new input rows the previous kernels leave compact in chg_rows
+  bool inc = false;           // incremental proxy enabled
+  bool inc_valid = false;     // ahat_all / score_all / chg_rows describe the current state
+  int graph_inc = 0;          // the captured step: 0 plain, 1 proxy state refreshed, 2 incremental
+  float* ahat_all = nullptr;  // [L, B, N, r]
+  float* score_all = nullptr; // [L, B, N]
+  void* chg_rows = nullptr;   // [B*N, d] compact changed rows (layer input of the next proxy)
+  int32_t* chg0_idx = nullptr;  // [B*N] rows changed at layer 0 (the last unmasked positions)
+  int chg0_u = 0;
 };
 
 static int check_desc(const spa_layer_desc* d) {
@@ -596,12 +608,17 @@ static int check_cache(const spa_layer* L, const spa_layer_cache* c) {
 }
 
 // Phase 1: proxy GEMM with the fused norm / score epilogue (or the P^c fill).
-static int run_proxy(spa_layer* L, const void* H, const spa_layer_cache* c, float* score, int fill,
-                     cudaStream_t s) {
-  const int M = c->B * c->N, d = L->desc.d, r = L->desc.r;
-  EpiParams ep = base_epi(L, M, c->N, c->N, nullptr);
+// X holds tps token rows per sequence: every cache row (rows == null, tps = N)
+// or the rows listed in `rows` ([B, tps] cache rows), compact.  a_hat and
+// score are [B*N, r] and [B*N], written at the tokens' cache rows.
+static int run_proxy_rows(spa_layer* L, const void* H, const int32_t* rows, int tps,
+                          const spa_layer_cache* c, float* a_hat, float* score, int fill,
+                          cudaStream_t s) {
+  const int M = c->B * tps, d = L->desc.d, r = L->desc.r;
+  if (M <= 0) return SPA_OK;
+  EpiParams ep = base_epi(L, M, tps, c->N, rows);
   ep.n_out = r;
-  ep.a_hat = L->ws->a_hat;
+  ep.a_hat = a_hat;
   ep.p_cache = c->p_cache;
   ep.score = score;
   ep.proxy_fill = fill;
@@ -639,9 +656,15 @@ static int run_proxy(spa_layer* L, const void* H, const spa_layer_cache* c, floa
   return run_simt(EPI_PROXY, p, M, 1, s, &L->ws->prof, w);
 }
 
+static int run_proxy(spa_layer* L, const void* H, const spa_layer_cache* c, float* score, int fill,
+                     cudaStream_t s) {
+  return run_proxy_rows(L, H, nullptr, c->N, c, fill ? nullptr : L->ws->a_hat, score, fill, s);
+}
+
 // Phases 2 and 3 for M = B * tps tokens; idx == null means every row (rho = 1).
 static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
-                     const spa_layer_cache* c, cudaStream_t s, bool x_ready = false) {
+                     const spa_layer_cache* c, cudaStream_t s, bool x_ready = false,
+                     void* row_copy = nullptr, float* score_zero = nullptr) {
   spa_workspace* ws = L->ws;
   const spa_layer_desc& D = L->desc;
   const int d = D.d, F = D.ffn, M = c->B * tps, N = c->N;
@@ -767,6 +790,8 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
     ep.n_out = d;
     ep.out = c->h_cache;
     ep.resid = ws->H1;
+    ep.row_copy = row_copy;
+    ep.score_zero = score_zero;
     if (bf && M <= 256) {
       TcWsParams p;
       std::memset(&p, 0, sizeof(p));
@@ -829,32 +854,54 @@ extern "C" int spa_partial_block(spa_layer* L, const void* H, const int32_t* idx
   return run_block(L, H, idx, k, c, (cudaStream_t)stream);
 }
 
+// One cached layer step.  Plain: the proxy of every row into the workspace,
+// then the select.  With a_hat / score given (the model's per-layer proxy
+// state, incremental mode): chg == null projects every row into them; else
+// only the chg_tps rows per sequence listed in chg_idx, whose new input rows
+// `chg` holds compact, and the other rows keep their proxy and score (their
+// input is unchanged, and a row selected last step scores 0 because
+// P^c = a_hat there).  The down GEMM then leaves this step's rewritten rows
+// compact in row_copy (the next layer's changed rows) and zeroes their
+// scores (P^c[I] = a_hat[I] now).
+static int layer_step_impl(spa_layer* L, const void* H, const spa_layer_cache* c, int k, int32_t* idx,
+                           cudaStream_t s, float* a_hat, float* score, const void* chg,
+                           const int32_t* chg_idx, int chg_tps, void* row_copy) {
+  const spa_layer_desc& D = L->desc;
+  spa_workspace* ws = L->ws;
+  if (!idx) return fail(SPA_ERR_INVALID, "null idx");
+  if (k < 1 || k > c->N) return fail(SPA_ERR_SHAPE, "k=%d outside [1, N=%d]", k, c->N);
+  const bool state = a_hat != nullptr;
+  if (!state) {
+    a_hat = ws->a_hat;
+    score = ws->score;
+  }
+  if (chg) SPA_TRY(run_proxy_rows(L, chg, chg_idx, chg_tps, c, a_hat, score, 0, s));
+  else SPA_TRY(run_proxy_rows(L, H, nullptr, c->N, c, a_hat, score, 0, s));
+  const double Bn = (double)c->B * c->N, Bk = (double)c->B * k;
+  const double es = D.dtype == SPA_BF16 ? 2.0 : 4.0;
+  cudaError_t e;
+  bool x_ready = false;
+  if (select_norm_supported(D.dtype, c->N, D.d)) {
+    // one launch for the select, the P^c scatter and RMSNorm(H[I])
+    ProfScope ps(&ws->prof, SPA_PROF_TOPK, 4.0 * Bn + 8.0 * Bk * D.r + 4.0 * Bk + 2.0 * Bk * D.d * es, 0.0, s);
+    e = launch_select_norm(D.dtype, score, c->B, c->N, k, idx, a_hat, c->p_cache, D.r, H, L->w.attn_norm,
+                           D.rms_eps, D.d, ws->X, ws->err, s);
+    x_ready = true;
+  } else {
+    ProfScope ps(&ws->prof, SPA_PROF_TOPK, 4.0 * Bn + 8.0 * Bk * D.r + 4.0 * Bk, 0.0, s);
+    e = launch_topk_select(score, c->B, c->N, k, idx, a_hat, c->p_cache, D.r, ws->err, s);
+  }
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "select launch: %s", cudaGetErrorString(e));
+  return run_block(L, H, idx, k, c, s, x_ready, row_copy, state ? score : nullptr);
+}
+
 extern "C" int spa_layer_step(spa_layer* L, const void* H, const spa_layer_cache* c, int k,
                               int32_t* idx, void* stream) {
   if (!L) return fail(SPA_ERR_INVALID, "null layer");
   SPA_TRY(check_H(H));
   SPA_TRY(check_cache(L, c));
-  const spa_layer_desc& D = L->desc;
-  if (!select_norm_supported(D.dtype, c->N, D.d)) {
-    SPA_TRY(spa_proxy_select(L, H, c, k, idx, nullptr, stream));
-    return run_block(L, H, idx, k, c, (cudaStream_t)stream);
-  }
-  // proxy, then one launch for the select, the P^c scatter and RMSNorm(H[I])
-  if (!idx) return fail(SPA_ERR_INVALID, "null idx");
-  if (k < 1 || k > c->N) return fail(SPA_ERR_SHAPE, "k=%d outside [1, N=%d]", k, c->N);
-  cudaStream_t s = (cudaStream_t)stream;
-  spa_workspace* ws = L->ws;
-  SPA_TRY(run_proxy(L, H, c, ws->score, 0, s));
-  cudaError_t e;
-  {
-    const double Bn = (double)c->B * c->N, Bk = (double)c->B * k;
-    const double es = D.dtype == SPA_BF16 ? 2.0 : 4.0;
-    ProfScope ps(&ws->prof, SPA_PROF_TOPK, 4.0 * Bn + 8.0 * Bk * D.r + 4.0 * Bk + 2.0 * Bk * D.d * es, 0.0, s);
-    e = launch_select_norm(D.dtype, ws->score, c->B, c->N, k, idx, ws->a_hat, c->p_cache, D.r, H,
-                           L->w.attn_norm, D.rms_eps, D.d, ws->X, ws->err, s);
-  }
-  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "select + norm launch: %s", cudaGetErrorString(e));
-  return run_block(L, H, idx, k, c, s, true);
+  return layer_step_impl(L, H, c, k, idx, (cudaStream_t)stream, nullptr, nullptr, nullptr, nullptr, 0,
+                         nullptr);
 }
 
 extern "C" int spa_full_block(spa_layer* L, const void* H, const spa_layer_cache* c, int fill_proxy,
@@ -876,6 +923,10 @@ extern "C" void spa_model_free(spa_model* m) {
   if (m->idx_all) cudaFree(m->idx_all);
   if (m->amax_val) cudaFree(m->amax_val);
   if (m->amax_idx) cudaFree(m->amax_idx);
+  if (m->ahat_all) cudaFree(m->ahat_all);
+  if (m->score_all) cudaFree(m->score_all);
+  if (m->chg_rows) cudaFree(m->chg_rows);
+  if (m->chg0_idx) cudaFree(m->chg0_idx);
   delete m;
 }
 
@@ -936,8 +987,32 @@ extern "C" int spa_model_layer_k(const spa_model* m, int layer) {
   return m->k[layer];
 }
 
+extern "C" int spa_model_set_incremental_proxy(spa_model* m, int enable) {
+  if (!m) return fail(SPA_ERR_INVALID, "null model");
+  if (enable && !m->ahat_all) {
+    const spa_layer_desc& D = m->layers[0]->desc;
+    const size_t rows = (size_t)m->desc.B * m->desc.N, L = m->desc.n_layers;
+    const size_t es = D.dtype == SPA_BF16 ? 2 : 4;
+    if (cudaMalloc(&m->ahat_all, L * rows * D.r * 4) != cudaSuccess ||
+        cudaMalloc(&m->score_all, L * rows * 4) != cudaSuccess ||
+        cudaMalloc(&m->chg_rows, rows * D.d * es) != cudaSuccess ||
+        cudaMalloc(&m->chg0_idx, rows * 4) != cudaSuccess) {
+      cudaGetLastError();
+      for (void** q : {(void**)&m->ahat_all, (void**)&m->score_all, &m->chg_rows, (void**)&m->chg0_idx}) {
+        if (*q) cudaFree(*q);
+        *q = nullptr;
+      }
+      return fail(SPA_ERR_NOMEM, "incremental proxy buffers: cudaMalloc failed");
+    }
+  }
+  m->inc = enable != 0;
+  m->inc_valid = false;  // the next step projects every row once
+  return SPA_OK;
+}
+
 extern "C" int spa_model_embed(spa_model* m, const int32_t* tokens, void* stream) {
   if (!m || !tokens) return fail(SPA_ERR_INVALID, "null argument");
+  m->inc_valid = false;  // every row of the layer-0 input may change
   spa_workspace* ws = m->layers[0]->ws;
   ProfScope ps(&ws->prof, SPA_PROF_MISC, 0.0, 0.0, (cudaStream_t)stream);
   cudaError_t e = launch_embed_rows(ws->desc.dtype, m->embed, tokens, nullptr, m->desc.B, m->desc.N,
@@ -957,12 +1032,31 @@ extern "C" int spa_decode_step(spa_model* m, const int32_t* pos, const int32_t* 
   const spa_layer_desc& D = ws->desc;
   const int L = m->desc.n_layers, B = m->desc.B, N = m->desc.N, d = D.d;
   const size_t rows = (size_t)B * N;
+  const bool inc = m->inc;
+  const bool use_chg = inc && m->inc_valid && !full;
+  const int r = D.r;
   for (int l = 0; l < L; ++l) {
     const void* H = (l == 0) ? m->h0 : m->caches[l - 1].h_cache;
-    if (full) {
-      SPA_TRY(spa_full_block(m->layers[l], H, &m->caches[l], full == 1 ? 1 : 0, stream));
+    spa_layer* ly = m->layers[l];
+    const spa_layer_cache* c = &m->caches[l];
+    float* A = inc ? m->ahat_all + (size_t)l * rows * r : nullptr;
+    float* S = inc ? m->score_all + (size_t)l * rows : nullptr;
+    if (full == 1 && inc) {
+      // the rho = 1 fill also sets the proxy state: a_hat = P^c, score 0
+      SPA_TRY(run_proxy_rows(ly, H, nullptr, N, c, A, S, 1, s));
+      SPA_TRY(run_block(ly, H, nullptr, N, c, s));
+    } else if (full) {
+      SPA_TRY(spa_full_block(ly, H, c, full == 1 ? 1 : 0, stream));
+    } else if (inc) {
+      const int32_t* ci = l == 0 ? m->chg0_idx : m->idx_all + (size_t)(l - 1) * rows;
+      const int ctps = l == 0 ? m->chg0_u : m->k[l - 1];
+      SPA_TRY(check_H(H));
+      SPA_TRY(check_cache(ly, c));
+      SPA_TRY(layer_step_impl(ly, H, c, m->k[l], m->idx_all + (size_t)l * rows, s, A, S,
+                              use_chg ? m->chg_rows : nullptr, use_chg ? ci : nullptr, use_chg ? ctps : 0,
+                              m->chg_rows));
     } else {
-      SPA_TRY(spa_layer_step(m->layers[l], H, &m->caches[l], m->k[l], m->idx_all + l * rows, stream));
+      SPA_TRY(spa_layer_step(ly, H, c, m->k[l], m->idx_all + (size_t)l * rows, stream));
     }
   }
   // final RMSNorm at the u positions, LM head, argmax
@@ -1020,9 +1114,13 @@ extern "C" int spa_decode_step(spa_model* m, const int32_t* pos, const int32_t* 
   {
     ProfScope ps(&ws->prof, SPA_PROF_MISC, 2.0 * M * d * es, 0.0, s);
     e = launch_embed_rows(D.dtype, m->embed, tok_in ? tok_in : tok_out, pos, B, u, N, d,
-                          m->desc.vocab, m->h0, ws->err, s);
+                          m->desc.vocab, m->h0, ws->err, s, inc ? m->chg_rows : nullptr,
+                          inc ? m->chg0_idx : nullptr);
   }
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "embed launch: %s", cudaGetErrorString(e));
+  // the proxy state follows the caches after a fill or a cached step in incremental mode
+  m->chg0_u = u;
+  m->inc_valid = inc && full != 2;
   return SPA_OK;
 }
 
@@ -1034,8 +1132,12 @@ extern "C" int spa_decode_graph_capture(spa_model* m, const int32_t* pos, const 
   spa_workspace* ws = m->layers[0]->ws;
   const bool prof_on = ws->prof.on;
   ws->prof.on = false;  // no timing events inside the graph
+  // the launches captured depend on the proxy state; capture runs nothing, so the state is unchanged
+  const bool saved_valid = m->inc_valid;
+  const int variant = !m->inc ? 0 : (m->inc_valid ? 2 : 1);
   SPA_CK(cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal));
   const int st = spa_decode_step(m, pos, tok_in, u, 0, tok_out, stream);
+  m->inc_valid = saved_valid;
   cudaGraph_t g = nullptr;
   const cudaError_t ec = cudaStreamEndCapture(s, &g);
   ws->prof.on = prof_on;
@@ -1051,12 +1153,18 @@ extern "C" int spa_decode_graph_capture(spa_model* m, const int32_t* pos, const 
   if (m->graph) cudaGraphExecDestroy(m->graph);
   m->graph = ex;
   m->graph_u = u;
+  m->graph_inc = variant;
   return SPA_OK;
 }
 
 extern "C" int spa_decode_graph_launch(spa_model* m, void* stream) {
   if (!m) return fail(SPA_ERR_INVALID, "null model");
   if (!m->graph) return fail(SPA_ERR_INVALID, "no decode step has been captured");
+  if (m->graph_inc == 2 && !m->inc_valid)
+    return fail(SPA_ERR_INVALID, "the captured step projects only changed rows, but the proxy state is stale "
+                                 "(a fill, a vanilla step or an embedding came in between): run one step "
+                                 "directly first");
   SPA_CK(cudaGraphLaunch(m->graph, (cudaStream_t)stream));
+  m->inc_valid = m->graph_inc != 0;
   return SPA_OK;
 }

@@ -102,6 +102,8 @@ __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_e
           } else {
             const int2 br = s_rows[row[u]];
             store4(reinterpret_cast<T*>(ep.out) + ((size_t)br.x * ep.N + br.y) * ep.d + gn, r);
+            if (ep.row_copy) store4(reinterpret_cast<T*>(ep.row_copy) + (size_t)t * ep.d + gn, r);
+            if (ep.score_zero && gn == 0) ep.score_zero[(size_t)br.x * ep.N + br.y] = 0.f;
           }
         }
       }
@@ -175,12 +177,15 @@ __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_e
     }
   } else if constexpr (MODE == EPI_PROXY) {
     // One warp per token row: norm, unit proxy, drift score.  r <= 256, so a
-    // lane holds at most 8 columns (c = lane + 32 j).
+    // lane holds at most 8 columns (c = lane + 32 j).  Results go to the
+    // token's cache row (b, s_rows[row].y): the tokens may be every row of
+    // the caches or a compact list of rows.
     const int lane = tid & 31, wid = tid >> 5, nw = nthr >> 5;
     const int r = ep.n_out;
     for (int row = row_begin + wid; row < row_end; row += nw) {
       const int t = gm0 + row;
-      if (t >= ep.M) continue;
+      if (t >= ep.M || s_rows[row].y < 0) continue;
+      const size_t dst = (size_t)s_rows[row].x * ep.N + s_rows[row].y;
       const float* src = tile + row * ld;
       float a[8], pc[8];
       float ss = 0.f;
@@ -188,7 +193,7 @@ __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_e
       for (int j = 0; j < 8; ++j) {
         const int c = lane + 32 * j;
         a[j] = c < r ? src[c] : 0.f;
-        pc[j] = (!ep.proxy_fill && c < r) ? ep.p_cache[(size_t)t * r + c] : 0.f;
+        pc[j] = (!ep.proxy_fill && c < r) ? ep.p_cache[dst * r + c] : 0.f;
         ss += a[j] * a[j];
       }
       ss = warp_sum(ss);
@@ -200,16 +205,19 @@ __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_e
         if (c >= r) continue;
         const float ah = ss > 0.f ? a[j] / nrm : 0.f;
         if (ep.proxy_fill) {
-          ep.p_cache[(size_t)t * r + c] = ah;
+          ep.p_cache[dst * r + c] = ah;
+          if (ep.a_hat) ep.a_hat[dst * r + c] = ah;
         } else {
-          ep.a_hat[(size_t)t * r + c] = ah;
+          ep.a_hat[dst * r + c] = ah;
           const float df = ah - pc[j];
           sd += df * df;
         }
       }
       if (!ep.proxy_fill) {
         sd = warp_sum(sd);
-        if (lane == 0) ep.score[t] = 0.5f * sd;
+        if (lane == 0) ep.score[dst] = 0.5f * sd;
+      } else if (ep.score && lane == 0) {
+        ep.score[dst] = 0.f;  // P^c = a_hat on this row
       }
     }
   } else if constexpr (MODE == EPI_ARGMAX) {

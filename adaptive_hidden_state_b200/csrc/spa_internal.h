@@ -46,10 +46,13 @@ struct EpiParams {
   const void* resid;
   const float* rope_cos;  // [N, head_dim / 2]
   const float* rope_sin;
-  float* a_hat;        // PROXY: [M, r]
-  float* p_cache;      // PROXY: [M, r]
-  float* score;        // PROXY: [M]
-  int proxy_fill;      // PROXY: 1 = write a_hat straight into p_cache
+  float* a_hat;        // PROXY: [B*N, r] (rows addressed through the token's cache row)
+  float* p_cache;      // PROXY: [B*N, r]
+  float* score;        // PROXY: [B*N]
+  int proxy_fill;      // PROXY: 1 = write the unit proxy into p_cache (and into a_hat, score = 0,
+                       // when those are given)
+  void* row_copy;      // RESID_SCATTER: also store the result rows compactly [M, d] (or null)
+  float* score_zero;   // RESID_SCATTER: score_zero[b*N + row] = 0 for the tile's rows (or null)
   float* amax_val;     // ARGMAX: [M, n_tiles]
   int32_t* amax_idx;
   int n_tiles;
@@ -141,7 +144,8 @@ cudaError_t launch_attention(int dtype, const void* Q, const void* Kc, const voi
 // h0[b, pos] <- embed[tok] for the listed (or all) positions.
 cudaError_t launch_embed_rows(int dtype, const void* embed, const int32_t* tokens,
                               const int32_t* pos, int B, int u, int N, int d, int vocab,
-                              void* h0, int* err, cudaStream_t stream);
+                              void* h0, int* err, cudaStream_t stream, void* row_copy = nullptr,
+                              int32_t* pos_copy = nullptr);
 // Gathers final-layer rows at pos and applies the final RMSNorm.
 cudaError_t launch_gather_final(int dtype, const void* hc, const int32_t* pos, int B, int u, int N,
                                 int d, const void* gamma, float eps, void* X, int* err,

@@ -407,7 +407,8 @@ cudaError_t launch_select_norm(int dtype, const float* score, int B, int N, int 
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void embed_rows_kernel(const T* embed, const int32_t* tokens, const int32_t* pos, int u,
-                                  int N, int d, int vocab, T* h0, int* err) {
+                                  int N, int d, int vocab, T* h0, int* err, T* row_copy,
+                                  int32_t* pos_copy) {
   griddep_launch_dependents();
   griddep_wait();
   const int j = blockIdx.x;  // row among B*u (or B*N when pos is null)
@@ -416,23 +417,31 @@ __global__ void embed_rows_kernel(const T* embed, const int32_t* tokens, const i
   const int tok = tokens[j];
   if (p < 0 || p >= N || tok < 0 || tok >= vocab) {
     if (threadIdx.x == 0) report_error(err, DEVERR_INDEX, 501);
+    if (pos_copy && threadIdx.x == 0) pos_copy[j] = -1;
     return;
   }
   const T* src = embed + (size_t)tok * d;
   T* dst = h0 + ((size_t)b * N + p) * d;
-  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) store4(dst + c, load4(src + c));
+  T* cpy = row_copy ? row_copy + (size_t)j * d : nullptr;  // the changed rows, compact
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+    const float4 v = load4(src + c);
+    store4(dst + c, v);
+    if (cpy) store4(cpy + c, v);
+  }
+  if (pos_copy && threadIdx.x == 0) pos_copy[j] = p;
 }
 
 cudaError_t launch_embed_rows(int dtype, const void* embed, const int32_t* tokens,
                               const int32_t* pos, int B, int u, int N, int d, int vocab, void* h0,
-                              int* err, cudaStream_t stream) {
+                              int* err, cudaStream_t stream, void* row_copy, int32_t* pos_copy) {
   const int rows = B * u;
   if (rows <= 0) return cudaSuccess;
   if (dtype == 1)
     return launch_k(embed_rows_kernel<__nv_bfloat16>, dim3(rows), dim3(128), 0, stream,
-                    (const __nv_bfloat16*)embed, tokens, pos, u, N, d, vocab, (__nv_bfloat16*)h0, err);
+                    (const __nv_bfloat16*)embed, tokens, pos, u, N, d, vocab, (__nv_bfloat16*)h0, err,
+                    (__nv_bfloat16*)row_copy, pos_copy);
   return launch_k(embed_rows_kernel<float>, dim3(rows), dim3(128), 0, stream, (const float*)embed,
-                  tokens, pos, u, N, d, vocab, (float*)h0, err);
+                  tokens, pos, u, N, d, vocab, (float*)h0, err, (float*)row_copy, pos_copy);
 }
 
 cudaError_t launch_gather_final(int dtype, const void* hc, const int32_t* pos, int B, int u, int N,

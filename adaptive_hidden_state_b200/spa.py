@@ -35,7 +35,7 @@ EXPORTS = [
     "spa_proxy_select", "spa_partial_block", "spa_layer_step", "spa_full_block",
     "spa_model_create", "spa_model_free", "spa_model_layer_k", "spa_model_embed",
     "spa_decode_step", "spa_decode_graph_capture", "spa_decode_graph_launch",
-    "spa_attention_noalloc",
+    "spa_model_set_incremental_proxy", "spa_attention_noalloc",
 ]
 
 
@@ -113,6 +113,7 @@ _sig("spa_model_create", c_int, POINTER(ModelDesc), POINTER(c_void_p), POINTER(L
      c_void_p, c_void_p, c_void_p, c_void_p, POINTER(c_void_p))
 _sig("spa_model_free", None, c_void_p)
 _sig("spa_model_layer_k", c_int, c_void_p, c_int)
+_sig("spa_model_set_incremental_proxy", c_int, c_void_p, c_int)
 _sig("spa_model_embed", c_int, c_void_p, c_void_p, c_void_p)
 _sig("spa_decode_step", c_int, c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p)
 _sig("spa_decode_graph_capture", c_int, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p)
@@ -318,6 +319,10 @@ class Model:
 
     def embed_tokens(self, tokens, stream=None):
         _check(lib.spa_model_embed(self.handle, _ptr(tokens), _stream(stream)), "spa_model_embed")
+
+    def set_incremental_proxy(self, enable: bool = True):
+        _check(lib.spa_model_set_incremental_proxy(self.handle, 1 if enable else 0),
+               "spa_model_set_incremental_proxy")
 
     def close(self):
         if self.handle:

@@ -54,6 +54,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--workload", choices=["decode", "layer"], default="decode")
+    ap.add_argument("--proxy", choices=["incremental", "plain"], default="incremental",
+                    help="decode: project only rows whose layer input changed (bit-identical), or every row")
     return ap.parse_args()
 
 
@@ -345,6 +347,7 @@ def main():
     total_steps = 1 + args.warmup + args.steps
     assert total_steps <= (N - c["n_prompt"]) // u, "more steps than masked positions"
     model, ws, layers, caches, weights, keep = build_model(spa, torch, args.seed + 1000 * rank)
+    model.set_incremental_proxy(args.proxy == "incremental")
     job = synth.decode_inputs(B=B, N=N, n_prompt=c["n_prompt"], vocab=c["vocab"],
                               steps=total_steps, u=u, seed=args.seed + rank)
     toks = torch.from_numpy(job.tokens.astype(np.int32)).cuda()
@@ -517,6 +520,9 @@ def main():
                            "parallelism": "replicas" if world > 1 else "single",
                            "l2": "inputs larger than L2: 14 GB of layer weights streamed per step",
                            "launch": "one CUDA graph replay per decode step",
+                           "proxy": ("incremental: each layer projects only the rows whose input changed "
+                                     "(bit-identical to projecting every row)" if args.proxy == "incremental"
+                                     else "plain: every row projected at every layer"),
                            "budget_k": model.k},
                 "us_per_layer": us_per_layer,
                 "us_per_layer_kernel_sum": us_per_layer_kernels,

@@ -239,6 +239,27 @@ int spa_decode_graph_capture(spa_model *model, const int32_t *pos, const int32_t
                              int32_t *tok_out, void *stream);
 int spa_decode_graph_launch(spa_model *model, void *stream);
 
+/* Incremental proxy (enable = 1; 0 restores the plain path).  Phase 1 of
+ * Algorithm 1 ([NOTES] 方法详解 > 整体框架; [GIST] Methodology 1) scores every
+ * token with the unit proxy of its current layer input against P^c.  A
+ * token's layer input changes in a decoding step only if the previous layer
+ * rewrote its row (I_{l-1}), or, at layer 0, if it was unmasked at the end of
+ * the last step; the other rows keep their proxy, and their score changes
+ * only where P^c was rewritten, to exactly 0 (P^c = a_hat there).  In this
+ * mode the model keeps, per layer, a_hat [B, N, r] and the score [B, N]
+ * (fp32, library-owned, allocated here: L*B*N*(r + 1)*4 bytes, plus a compact
+ * [B*N, d] buffer of changed rows), and a cached step projects only the
+ * changed rows (B*k_{l-1} per layer, B*u at layer 0) instead of all B*N.
+ * The scores, index sets and outputs are bit-identical to the plain path:
+ * the proxy GEMM reduces each row in a fixed order that does not depend on
+ * the other rows.  The first cached step after enabling, after
+ * spa_model_embed or after a vanilla step (full = 2) projects every row once;
+ * a fill (full = 1) sets the state directly.  A graph captured while the
+ * state is current replays the incremental step and refuses to launch
+ * (SPA_ERR_INVALID) once the state has gone stale.  Errors: SPA_ERR_INVALID
+ * (null model), SPA_ERR_NOMEM. */
+int spa_model_set_incremental_proxy(spa_model *model, int enable);
+
 /* ------------------------------------------------- allocation-free variant --
  * No counterpart on the pages: an engineering addition for callers that may
  * not allocate device memory (custom memory managers and allocator hooks that

@@ -156,3 +156,50 @@ def test_bf16_decode_loop_and_graph_replay():
             assert torch.equal(tout_buf, tok_out[t])
     stream.synchronize()
     lps[0].ws.check()
+
+
+def _state(model, caches, h0, tok):
+    return [tok.clone(), h0.clone()] + [t.clone() for c in caches for t in (c.k, c.v, c.h, c.p)]
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_incremental_proxy_decode_is_bit_identical(bf16):
+    """The incremental proxy (only rows whose layer input changed are
+    projected again) against the plain path, from the same start, over cached
+    steps with the argmax ids fed back (no teacher forcing), a vanilla step in
+    between (the state goes stale and is rebuilt), a re-fill, and graph
+    replays of the incremental step: ids, h0 and every cache bit for bit."""
+    dtype = spa.SPA_BF16 if bf16 else spa.SPA_F32
+    shape = SMALL_BF16 if bf16 else synth.TINY_LAYER
+    B, N, vocab, u, L = 2, 96, 1024, 2, 3
+    model, om, lps, caches, h0, keep = _tiny_model(dtype, shape, L, vocab, B, N, 0.2, seed=90 + bf16,
+                                                   )
+    job = synth.decode_inputs(B=B, N=N, n_prompt=24, vocab=vocab, steps=10, u=u, seed=91)
+    toks = torch.from_numpy(job.tokens.astype(np.int32)).cuda()
+    pos = [torch.from_numpy(p.astype(np.int32)).cuda() for p in job.positions]
+    # step t: 0 fill, 1-3 cached, 4 vanilla, 5-6 cached, 7 fill, 8-9 cached (graph in the second run)
+    full = [1, 0, 0, 0, 2, 0, 0, 1, 0, 0]
+    stream = torch.cuda.Stream()
+    runs = []
+    with torch.cuda.stream(stream):
+        pos_buf = torch.empty((B, u), dtype=torch.int32, device="cuda")
+        tok_buf = torch.empty((B, u), dtype=torch.int32, device="cuda")
+        for inc in (False, True):
+            model.set_incremental_proxy(inc)
+            model.embed_tokens(toks)
+            out = []
+            for t in range(10):
+                if inc and t == 8:
+                    spa.spa_decode_graph_capture(model, pos_buf, None, u, tok_buf)
+                if inc and t >= 8:
+                    pos_buf.copy_(pos[t])
+                    spa.spa_decode_graph_launch(model)
+                else:
+                    spa.spa_decode_step(model, pos[t], None, u, full[t], tok_buf)
+                lps[0].ws.check()
+                out.append(_state(model, caches, h0, tok_buf))
+            runs.append(out)
+    stream.synchronize()
+    for t in range(10):
+        for i, (a, b) in enumerate(zip(runs[0][t], runs[1][t])):
+            assert torch.equal(a, b), f"step {t}: tensor {i} differs between the plain and incremental proxy"

@@ -7,8 +7,9 @@ seeded random weights of that shape (W_v with the i^-0.8 power-law spectrum).
 
 The oracle cannot run whole steps at these sizes, so the checks are sampled
 and by property:
-- one graph-replayed cached step equals the same step launched directly, bit
-  for bit (all 32 layers' caches and the unmasked ids);
+- one graph-replayed cached step with the incremental proxy (only rows whose
+  layer input changed are projected) equals the same step launched directly
+  with the plain proxy, bit for bit (all 32 layers' caches, h0 and the ids);
 - at a few layers of a later step (the first, the widest k = 256 / 512, the
   last) and a few sequences, the layer's input and caches are copied before
   the layer runs, and the oracle's proxy scores, top-k and cached block on
@@ -87,6 +88,8 @@ def _run_on_stream(B, N, n_prompt, u, sample_layers, seqs, check_graph):
     pos = [torch.from_numpy(p.astype(np.int32)).cuda() for p in job.positions]
     tok_out = torch.empty((steps, B, u), dtype=torch.int32, device="cuda")
     model.embed_tokens(toks)
+    if check_graph:
+        model.set_incremental_proxy(True)
     spa.spa_decode_step(model, pos[0], None, u, 1, tok_out[0])
     spa.spa_decode_step(model, pos[1], None, u, 0, tok_out[1])
     ws.check()
@@ -108,6 +111,7 @@ def _run_on_stream(B, N, n_prompt, u, sample_layers, seqs, check_graph):
             for j, t in enumerate((c.k, c.v, c.h, c.p)):
                 t.copy_(state[1 + 4 * i + j])
         del state
+        model.set_incremental_proxy(False)
         spa.spa_decode_step(model, pos[2], None, u, 0, tok_out[2])
         ws.check()
         direct = [tok_out[2], h0] + [t for c in caches for t in (c.k, c.v, c.h, c.p)]
