@@ -178,6 +178,7 @@ struct spa_workspace {
   size_t elem = 4;
   float* a_hat = nullptr;   // [cap, r]
   float* score = nullptr;   // [cap]
+  float* proxy_raw = nullptr;  // [cap, r] raw proxies when r > 256 (bf16)
   int32_t* idx = nullptr;   // [cap]
   void* X = nullptr;        // [cap, d]
   void* Q = nullptr;        // [cap, d]
@@ -250,7 +251,7 @@ static int check_desc(const spa_layer_desc* d) {
   if (d->dtype == SPA_BF16) {
     if (d->d % 256 != 0) return fail(SPA_ERR_UNSUPPORTED, "bf16: d must be a multiple of 256");
     if (d->ffn % 128 != 0) return fail(SPA_ERR_UNSUPPORTED, "bf16: ffn must be a multiple of 128");
-    if (d->r > 256) return fail(SPA_ERR_UNSUPPORTED, "bf16: r must be <= 256");
+    if (d->r > 256 && d->r % 4 != 0) return fail(SPA_ERR_UNSUPPORTED, "bf16: r > 256 must be a multiple of 4");
   } else {
     if (d->d % 4 != 0 || d->ffn % 4 != 0) return fail(SPA_ERR_UNSUPPORTED, "f32: d and ffn must be multiples of 4");
     if (d->r > 128) return fail(SPA_ERR_UNSUPPORTED, "f32: r must be <= 128");
@@ -302,6 +303,7 @@ extern "C" int spa_workspace_create(const spa_layer_desc* desc, int max_B, int m
   if (st == SPA_OK) { st = ws_alloc(ws, &p, (bytes)); if (st == SPA_OK) ws->field = (decltype(ws->field))p; }
   WS_ALLOC(a_hat, cap * r * 4)
   WS_ALLOC(score, cap * 4)
+  if (desc->dtype == SPA_BF16 && r > 256) WS_ALLOC(proxy_raw, cap * r * 4)
   WS_ALLOC(idx, cap * 4)
   WS_ALLOC(X, cap * d * e)
   WS_ALLOC(Q, cap * d * e)
@@ -643,7 +645,15 @@ static int run_proxy_rows(spa_layer* L, const void* H, const int32_t* rows, int 
       const int v = std::atoi(env);
       if (v >= 1 && v <= 16 && (d / 64) / v >= 1) splits = v;
     }
-    return run_tc(EPI_PROXY, r <= 128 ? 128 : 256, p, M, 1, splits, s, &L->ws->prof, w);
+    if (r <= 256) return run_tc(EPI_PROXY, r <= 128 ? 128 : 256, p, M, 1, splits, s, &L->ws->prof, w);
+    // wide r: raw proxies in 256-column tiles, then norms and scores per row
+    p.ep.out = L->ws->proxy_raw;
+    SPA_TRY(run_tc(EPI_PROXY_RAW, 256, p, M, (r + 255) / 256, splits, s, &L->ws->prof, w));
+    ProfScope ps(&L->ws->prof, SPA_PROF_PROXY, (double)M * r * 4 * 3, 0.0, s);
+    const cudaError_t e2 = launch_proxy_finish(L->ws->proxy_raw, M, r, tps, c->N, rows, a_hat, c->p_cache,
+                                               score, fill, L->ws->err, s);
+    if (e2 != cudaSuccess) return fail(SPA_ERR_CUDA, "proxy finish launch: %s", cudaGetErrorString(e2));
+    return SPA_OK;
   }
   SimtGemmParams p;
   std::memset(&p, 0, sizeof(p));

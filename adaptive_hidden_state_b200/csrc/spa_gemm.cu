@@ -220,6 +220,17 @@ __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_e
         ep.score[dst] = 0.f;  // P^c = a_hat on this row
       }
     }
+  } else if constexpr (MODE == EPI_PROXY_RAW) {
+    constexpr int C4 = BN / 4;
+    const int gn0 = n_tile * BN;
+    float* out = reinterpret_cast<float*>(ep.out);
+    for (int it = tid; it < nrows * C4; it += nthr) {
+      const int row = row_begin + it / C4, c = (it % C4) * 4;
+      const int t = gm0 + row, gn = gn0 + c;
+      if (t >= ep.M || gn >= ep.n_out) continue;  // n_out is a multiple of 4
+      *reinterpret_cast<float4*>(out + (size_t)t * ep.n_out + gn) =
+          *reinterpret_cast<const float4*>(tile + row * ld + c);
+    }
   } else if constexpr (MODE == EPI_ARGMAX) {
     const int lane = tid & 31, wid = tid >> 5, nw = nthr >> 5;
     const int gn0 = n_tile * BN;
@@ -499,6 +510,7 @@ cudaError_t launch_tc_gemm(int mode, int BN, const TcGemmParams& p, int m_tiles,
   SPA_TC_CASE(EPI_PROXY, 128)
   SPA_TC_CASE(EPI_PROXY, 256)
   SPA_TC_CASE(EPI_ARGMAX, 256)
+  SPA_TC_CASE(EPI_PROXY_RAW, 256)
 #undef SPA_TC_CASE
   return cudaErrorInvalidValue;
 }

@@ -23,6 +23,7 @@ enum EpiMode : int {
   EPI_RESID_SCATTER = 4,  // H^c[b, I[t]] = acc + H1[t]
   EPI_PROXY = 5,          // a_hat = acc/|acc|; s = 1/2|a_hat - P^c|^2 (or fill P^c)
   EPI_ARGMAX = 6,         // per-tile (max, argmax) of the logits of each row
+  EPI_PROXY_RAW = 7,      // out[t, n] = acc (fp32): the proxy of a wide r, finished per row
 };
 
 // How column tile n maps to rows of the weight sources.
@@ -127,6 +128,13 @@ cudaError_t launch_topk_select(const float* score, int B, int N, int k, int32_t*
 // (X[b*k + j] = RMSNorm(H[b, idx[b, j]]) * gamma), bit-identical to running
 // launch_topk_select then launch_rmsnorm_rows; for N <= 2048 and rows of at
 // most 512 16-byte chunks (select_norm_supported).
+// Rows of raw proxies a [M, r] fp32 (token t: sequence t / tps, cache row
+// idx[t], or t % tps when idx is null) -> unit proxies and drift scores, as
+// the EPI_PROXY epilogue computes them for r <= 256: fill = 1 writes P^c (and
+// a_hat, score = 0 when given), else a_hat and score = 1/2 |a_hat - P^c|^2.
+cudaError_t launch_proxy_finish(const float* raw, int M, int r, int tps, int N, const int32_t* idx,
+                                float* a_hat, float* p_cache, float* score, int fill, int* err,
+                                cudaStream_t stream);
 bool select_norm_supported(int dtype, int N, int d);
 cudaError_t launch_select_norm(int dtype, const float* score, int B, int N, int k, int32_t* idx,
                                const float* a_hat, float* p_cache, int r, const void* H,

@@ -403,6 +403,71 @@ cudaError_t launch_select_norm(int dtype, const float* score, int B, int N, int 
 }
 
 // ---------------------------------------------------------------------------
+// Proxy rows of a wide r (> 256): the GEMM leaves the raw proxies a; one CTA
+// of 256 threads per token row takes the norm, the unit proxy and the drift
+// score (block sums in a fixed order), and writes them at the token's cache
+// row.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) proxy_finish_kernel(const float* raw, int M, int r, int tps, int N,
+                                                           const int32_t* idx, float* a_hat,
+                                                           float* p_cache, float* score, int fill,
+                                                           int* err) {
+  griddep_launch_dependents();
+  griddep_wait();
+  __shared__ float red[8];
+  const int t = blockIdx.x;
+  if (t >= M) return;
+  const int b = t / tps;
+  const int pos = idx ? idx[t] : (t % tps);
+  if (pos < 0 || pos >= N) {
+    if (threadIdx.x == 0) report_error(err, DEVERR_INDEX, 701);
+    return;
+  }
+  const size_t dst = ((size_t)b * N + pos) * r;
+  const float* a = raw + (size_t)t * r;
+  auto block_sum = [&](float v) {
+    v = warp_sum(v);
+    __syncthreads();  // red[] is reused by the next sum
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += red[w];
+    return s;
+  };
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < r; c += 256) ss += a[c] * a[c];
+  ss = block_sum(ss);
+  const float nrm = sqrtf(ss);
+  float sd = 0.f;
+  for (int c = threadIdx.x; c < r; c += 256) {
+    const float ah = ss > 0.f ? a[c] / nrm : 0.f;
+    if (fill) {
+      p_cache[dst + c] = ah;
+      if (a_hat) a_hat[dst + c] = ah;
+    } else {
+      const float df = ah - p_cache[dst + c];
+      a_hat[dst + c] = ah;
+      sd += df * df;
+    }
+  }
+  if (!fill) {
+    sd = block_sum(sd);
+    if (threadIdx.x == 0) score[(size_t)b * N + pos] = 0.5f * sd;
+  } else if (score && threadIdx.x == 0) {
+    score[(size_t)b * N + pos] = 0.f;
+  }
+}
+
+cudaError_t launch_proxy_finish(const float* raw, int M, int r, int tps, int N, const int32_t* idx,
+                                float* a_hat, float* p_cache, float* score, int fill, int* err,
+                                cudaStream_t stream) {
+  if (M <= 0) return cudaSuccess;
+  return launch_k(proxy_finish_kernel, dim3(M), dim3(256), 0, stream, raw, M, r, tps, N, idx, a_hat,
+                  p_cache, score, fill, err);
+}
+
+// ---------------------------------------------------------------------------
 // Embedding rows, final-norm gather, argmax reduction
 // ---------------------------------------------------------------------------
 template <typename T>

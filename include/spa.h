@@ -77,7 +77,8 @@ typedef struct {
   int n_heads;    /* d = n_heads * head_dim */
   int head_dim;   /* even; <= 128 */
   int ffn;        /* SwiGLU hidden width F; multiple of 128 for SPA_BF16 */
-  int r;          /* proxy rank, 1 <= r <= min(d, 256) (SPA_F32: <= 128) */
+  int r;          /* proxy rank, 1 <= r <= d; SPA_BF16: r > 256 (up to r = d, the full-d
+                   * Value identifier) must be a multiple of 4; SPA_F32: r <= 128 */
   int dtype;      /* SPA_F32 or SPA_BF16 */
   float rms_eps;  /* RMSNorm epsilon */
   float rope_theta;

@@ -92,10 +92,13 @@ def test_host_svd_argument_checks():
 
 def test_layer_calls_reject_bad_arguments_before_any_launch():
     # every check below fails before the library touches the device
-    bad = spa.LayerDesc(d=4096, n_heads=32, head_dim=128, ffn=12288, r=300, dtype=spa.SPA_BF16,
+    # a wide bf16 proxy (r > 256) must be a multiple of 4; r > d is a shape error
+    bad = spa.LayerDesc(d=4096, n_heads=32, head_dim=128, ffn=12288, r=302, dtype=spa.SPA_BF16,
                         rms_eps=1e-5, rope_theta=1e4)
     h = ctypes.c_void_p()
     assert spa.lib.spa_workspace_create(ctypes.byref(bad), 1, 512, ctypes.byref(h)) == -5
+    bad.r = 4100
+    assert spa.lib.spa_workspace_create(ctypes.byref(bad), 1, 512, ctypes.byref(h)) == -2
     bad.r, bad.d = 128, 4000
     assert spa.lib.spa_workspace_create(ctypes.byref(bad), 1, 512, ctypes.byref(h)) == -2
     bad.d, bad.dtype = 4096, 7

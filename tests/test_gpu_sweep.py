@@ -1,9 +1,12 @@
 """GPU parity on points of the single-layer sweep at the LLaDA-8B layer shape
 (d=4096, 32x128 heads, F=12288, bf16, batch 1): proxy ranks r in {64, 128,
-256}, cache lengths N in {256, 1024, 4096}, budgets rho in {0.1, 0.16, 0.5,
+256, 512} and r = d = 4096 (the full-d Value identifier: W_r = Lambda V^T at
+full rank scores every token exactly like its value vector W_v h), cache
+lengths N in {256, 512, 1024, 4096}, budgets rho in {0.1, 0.16, 0.25, 0.5,
 1.0}, inputs N(0, 1) with 5% of the rows drifted by N(0, 0.3) after the
 rho = 1 fill.  W_v has the i^-0.8 power-law spectrum and W_r is its exact
-rank-r proxy.
+rank-r proxy.  r > 256 takes the wide-proxy path (raw proxy tiles, then a
+per-row norm and score).
 
 - Each cached point is compared with the oracle on the same inputs and
   caches (index set, Q, O, H1, A, rewritten cache rows; other rows
@@ -12,7 +15,7 @@ rank-r proxy.
 - At rho = 1 the cached step must equal the rho = 1 full recompute: every
   row is selected, and K^c, V^c, H^c come out bit-identical to
   spa_full_block's on the same input.
-r = 512 is outside the bf16 proxy's supported range (r <= 256)."""
+"""
 import numpy as np
 import pytest
 import torch
@@ -59,7 +62,8 @@ def _inputs(N, seed):
     return to(H), to(H2)
 
 
-@pytest.mark.parametrize("r,N,rho", [(64, 256, 0.5), (256, 1024, 0.16), (128, 4096, 0.1)])
+@pytest.mark.parametrize("r,N,rho", [(64, 256, 0.5), (256, 1024, 0.16), (128, 4096, 0.1), (512, 1024, 0.25),
+                                   (4096, 512, 0.25)])
 def test_sweep_point_cached_step(r, N, rho):
     layer, w, ws = _layer(r, N, seed=900 + r + N)
     H, H2 = _inputs(N, seed=N + r)
