@@ -6,7 +6,10 @@ lengths N in {256, 512, 1024, 4096}, budgets rho in {0.1, 0.16, 0.25, 0.5,
 1.0}, inputs N(0, 1) with 5% of the rows drifted by N(0, 0.3) after the
 rho = 1 fill.  W_v has the i^-0.8 power-law spectrum and W_r is its exact
 rank-r proxy.  r > 256 takes the wide-proxy path (raw proxy tiles, then a
-per-row norm and score).
+per-row norm and score).  The Query and Key identifiers of the pages'
+identifier comparison are the same machinery with W_r = W_q or W_k (r = d;
+RoPE rotates a token's query and key by its own position, so their drift
+cosines are the pre-RoPE ones).
 
 - Each cached point is compared with the oracle on the same inputs and
   caches (index set, Q, O, H1, A, rewritten cache rows; other rows
@@ -30,7 +33,7 @@ spa = pytest.importorskip("adaptive_hidden_state_b200.spa")
 D, NH, HD, F = 4096, 32, 128, 12288
 
 
-def _layer(r, N, seed):
+def _layer(r, N, seed, identifier="value"):
     dev = "cuda"
     g = torch.Generator(device=dev).manual_seed(seed)
 
@@ -49,10 +52,15 @@ def _layer(r, N, seed):
     w = {"wq": randn((D, D), .02), "wk": randn((D, D), .02), "wv": wv, "wo": randn((D, D), .02),
          "w_gate": randn((F, D), .02), "w_up": randn((F, D), .02), "w_down": randn((D, F), .02),
          "attn_norm": ones, "ffn_norm": ones}
+    if identifier != "value":  # the Query / Key identifiers: the projection itself as the proxy
+        w_r = w["wq" if identifier == "query" else "wk"].float().cpu()
     desc = spa.LayerDesc(d=D, n_heads=NH, head_dim=HD, ffn=F, r=r, dtype=spa.SPA_BF16, rms_eps=1e-5,
                          rope_theta=1e4)
     ws = spa.Workspace(desc, 1, N)
-    return spa.Layer(desc, w, ws, w_r_host=w_r), w, ws
+    layer = spa.Layer(desc, w, ws, w_r_host=w_r)
+    if identifier != "value":
+        assert torch.equal(layer.proxy_weights(), w_r)  # bf16 values, stored exactly
+    return layer, w, ws
 
 
 def _inputs(N, seed):
@@ -62,10 +70,12 @@ def _inputs(N, seed):
     return to(H), to(H2)
 
 
-@pytest.mark.parametrize("r,N,rho", [(64, 256, 0.5), (256, 1024, 0.16), (128, 4096, 0.1), (512, 1024, 0.25),
-                                   (4096, 512, 0.25)])
-def test_sweep_point_cached_step(r, N, rho):
-    layer, w, ws = _layer(r, N, seed=900 + r + N)
+@pytest.mark.parametrize("r,N,rho,identifier", [(64, 256, 0.5, "value"), (256, 1024, 0.16, "value"),
+                                              (128, 4096, 0.1, "value"), (512, 1024, 0.25, "value"),
+                                              (4096, 512, 0.25, "value"), (4096, 512, 0.25, "key"),
+                                              (4096, 512, 0.25, "query")])
+def test_sweep_point_cached_step(r, N, rho, identifier):
+    layer, w, ws = _layer(r, N, seed=900 + r + N, identifier=identifier)
     H, H2 = _inputs(N, seed=N + r)
     k = spa.spa_budget_k(N, rho)
     cache = spa.Cache(1, N, D, r, spa.SPA_BF16)
@@ -75,7 +85,8 @@ def test_sweep_point_cached_step(r, N, rho):
     idx = torch.empty((1, k), dtype=torch.int32, device="cuda")
     spa.spa_layer_step(layer, H2, cache, k, idx)
     ws.check()
-    check_layer_step(spa, layer, w, H2.clone(), snap, cache, k, idx, ws, (0,), f"r={r} N={N} rho={rho}")
+    check_layer_step(spa, layer, w, H2.clone(), snap, cache, k, idx, ws, (0,),
+                     f"r={r} N={N} rho={rho} {identifier}")
 
 
 def test_sweep_rho1_cached_step_equals_full_recompute():
