@@ -81,8 +81,9 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(const T* Q, const T* Kc,
 //               memory, V as an MN-major operand), so the tensor core works on
 //               the next scores while the softmax warps work on these
 //   warps 4-7   softmax: thread i owns query row i (TMEM lane i).  It reads
-//               its 128 scores, keeps the running max m and sum l in
-//               registers, writes P = 2^(s*log2e/sqrt(d_h) - m) as bf16 into
+//               its 128 scores from TMEM twice, 32 columns at a time (the
+//               row max, then the probabilities), keeps the running max m
+//               and sum l in registers, writes P = 2^(s*log2e/sqrt(d_h) - m) as bf16 into
 //               the 128-byte-swizzled K-major layout the MMA reads, and
 //               rescales O in TMEM only when the max grows by more than 2^8
 //               (the result is exact for any reference max: the final

@@ -32,8 +32,9 @@ namespace spa {
 // ---------------------------------------------------------------------------
 constexpr int kUnroll = 8;
 
-// silu(g) = g / (1 + e^-g) with the fast exponential and reciprocal
-// intrinsics: relative error ~1e-6, far below the bf16 rounding of the result.
+// silu(g) = g / (1 + e^-g) with the fast exponential intrinsic and a
+// correctly rounded reciprocal: relative error ~1e-6, far below the bf16
+// rounding of the result.
 __device__ __forceinline__ float silu(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
 
 // s_rows[row] = (sequence b, cache row) of token t = gm0 + row; (0, -1) when

@@ -1,6 +1,8 @@
-// Memory-bound kernels of the SPA-Cache layer step: gathered RMSNorm, the
-// per-sequence top-k select with the proxy-cache scatter, embedding row
-// updates, the final-norm gather and the LM-head argmax reduction.
+// Memory- and latency-bound kernels of the SPA-Cache layer step: gathered
+// RMSNorm, the per-sequence top-k select with the proxy-cache scatter (alone,
+// or fused with the gather and RMSNorm of the selected rows), the per-row
+// finish of wide proxies, embedding row updates, the final-norm gather and
+// the LM-head argmax reduction.
 #include <cfloat>
 
 #include "spa_device.cuh"
