@@ -422,3 +422,65 @@ def test_decode_layer1_selects_unmasked_rows():
     assert chg <= set(I1)
     assert I1 == sorted(chg | set(sorted(set(range(16)) - chg)[:2]))
     assert np.array_equal(st.tokens[0, job.positions[1][0]], job.forced[1][0])
+
+
+def test_layer_inputs_change_only_at_rewritten_rows_and_scores_carry_over():
+    """The facts the incremental proxy relies on, in the oracle's own decode
+    loop: between two steps, layer l's input changes only at the rows layer
+    l-1 rewrote in the later step (layer 0: the rows unmasked at the end of
+    the earlier step); a row outside those and outside the rows layer l
+    selected in the earlier step keeps its score exactly; a row selected in
+    the earlier step and unchanged since scores exactly 0."""
+    model = _tiny_model(40, L=3)
+    B, N, u, ks = 1, 20, 2, [5, 6, 4]
+    job = synth.decode_inputs(B=B, N=N, n_prompt=6, vocab=40, steps=5, u=u, seed=41)
+    st = O.init_decode_state(model, job.tokens)
+    O.decode_step(model, st, job.positions[0], ks, full=True, forced=job.forced[0])
+    prev_in, prev_s, prev_I = None, None, None
+    for t in range(1, 5):
+        # this step's per-layer inputs, scores and index sets, by the oracle's own layer step
+        inputs, scores, sets = [], [], []
+        H = st.H0[0].copy()
+        for l, layer in enumerate(model.layers):
+            inputs.append(H.copy())
+            cache = st.caches[l][0]
+            _, s = O.proxy_identify(H, layer.W_r, cache.P_c)
+            out = O.layer_step(layer, H, cache, ks[l])
+            assert np.array_equal(out["s"], s)
+            scores.append(s)
+            sets.append(out["I"])
+            H = cache.H_c
+        if prev_in is not None:
+            for l in range(3):
+                chg = np.flatnonzero(np.any(inputs[l] != prev_in[l], axis=1))
+                allowed = set(job.positions[t - 1][0].tolist()) if l == 0 else set(sets[l - 1].tolist())
+                assert set(chg.tolist()) <= allowed, (t, l)
+                for i in range(N):
+                    if i in allowed:
+                        continue
+                    if i in set(prev_I[l].tolist()):
+                        assert scores[l][i] == 0.0, (t, l, i)
+                    else:
+                        assert scores[l][i] == prev_s[l][i], (t, l, i)
+        # finish the step as decode_step does: LM head at this step's positions, write the ids
+        emb = np.asarray(model.embed, dtype=np.float64)
+        st.tokens[0, job.positions[t][0]] = job.forced[t][0]
+        st.H0[0, job.positions[t][0]] = emb[job.forced[t][0]]
+        prev_in, prev_s, prev_I = inputs, scores, sets
+
+
+def test_rope_keeps_the_query_key_drift_cosine():
+    """The Query / Key identifiers score the pre-RoPE projections: RoPE turns
+    every head of a token's query or key by the same angles (its own
+    position), an orthogonal map, so the cosine between a token's old and new
+    vectors is the same before and after it."""
+    rng = np.random.default_rng(50)
+    heads, dh = 4, 16
+    for p in (0, 3, 1023, 4095):
+        a = rng.standard_normal((1, heads, dh))
+        b = a + 0.3 * rng.standard_normal((1, heads, dh))
+        pos = np.array([p])
+        ra, rb = O.rope(a, pos, 1e4).ravel(), O.rope(b, pos, 1e4).ravel()
+        cos_pre = a.ravel() @ b.ravel() / (np.linalg.norm(a) * np.linalg.norm(b))
+        cos_post = ra @ rb / (np.linalg.norm(ra) * np.linalg.norm(rb))
+        assert abs(cos_pre - cos_post) < 1e-12
