@@ -220,6 +220,7 @@ struct spa_model {
   int32_t* idx_all = nullptr;  // [L, B, N] index sets of the last step
   float* amax_val = nullptr;   // [B*N, n_tiles]
   int32_t* amax_idx = nullptr;
+  float* amax_sum = nullptr;   // [B*N, n_tiles] sums of exp for the argmax probability
   int lm_tiles = 0;
   CUtensorMap tm_lm;
   cudaGraphExec_t graph = nullptr;  // a captured cached decode step
@@ -933,6 +934,7 @@ extern "C" void spa_model_free(spa_model* m) {
   if (m->idx_all) cudaFree(m->idx_all);
   if (m->amax_val) cudaFree(m->amax_val);
   if (m->amax_idx) cudaFree(m->amax_idx);
+  if (m->amax_sum) cudaFree(m->amax_sum);
   if (m->ahat_all) cudaFree(m->ahat_all);
   if (m->score_all) cudaFree(m->score_all);
   if (m->chg_rows) cudaFree(m->chg_rows);
@@ -979,7 +981,8 @@ extern "C" int spa_model_create(const spa_model_desc* desc, spa_layer* const* la
   const size_t rows = (size_t)desc->B * desc->N;
   if (cudaMalloc(&m->idx_all, (size_t)desc->n_layers * rows * 4) != cudaSuccess ||
       cudaMalloc(&m->amax_val, rows * m->lm_tiles * 4) != cudaSuccess ||
-      cudaMalloc(&m->amax_idx, rows * m->lm_tiles * 4) != cudaSuccess) {
+      cudaMalloc(&m->amax_idx, rows * m->lm_tiles * 4) != cudaSuccess ||
+      cudaMalloc(&m->amax_sum, rows * m->lm_tiles * 4) != cudaSuccess) {
     cudaGetLastError();
     spa_model_free(m);
     return fail(SPA_ERR_NOMEM, "model buffers: cudaMalloc failed");
@@ -1032,16 +1035,13 @@ extern "C" int spa_model_embed(spa_model* m, const int32_t* tokens, void* stream
   return SPA_OK;
 }
 
-extern "C" int spa_decode_step(spa_model* m, const int32_t* pos, const int32_t* tok_in, int u,
-                               int full, int32_t* tok_out, void* stream) {
-  if (!m || !pos || !tok_out) return fail(SPA_ERR_INVALID, "null argument");
-  if (full < 0 || full > 2) return fail(SPA_ERR_INVALID, "full must be 0, 1 or 2");
-  if (u < 1 || u > m->desc.N) return fail(SPA_ERR_SHAPE, "u=%d outside [1, N]", u);
-  cudaStream_t s = (cudaStream_t)stream;
+// The L layers of one decoding step (full: 0 cached, 1 rho = 1 fill, 2 vanilla).
+static int decode_layers_impl(spa_model* m, int full, cudaStream_t s) {
   spa_workspace* ws = m->layers[0]->ws;
   const spa_layer_desc& D = ws->desc;
-  const int L = m->desc.n_layers, B = m->desc.B, N = m->desc.N, d = D.d;
+  const int L = m->desc.n_layers, B = m->desc.B, N = m->desc.N;
   const size_t rows = (size_t)B * N;
+  void* stream = (void*)s;
   const bool inc = m->inc;
   const bool use_chg = inc && m->inc_valid && !full;
   const int r = D.r;
@@ -1069,6 +1069,21 @@ extern "C" int spa_decode_step(spa_model* m, const int32_t* pos, const int32_t* 
       SPA_TRY(spa_layer_step(ly, H, c, m->k[l], m->idx_all + (size_t)l * rows, stream));
     }
   }
+  // the proxy state follows the caches after a fill or a cached step in
+  // incremental mode; no layer-0 row has changed since (until tokens are written)
+  m->chg0_u = 0;
+  m->inc_valid = inc && full != 2;
+  return SPA_OK;
+}
+
+// Final RMSNorm at the u positions pos ([B, u]) of the last layer's output,
+// LM head, and per row the argmax id (lowest on ties) into tok_out; with
+// conf_out, also that id's softmax probability.
+static int lm_head_impl(spa_model* m, const int32_t* pos, int u, int32_t* tok_out, float* conf_out,
+                        cudaStream_t s) {
+  spa_workspace* ws = m->layers[0]->ws;
+  const spa_layer_desc& D = ws->desc;
+  const int L = m->desc.n_layers, B = m->desc.B, N = m->desc.N, d = D.d;
   // final RMSNorm at the u positions, LM head, argmax
   const double es = D.dtype == SPA_BF16 ? 2.0 : 4.0;
   cudaError_t e;
@@ -1090,6 +1105,7 @@ extern "C" int spa_decode_step(spa_model* m, const int32_t* pos, const int32_t* 
   ep.N = N;
   ep.amax_val = m->amax_val;
   ep.amax_idx = m->amax_idx;
+  ep.amax_sum = conf_out ? m->amax_sum : nullptr;
   ep.err = ws->err;
   int tiles = m->lm_tiles;
   if (D.dtype == SPA_BF16 && M <= 256) {
@@ -1117,21 +1133,61 @@ extern "C" int spa_decode_step(spa_model* m, const int32_t* pos, const int32_t* 
   }
   {
     ProfScope ps(&ws->prof, SPA_PROF_MISC, 8.0 * M * m->lm_tiles, 0.0, s);
-    e = launch_argmax_reduce(m->amax_val, m->amax_idx, M, tiles, tok_out, s);
+    e = conf_out ? launch_confidence_reduce(m->amax_val, m->amax_idx, m->amax_sum, M, tiles, tok_out, conf_out, s)
+                 : launch_argmax_reduce(m->amax_val, m->amax_idx, M, tiles, tok_out, s);
   }
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "argmax launch: %s", cudaGetErrorString(e));
-  // next step's layer-0 input: embeddings of the written ids at pos
+  return SPA_OK;
+}
+
+// h0[b, pos] <- embed[tok] ([B, u]): the next step's layer-0 input.
+static int write_tokens_impl(spa_model* m, const int32_t* pos, const int32_t* tok, int u, cudaStream_t s) {
+  spa_workspace* ws = m->layers[0]->ws;
+  const spa_layer_desc& D = ws->desc;
+  const int B = m->desc.B, N = m->desc.N, d = D.d;
+  const double es = D.dtype == SPA_BF16 ? 2.0 : 4.0;
+  const bool inc = m->inc;
+  const int M = B * u;
+  cudaError_t e;
   {
     ProfScope ps(&ws->prof, SPA_PROF_MISC, 2.0 * M * d * es, 0.0, s);
-    e = launch_embed_rows(D.dtype, m->embed, tok_in ? tok_in : tok_out, pos, B, u, N, d,
-                          m->desc.vocab, m->h0, ws->err, s, inc ? m->chg_rows : nullptr,
-                          inc ? m->chg0_idx : nullptr);
+    e = launch_embed_rows(D.dtype, m->embed, tok, pos, B, u, N, d, m->desc.vocab, m->h0, ws->err, s,
+                          inc ? m->chg_rows : nullptr, inc ? m->chg0_idx : nullptr);
   }
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "embed launch: %s", cudaGetErrorString(e));
-  // the proxy state follows the caches after a fill or a cached step in incremental mode
-  m->chg0_u = u;
-  m->inc_valid = inc && full != 2;
+  m->chg0_u = u;  // these rows of the layer-0 input changed
   return SPA_OK;
+}
+
+extern "C" int spa_decode_step(spa_model* m, const int32_t* pos, const int32_t* tok_in, int u,
+                               int full, int32_t* tok_out, void* stream) {
+  if (!m || !pos || !tok_out) return fail(SPA_ERR_INVALID, "null argument");
+  if (full < 0 || full > 2) return fail(SPA_ERR_INVALID, "full must be 0, 1 or 2");
+  if (u < 1 || u > m->desc.N) return fail(SPA_ERR_SHAPE, "u=%d outside [1, N]", u);
+  cudaStream_t s = (cudaStream_t)stream;
+  SPA_TRY(decode_layers_impl(m, full, s));
+  SPA_TRY(lm_head_impl(m, pos, u, tok_out, nullptr, s));
+  return write_tokens_impl(m, pos, tok_in ? tok_in : tok_out, u, s);
+}
+
+extern "C" int spa_decode_layers(spa_model* m, int full, void* stream) {
+  if (!m) return fail(SPA_ERR_INVALID, "null model");
+  if (full < 0 || full > 2) return fail(SPA_ERR_INVALID, "full must be 0, 1 or 2");
+  return decode_layers_impl(m, full, (cudaStream_t)stream);
+}
+
+extern "C" int spa_decode_confidence(spa_model* m, const int32_t* pos, int u, int32_t* tok_out,
+                                     float* conf_out, void* stream) {
+  if (!m || !pos || !tok_out || !conf_out) return fail(SPA_ERR_INVALID, "null argument");
+  if (u < 1 || u > m->desc.N) return fail(SPA_ERR_SHAPE, "u=%d outside [1, N]", u);
+  return lm_head_impl(m, pos, u, tok_out, conf_out, (cudaStream_t)stream);
+}
+
+extern "C" int spa_model_write_tokens(spa_model* m, const int32_t* pos, const int32_t* tok, int u,
+                                      void* stream) {
+  if (!m || !pos || !tok) return fail(SPA_ERR_INVALID, "null argument");
+  if (u < 1 || u > m->desc.N) return fail(SPA_ERR_SHAPE, "u=%d outside [1, N]", u);
+  return write_tokens_impl(m, pos, tok, u, (cudaStream_t)stream);
 }
 
 extern "C" int spa_decode_graph_capture(spa_model* m, const int32_t* pos, const int32_t* tok_in,

@@ -256,6 +256,15 @@ __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_e
         ep.amax_val[(size_t)t * ep.n_tiles + n_tile] = best;
         ep.amax_idx[(size_t)t * ep.n_tiles + n_tile] = bi;
       }
+      if (ep.amax_sum) {  // for the softmax probability of the argmax
+        float se = 0.f;
+        for (int c = lane; c < BN; c += 32) {
+          if (gn0 + c >= ep.n_out) break;
+          se += expf(tile[row * ld + c] - best);
+        }
+        se = warp_sum(se);
+        if (lane == 0) ep.amax_sum[(size_t)t * ep.n_tiles + n_tile] = se;
+      }
     }
   }
 }

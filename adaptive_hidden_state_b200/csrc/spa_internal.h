@@ -56,6 +56,7 @@ struct EpiParams {
   float* score_zero;   // RESID_SCATTER: score_zero[b*N + row] = 0 for the tile's rows (or null)
   float* amax_val;     // ARGMAX: [M, n_tiles]
   int32_t* amax_idx;
+  float* amax_sum;     // ARGMAX: sum over the tile of exp(logit - tile max) [M, n_tiles], or null
   int n_tiles;
   int* err;            // device error word
 };
@@ -161,6 +162,10 @@ cudaError_t launch_gather_final(int dtype, const void* hc, const int32_t* pos, i
 // Reduces per-tile (max, argmax) partials to one id per row, lowest id on ties.
 cudaError_t launch_argmax_reduce(const float* val, const int32_t* idx, int rows, int n_tiles,
                                  int32_t* out, cudaStream_t stream);
+// Per row: the argmax id (lowest on ties) and its softmax probability
+// 1 / sum_v exp(l_v - max) from per-tile (max, argmax, sum of exp) partials.
+cudaError_t launch_confidence_reduce(const float* val, const int32_t* idx, const float* sum, int rows,
+                                     int n_tiles, int32_t* tok, float* conf, cudaStream_t stream);
 // Copies a [rows] int32 array (device) element-wise.
 cudaError_t launch_copy_i32(const int32_t* src, int32_t* dst, int n, cudaStream_t stream);
 

@@ -545,6 +545,45 @@ cudaError_t launch_argmax_reduce(const float* val, const int32_t* idx, int rows,
   return launch_k(argmax_reduce_kernel, dim3(rows), dim3(32), 0, stream, val, idx, rows, n_tiles, out);
 }
 
+// One warp per row: the row's max over the tiles and its argmax (lowest id on
+// ties, as argmax_reduce_kernel), then total = sum_t sum_t * exp(max_t - max)
+// (lane-strided partial sums, a fixed tree), conf = 1 / total.
+__global__ void confidence_reduce_kernel(const float* val, const int32_t* idx, const float* sum, int rows,
+                                         int n_tiles, int32_t* tok, float* conf) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int row = blockIdx.x;
+  const int lane = threadIdx.x;
+  const float* v = val + (size_t)row * n_tiles;
+  const int32_t* ix = idx + (size_t)row * n_tiles;
+  const float* sm = sum + (size_t)row * n_tiles;
+  float best = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int t = lane; t < n_tiles; t += 32) {
+    if (v[t] > best || (v[t] == best && ix[t] < bi)) { best = v[t]; bi = ix[t]; }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ov > best || (ov == best && oi < bi)) { best = ov; bi = oi; }
+  }
+  float total = 0.f;
+  for (int t = lane; t < n_tiles; t += 32) total += sm[t] * expf(v[t] - best);
+  total = warp_sum(total);
+  if (lane == 0) {
+    tok[row] = bi;
+    conf[row] = total > 0.f ? 1.0f / total : 0.f;
+  }
+}
+
+cudaError_t launch_confidence_reduce(const float* val, const int32_t* idx, const float* sum, int rows,
+                                     int n_tiles, int32_t* tok, float* conf, cudaStream_t stream) {
+  if (rows <= 0) return cudaSuccess;
+  return launch_k(confidence_reduce_kernel, dim3(rows), dim3(32), 0, stream, val, idx, sum, rows, n_tiles,
+                  tok, conf);
+}
+
 __global__ void copy_i32_kernel(const int32_t* src, int32_t* dst, int n) {
   griddep_launch_dependents();
   griddep_wait();

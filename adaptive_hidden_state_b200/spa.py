@@ -34,7 +34,8 @@ EXPORTS = [
     "spa_profile_read", "spa_launch_count", "spa_init_layer", "spa_free_layer", "spa_layer_proxy_weights",
     "spa_proxy_select", "spa_partial_block", "spa_layer_step", "spa_full_block",
     "spa_model_create", "spa_model_free", "spa_model_layer_k", "spa_model_embed",
-    "spa_decode_step", "spa_decode_graph_capture", "spa_decode_graph_launch",
+    "spa_decode_step", "spa_decode_layers", "spa_decode_confidence", "spa_model_write_tokens",
+    "spa_decode_graph_capture", "spa_decode_graph_launch",
     "spa_model_set_incremental_proxy", "spa_attention_noalloc",
 ]
 
@@ -116,6 +117,9 @@ _sig("spa_model_layer_k", c_int, c_void_p, c_int)
 _sig("spa_model_set_incremental_proxy", c_int, c_void_p, c_int)
 _sig("spa_model_embed", c_int, c_void_p, c_void_p, c_void_p)
 _sig("spa_decode_step", c_int, c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p)
+_sig("spa_decode_layers", c_int, c_void_p, c_int, c_void_p)
+_sig("spa_decode_confidence", c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p)
+_sig("spa_model_write_tokens", c_int, c_void_p, c_void_p, c_void_p, c_int, c_void_p)
 _sig("spa_decode_graph_capture", c_int, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p)
 _sig("spa_decode_graph_launch", c_int, c_void_p, c_void_p)
 _sig("spa_attention_noalloc", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
@@ -334,6 +338,20 @@ class Model:
             self.close()
         except Exception:
             pass
+
+
+def spa_decode_layers(model: Model, full: int, stream=None):
+    _check(lib.spa_decode_layers(model.handle, full, _stream(stream)), "spa_decode_layers")
+
+
+def spa_decode_confidence(model: Model, pos, u: int, tok_out, conf_out, stream=None):
+    _check(lib.spa_decode_confidence(model.handle, _ptr(pos), u, _ptr(tok_out), _ptr(conf_out),
+                                     _stream(stream)), "spa_decode_confidence")
+
+
+def spa_model_write_tokens(model: Model, pos, tok, u: int, stream=None):
+    _check(lib.spa_model_write_tokens(model.handle, _ptr(pos), _ptr(tok), u, _stream(stream)),
+           "spa_model_write_tokens")
 
 
 def spa_decode_step(model: Model, pos, tok_in, u: int, full: int, tok_out, stream=None):

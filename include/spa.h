@@ -229,6 +229,25 @@ int spa_model_embed(spa_model *model, const int32_t *tokens, void *stream);
 int spa_decode_step(spa_model *model, const int32_t *pos, const int32_t *tok_in, int u, int full,
                     int32_t *tok_out, void *stream);
 
+/* The same step in three calls, for callers that choose the positions to
+ * unmask from the logits (confidence-based parallel unmasking, [NOTES]
+ * 实验: SPA-Cache combined with parallel decoding; the threshold rule is the
+ * caller's):
+ * - spa_decode_layers runs the L layers of one step (full as above);
+ * - spa_decode_confidence takes the final RMSNorm and the LM head at u
+ *   positions pos ([B, u] int32 device, e.g. every still-masked position) and
+ *   writes per position the argmax id (lowest on ties) into tok_out ([B, u]
+ *   int32) and its softmax probability 1 / sum_v exp(l_v - max_v l) into
+ *   conf_out ([B, u] float);
+ * - spa_model_write_tokens puts embed[tok] ([B, u] int32 device) into h0 at
+ *   pos ([B, u]), the next step's layer-0 input.
+ * spa_decode_step is spa_decode_layers, the argmax at pos, and
+ * spa_model_write_tokens.  u <= N; errors as spa_decode_step. */
+int spa_decode_layers(spa_model *model, int full, void *stream);
+int spa_decode_confidence(spa_model *model, const int32_t *pos, int u, int32_t *tok_out, float *conf_out,
+                          void *stream);
+int spa_model_write_tokens(spa_model *model, const int32_t *pos, const int32_t *tok, int u, void *stream);
+
 /* CUDA-graph form of the cached decode step (full = 0).  Capture records one
  * step with fixed device buffers pos ([B, u]), tok_in ([B, u] or NULL) and
  * tok_out ([B, u]) on `stream` (must not be the legacy default stream; the

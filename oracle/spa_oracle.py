@@ -38,7 +38,7 @@ __all__ = [
     "attention", "swiglu_ffn", "OracleLayer", "LayerCache", "empty_cache",
     "phase2_attention", "phase3_ffn_scatter", "partial_block", "layer_step",
     "full_block", "vanilla_block", "OracleModel", "DecodeState",
-    "init_decode_state", "decode_step", "lm_head_argmax",
+    "init_decode_state", "decode_step", "lm_head_argmax", "confidence", "confident_positions",
 ]
 
 
@@ -372,6 +372,29 @@ def lm_head_argmax(model: OracleModel, h: np.ndarray) -> tuple:
     x = rmsnorm(h, model.final_norm, model.eps)
     logits = x @ np.asarray(model.lm_head, dtype=np.float64).T
     return np.argmax(logits, axis=-1).astype(np.int64), logits
+
+
+def confidence(logits: np.ndarray) -> tuple:
+    """Per row of logits [n, V]: the argmax id (lowest on ties) and its
+    softmax probability 1 / sum_v exp(l_v - max l), the confidence that
+    parallel decoding thresholds [GIST Key Findings, "Integration with
+    Parallel Decoding"; NOTES 实验关键数据, 叠加并行解码 (Table 3); reading A23]."""
+    lg = np.asarray(logits, dtype=np.float64)
+    ids = np.argmax(lg, axis=1)
+    top = lg[np.arange(lg.shape[0]), ids]
+    return ids.astype(np.int64), 1.0 / np.sum(np.exp(lg - top[:, None]), axis=1)
+
+
+def confident_positions(conf: np.ndarray, tau: float) -> np.ndarray:
+    """Reading A23 (the pages name parallel decoding but not its rule): of a
+    sequence's still-masked positions with confidences `conf`, unmask every
+    one whose confidence is >= tau; if none is, the single most confident one
+    (the first on ties).  Returns indices into `conf`, ascending."""
+    conf = np.asarray(conf, dtype=np.float64)
+    chosen = np.flatnonzero(conf >= tau)
+    if chosen.size == 0:
+        chosen = np.array([int(np.argmax(conf))])
+    return chosen.astype(np.int64)
 
 
 def decode_step(model: OracleModel, state: DecodeState, positions: np.ndarray,

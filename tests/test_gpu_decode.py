@@ -203,3 +203,100 @@ def test_incremental_proxy_decode_is_bit_identical(bf16):
     for t in range(10):
         for i, (a, b) in enumerate(zip(runs[0][t], runs[1][t])):
             assert torch.equal(a, b), f"step {t}: tensor {i} differs between the plain and incremental proxy"
+
+
+def test_confidence_parallel_unmasking_tiny_fp32():
+    """Confidence-based parallel unmasking through the split step
+    (spa_decode_layers, spa_decode_confidence at every still-masked
+    position, spa_model_write_tokens of the chosen ones) against the oracle
+    on the tiny fp32 model: argmax ids where the top-2 gap is clear, softmax
+    probabilities, and after four steps h0 and every cache.  Both sides
+    unmask the positions the threshold rule picks from the GPU's
+    confidences, with tau at the 70th percentile of the step's confidences
+    (random weights give tiny probabilities, so a fixed tau would pick one)."""
+    B, N, vocab = 1, 64, 1024
+    model, om, lps, caches, h0, keep = _tiny_model(spa.SPA_F32, synth.TINY_LAYER, 2, vocab, B, N,
+                                                   0.25, seed=70)
+    job = synth.decode_inputs(B=B, N=N, n_prompt=24, vocab=vocab, steps=1, u=2, seed=71)
+    toks = torch.from_numpy(job.tokens.astype(np.int32)).cuda()
+    model.embed_tokens(toks)
+    state = O.init_decode_state(om, job.tokens)
+    emb = np.asarray(om.embed, dtype=np.float64)
+    masked = [i for i in range(N) if job.tokens[0, i] == job.mask_id]
+    for t in range(4):
+        full = t == 0
+        spa.spa_decode_layers(model, 1 if full else 0)
+        H = state.H0[0]
+        for l, layer in enumerate(om.layers):
+            if full:
+                state.caches[l] = [O.full_block(layer, H)[0]]
+            else:
+                O.layer_step(layer, H, state.caches[l][0], model.k[l])
+            H = state.caches[l][0].H_c
+        m = len(masked)
+        pos = torch.tensor([masked], dtype=torch.int32, device="cuda")
+        tok = torch.empty((1, m), dtype=torch.int32, device="cuda")
+        conf = torch.empty((1, m), dtype=torch.float32, device="cuda")
+        spa.spa_decode_confidence(model, pos, m, tok, conf)
+        lps[0].ws.check()
+        logits = O.lm_head_argmax(om, H[masked][None])[1][0]
+        ids_ref, conf_ref = O.confidence(logits)
+        got_ids, got_conf = tok.cpu().numpy()[0], conf.cpu().numpy()[0].astype(np.float64)
+        assert np.max(np.abs(got_conf - conf_ref) / conf_ref) < 1e-3, f"step {t} confidence"
+        for j in range(m):
+            top2 = np.sort(logits[j])[-2:]
+            if top2[1] - top2[0] > 1e-3 * max(1.0, abs(top2[1])):
+                assert got_ids[j] == ids_ref[j], f"step {t} position {masked[j]}"
+        chosen = O.confident_positions(got_conf, float(np.quantile(got_conf, 0.7)))
+        sel_pos = [masked[j] for j in chosen]
+        sel_tok = got_ids[chosen]
+        spa.spa_model_write_tokens(model, torch.tensor(np.array([sel_pos]), dtype=torch.int32, device="cuda"),
+                                   torch.tensor(np.array([sel_tok]), dtype=torch.int32, device="cuda"),
+                                   len(sel_pos))
+        state.tokens[0, sel_pos] = sel_tok
+        state.H0[0, sel_pos] = emb[sel_tok]
+        masked = [p for p in masked if p not in set(sel_pos)]
+    spa.spa_decode_layers(model, 0)
+    H = state.H0[0]
+    for l, layer in enumerate(om.layers):
+        O.layer_step(layer, H, state.caches[l][0], model.k[l])
+        H = state.caches[l][0].H_c
+    torch.cuda.synchronize()
+    assert_close(h0, state.H0, False, "h0")
+    for l in range(2):
+        assert_close(caches[l].h, np.stack([state.caches[l][0].H_c]), False, f"layer {l} H^c")
+        assert_close(caches[l].k, np.stack([state.caches[l][0].K_c]), False, f"layer {l} K^c")
+
+
+@pytest.mark.parametrize("inc", [False, True])
+def test_split_decode_step_equals_decode_step_bf16(inc):
+    """spa_decode_layers + spa_decode_confidence + spa_model_write_tokens at
+    the step's positions reproduce spa_decode_step bit for bit (ids, h0,
+    caches), with the plain and the incremental proxy; the confidence pass's
+    ids are the step's argmax ids."""
+    B, N, vocab, u = 2, 96, 8192, 2
+    model, om, lps, caches, h0, keep = _tiny_model(spa.SPA_BF16, SMALL_BF16, 2, vocab, B, N, 0.3, seed=80)
+    model.set_incremental_proxy(inc)
+    job = synth.decode_inputs(B=B, N=N, n_prompt=32, vocab=vocab, steps=4, u=u, seed=81)
+    toks = torch.from_numpy(job.tokens.astype(np.int32)).cuda()
+    runs = []
+    for split in (False, True):
+        model.embed_tokens(toks)
+        out = []
+        for t in range(4):
+            pos = torch.from_numpy(job.positions[t].astype(np.int32)).cuda()
+            tok = torch.empty((B, u), dtype=torch.int32, device="cuda")
+            if split:
+                conf = torch.empty((B, u), dtype=torch.float32, device="cuda")
+                spa.spa_decode_layers(model, 1 if t == 0 else 0)
+                spa.spa_decode_confidence(model, pos, u, tok, conf)
+                assert torch.all((conf > 0) & (conf <= 1))
+                spa.spa_model_write_tokens(model, pos, tok, u)
+            else:
+                spa.spa_decode_step(model, pos, None, u, 1 if t == 0 else 0, tok)
+            lps[0].ws.check()
+            out.append([tok.clone(), h0.clone()] + [x.clone() for c in caches for x in (c.k, c.v, c.h, c.p)])
+        runs.append(out)
+    for t in range(4):
+        for i, (a, b) in enumerate(zip(runs[0][t], runs[1][t])):
+            assert torch.equal(a, b), f"step {t}: tensor {i} differs"

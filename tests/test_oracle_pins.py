@@ -484,3 +484,30 @@ def test_rope_keeps_the_query_key_drift_cosine():
         cos_pre = a.ravel() @ b.ravel() / (np.linalg.norm(a) * np.linalg.norm(b))
         cos_post = ra @ rb / (np.linalg.norm(ra) * np.linalg.norm(rb))
         assert abs(cos_pre - cos_post) < 1e-12
+
+
+def test_confidence_is_softmax_max_probability():
+    from scipy.special import softmax
+    rng = np.random.default_rng(60)
+    lg = rng.standard_normal((7, 50)) * 3
+    lg[2, 10] = lg[2, 20] = lg[2].max() + 1.0  # a tie: the lower id wins
+    ids, conf = O.confidence(lg)
+    p = softmax(lg, axis=1)
+    assert np.array_equal(ids, np.argmax(p, axis=1))
+    assert ids[2] == 10
+    assert np.max(np.abs(conf - p.max(axis=1))) < 1e-12
+
+
+def test_confident_positions_rule_brute_force():
+    rng = np.random.default_rng(61)
+    for _ in range(200):
+        n = int(rng.integers(1, 8))
+        conf = rng.choice([0.1, 0.3, 0.5, 0.7, 0.9], size=n)
+        tau = float(rng.choice([0.2, 0.5, 0.8, 0.95]))
+        got = O.confident_positions(conf, tau).tolist()
+        above = [i for i in range(n) if conf[i] >= tau]
+        if above:
+            assert got == above
+        else:
+            best = max(conf)
+            assert got == [min(i for i in range(n) if conf[i] == best)]
