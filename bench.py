@@ -224,6 +224,25 @@ def traffic_record(cls: str):
     return None
 
 
+# ------------------------------------------------------------------ ranks (replicas)
+
+def max_over_ranks(dist, world: int, x: float, device) -> float:
+    """The largest of every rank's x (the slowest replica's time); every rank
+    takes part.  NCCL on the GPU in the bench; gloo on the CPU in the tests."""
+    if world == 1:
+        return x
+    import torch
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, B: int, u: int, steps: int, t_ms: float) -> float:
+    """Whole-job throughput: every replica unmasks B*u tokens per step, and the
+    job takes as long as its slowest replica (t_ms for `steps` steps)."""
+    return world * B * u * steps / (t_ms / 1e3)
+
+
 # ------------------------------------------------------------------ reference arm
 
 def run_reference(args, rank: int):
@@ -363,13 +382,6 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     def rewind():
         """Back to the state after step 0 and the warm-up steps."""
         model.embed_tokens(toks)
@@ -408,10 +420,9 @@ def main():
     barrier()
     clk = clocks.stop()
     ws.check()
-    t_ms = max_over_ranks(ev0.elapsed_time(ev1))
+    t_ms = max_over_ranks(dist, world, ev0.elapsed_time(ev1), "cuda")
     K = args.steps
-    tokens = world * B * u * K
-    value = tokens / (t_ms / 1e3)
+    value = job_tokens_per_s(world, B, u, K, t_ms)
     ms_step = t_ms / K
 
     # ---- profiled region: the same K steps launched directly, CUDA events per kernel
@@ -475,8 +486,8 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e = {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+    e2e_ms = max_over_ranks(dist, world, e0.elapsed_time(e1), "cuda")
+    e2e = {"value": job_tokens_per_s(world, B, u, K, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": B * u * 4, "d2h_bytes_per_step": B * u * 4}
 
     # ---- rho = 1 vanilla decoding (full recompute, no proxy) on the same GPU
@@ -492,7 +503,7 @@ def main():
     v1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    v_ms = max_over_ranks(v0.elapsed_time(v1)) / vk
+    v_ms = max_over_ranks(dist, world, v0.elapsed_time(v1), "cuda") / vk
     ws.check()
 
     # ---- CPU oracle on a bounded sample (rank 0, one GPU only)
