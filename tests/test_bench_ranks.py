@@ -37,7 +37,7 @@ def _worker(rank, world, port, times, out):
 def test_max_over_ranks_gloo_world2():
     world, port = 2, _free_port()
     times = [12.5, 17.25]
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_worker, args=(world, port, times, out), nprocs=world, join=True)
     assert dict(out) == {0: 17.25, 1: 17.25}
 
