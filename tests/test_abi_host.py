@@ -113,4 +113,11 @@ def test_layer_calls_reject_bad_arguments_before_any_launch():
     assert spa.lib.spa_full_block(None, None, ctypes.byref(cache), 1, None) == -1
     assert spa.lib.spa_decode_step(None, None, None, 1, 0, None, None) == -1
     assert spa.lib.spa_model_layer_k(None, 0) == -1
+    assert spa.lib.spa_layer_step(None, None, ctypes.byref(cache), 1, None, None) == -1
+    assert spa.lib.spa_decode_layers(None, 0, None) == -1
+    assert spa.lib.spa_decode_confidence(None, None, 1, None, None, None) == -1
+    assert spa.lib.spa_model_write_tokens(None, None, None, 1, None) == -1
+    assert spa.lib.spa_model_set_incremental_proxy(None, 1) == -1
+    assert spa.lib.spa_model_embed(None, None, None) == -1
+    assert spa.lib.spa_decode_graph_launch(None, None) == -1
     assert "null" in spa.lib.spa_last_error().decode()
