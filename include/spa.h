@@ -230,9 +230,9 @@ int spa_decode_step(spa_model *model, const int32_t *pos, const int32_t *tok_in,
                     int32_t *tok_out, void *stream);
 
 /* The same step in three calls, for callers that choose the positions to
- * unmask from the logits (confidence-based parallel unmasking, [NOTES]
- * 实验: SPA-Cache combined with parallel decoding; the threshold rule is the
- * caller's):
+ * unmask from the logits (confidence-based parallel unmasking: [NOTES]
+ * 实验关键数据 > 叠加并行解码 (Table 3); [GIST] Key Findings, "Integration
+ * with Parallel Decoding"; the threshold rule is the caller's):
  * - spa_decode_layers runs the L layers of one step (full as above);
  * - spa_decode_confidence takes the final RMSNorm and the LM head at u
  *   positions pos ([B, u] int32 device, e.g. every still-masked position) and
@@ -240,7 +240,8 @@ int spa_decode_step(spa_model *model, const int32_t *pos, const int32_t *tok_in,
  *   int32) and its softmax probability 1 / sum_v exp(l_v - max_v l) into
  *   conf_out ([B, u] float);
  * - spa_model_write_tokens puts embed[tok] ([B, u] int32 device) into h0 at
- *   pos ([B, u]), the next step's layer-0 input.
+ *   pos ([B, u]), the next step's layer-0 input (with the incremental proxy,
+ *   these are the rows the next step's layer 0 projects again).
  * spa_decode_step is spa_decode_layers, the argmax at pos, and
  * spa_model_write_tokens.  u <= N; errors as spa_decode_step. */
 int spa_decode_layers(spa_model *model, int full, void *stream);
