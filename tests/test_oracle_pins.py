@@ -511,3 +511,17 @@ def test_confident_positions_rule_brute_force():
         else:
             best = max(conf)
             assert got == [min(i for i in range(n) if conf[i] == best)]
+
+
+def test_lm_head_argmax_matches_torch():
+    rng = np.random.default_rng(62)
+    d, V = 32, 50
+    model = O.OracleModel(layers=[], embed=rng.standard_normal((V, d)),
+                          final_norm=rng.uniform(0.5, 1.5, d), lm_head=rng.standard_normal((V, d)))
+    h = rng.standard_normal((2, 3, d))
+    ids, logits = O.lm_head_argmax(model, h)
+    ht = torch.from_numpy(h)
+    x = ht * torch.rsqrt(ht.pow(2).mean(-1, keepdim=True) + model.eps) * torch.from_numpy(model.final_norm)
+    ref = x @ torch.from_numpy(model.lm_head).T
+    assert np.max(np.abs(logits - ref.numpy())) < 1e-10
+    assert np.array_equal(ids, ref.argmax(-1).numpy())
