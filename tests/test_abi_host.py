@@ -121,3 +121,17 @@ def test_layer_calls_reject_bad_arguments_before_any_launch():
     assert spa.lib.spa_model_embed(None, None, None) == -1
     assert spa.lib.spa_decode_graph_launch(None, None) == -1
     assert "null" in spa.lib.spa_last_error().decode()
+
+
+def test_host_svd_full_rank_gives_the_value_cosine():
+    # r = d (the full-d Value identifier): the host proxy scores every pair of
+    # inputs exactly like the value projection itself
+    rng = np.random.default_rng(70)
+    d = 64
+    W, *_ = synth.power_law_wv(d, rng)
+    W = W.astype(np.float32)
+    Wr = spa.spa_singular_proxy_host(torch.from_numpy(W), d).numpy().astype(np.float64)
+    h, h2 = rng.standard_normal((2, 10, d))
+    cos = lambda A, x, y: np.sum((x @ A.T) * (y @ A.T), 1) / (
+        np.linalg.norm(x @ A.T, axis=1) * np.linalg.norm(y @ A.T, axis=1))
+    assert np.max(np.abs(cos(Wr, h, h2) - cos(W.astype(np.float64), h, h2))) < 1e-5
