@@ -1,5 +1,6 @@
 // Host side of libspa: argument checks, workspace and handle management,
 // tensor-map encoding and the launch sequence of each C-ABI call.
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -261,9 +262,33 @@ static int check_desc(const spa_layer_desc* d) {
   return SPA_OK;
 }
 
+// Failure injection for tests of the error paths: after this many more
+// successful device allocations, the next one fails once (negative: never).
+static std::atomic<long long> g_fail_alloc_after{-1};
+
+// Every device allocation of the library goes through here.
+static cudaError_t dev_alloc(void** p, size_t bytes) {
+  long long n = g_fail_alloc_after.load();
+  while (n >= 0) {
+    if (g_fail_alloc_after.compare_exchange_weak(n, n - 1)) {
+      if (n == 0) {
+        *p = nullptr;
+        return cudaErrorMemoryAllocation;
+      }
+      break;
+    }
+  }
+  return cudaMalloc(p, bytes);
+}
+
+extern "C" int spa_debug_fail_alloc_after(long long n) {
+  g_fail_alloc_after.store(n < 0 ? -1 : n);
+  return SPA_OK;
+}
+
 static int ws_alloc(spa_workspace* ws, void** p, size_t bytes) {
   if (bytes == 0) bytes = 16;
-  cudaError_t e = cudaMalloc(p, bytes);
+  cudaError_t e = dev_alloc(p, bytes);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return fail(SPA_ERR_NOMEM, "cudaMalloc(%zu) failed: %s", bytes, cudaGetErrorString(e));
@@ -363,6 +388,17 @@ extern "C" int spa_workspace_status(spa_workspace* ws, void* stream) {
   return fail(SPA_ERR_DEVICE, "device check failed: bits 0x%x site %d", h[0], h[1]);
 }
 
+extern "C" int spa_debug_bounded_wait(spa_workspace* ws, const int* flag, int expect, double limit_us,
+                                      void* stream) {
+  if (!ws) return fail(SPA_ERR_INVALID, "null workspace");
+  if (!(limit_us >= 0.0) || limit_us > 1e6) return fail(SPA_ERR_INVALID, "limit_us must be in [0, 1e6]");
+  const cudaError_t e = launch_wait_probe(flag, expect, (unsigned long long)(limit_us * 1e3), ws->err,
+                                          (cudaStream_t)stream);
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "wait probe launch: %s", cudaGetErrorString(e));
+  ++g_launches;
+  return SPA_OK;
+}
+
 extern "C" int spa_workspace_intermediates(const spa_workspace* ws, spa_intermediates* out) {
   if (!ws || !out) return fail(SPA_ERR_INVALID, "null argument");
   out->x = ws->X;
@@ -451,7 +487,7 @@ extern "C" int spa_init_layer(const spa_layer_desc* desc, const spa_layer_weight
   L->w = *w;
   L->ws = ws;
   const size_t e = desc->dtype == SPA_BF16 ? 2 : 4;
-  if (cudaMalloc(&L->w_r, (size_t)r * d * e) != cudaSuccess) {
+  if (dev_alloc(&L->w_r, (size_t)r * d * e) != cudaSuccess) {
     cudaGetLastError();
     delete L;
     return fail(SPA_ERR_NOMEM, "cudaMalloc of the proxy weights failed");
@@ -979,10 +1015,10 @@ extern "C" int spa_model_create(const spa_model_desc* desc, spa_layer* const* la
   const spa_layer_desc& D = ws->desc;
   m->lm_tiles = (desc->vocab + 127) / 128;  // the widest split: 128-column tiles
   const size_t rows = (size_t)desc->B * desc->N;
-  if (cudaMalloc(&m->idx_all, (size_t)desc->n_layers * rows * 4) != cudaSuccess ||
-      cudaMalloc(&m->amax_val, rows * m->lm_tiles * 4) != cudaSuccess ||
-      cudaMalloc(&m->amax_idx, rows * m->lm_tiles * 4) != cudaSuccess ||
-      cudaMalloc(&m->amax_sum, rows * m->lm_tiles * 4) != cudaSuccess) {
+  if (dev_alloc((void**)&m->idx_all, (size_t)desc->n_layers * rows * 4) != cudaSuccess ||
+      dev_alloc((void**)&m->amax_val, rows * m->lm_tiles * 4) != cudaSuccess ||
+      dev_alloc((void**)&m->amax_idx, rows * m->lm_tiles * 4) != cudaSuccess ||
+      dev_alloc((void**)&m->amax_sum, rows * m->lm_tiles * 4) != cudaSuccess) {
     cudaGetLastError();
     spa_model_free(m);
     return fail(SPA_ERR_NOMEM, "model buffers: cudaMalloc failed");
@@ -1000,16 +1036,25 @@ extern "C" int spa_model_layer_k(const spa_model* m, int layer) {
   return m->k[layer];
 }
 
+extern "C" int spa_model_index_set(const spa_model* m, int layer, int32_t* idx_out, void* stream) {
+  if (!m || !idx_out) return fail(SPA_ERR_INVALID, "null argument");
+  if (layer < 0 || layer >= (int)m->k.size()) return fail(SPA_ERR_SHAPE, "layer %d outside [0, %d)", layer, (int)m->k.size());
+  const size_t rows = (size_t)m->desc.B * m->desc.N;
+  SPA_CK(cudaMemcpyAsync(idx_out, m->idx_all + (size_t)layer * rows, (size_t)m->desc.B * m->k[layer] * sizeof(int32_t),
+                         cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+  return SPA_OK;
+}
+
 extern "C" int spa_model_set_incremental_proxy(spa_model* m, int enable) {
   if (!m) return fail(SPA_ERR_INVALID, "null model");
   if (enable && !m->ahat_all) {
     const spa_layer_desc& D = m->layers[0]->desc;
     const size_t rows = (size_t)m->desc.B * m->desc.N, L = m->desc.n_layers;
     const size_t es = D.dtype == SPA_BF16 ? 2 : 4;
-    if (cudaMalloc(&m->ahat_all, L * rows * D.r * 4) != cudaSuccess ||
-        cudaMalloc(&m->score_all, L * rows * 4) != cudaSuccess ||
-        cudaMalloc(&m->chg_rows, rows * D.d * es) != cudaSuccess ||
-        cudaMalloc(&m->chg0_idx, rows * 4) != cudaSuccess) {
+    if (dev_alloc((void**)&m->ahat_all, L * rows * D.r * 4) != cudaSuccess ||
+        dev_alloc((void**)&m->score_all, L * rows * 4) != cudaSuccess ||
+        dev_alloc(&m->chg_rows, rows * D.d * es) != cudaSuccess ||
+        dev_alloc((void**)&m->chg0_idx, rows * 4) != cudaSuccess) {
       cudaGetLastError();
       for (void** q : {(void**)&m->ahat_all, (void**)&m->score_all, &m->chg_rows, (void**)&m->chg0_idx}) {
         if (*q) cudaFree(*q);

@@ -572,9 +572,16 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_tc_kernel(const __grid_cons
 
 // How many clusters of `splits` attention CTAs the GPU holds at once (0: none).
 static int attn_max_clusters(int splits) {
-  static int cache[9] = {0};
+  static int cache_all[kMaxDevices][9] = {{0}};  // per device, filled once (benign race: same value)
   if (splits < 2 || splits > 8) return 0;
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 0;
+  int* cache = cache_all[dev];
   if (cache[splits] == 0) {
+    if (configure_kernel((const void*)attn_tc_kernel, kASmem, false) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(splits, 1, 1);
     cfg.blockDim = dim3(kAThreads, 1, 1);
@@ -608,12 +615,8 @@ cudaError_t launch_attention(int dtype, const void* Q, const void* Kc, const voi
     const long long groups = (long long)B * n_heads * q_tiles;
     // capacity of the scratch in (128-row, one-head) partial slots
     const long long slots = (long long)max_rows * n_heads / kAT;
-    static bool configured = false;
-    if (!configured) {
-      cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kASmem);
-      if (e != cudaSuccess) return e;
-      configured = true;
-    }
+    const cudaError_t ec = configure_kernel((const void*)attn_tc_kernel, kASmem, false);
+    if (ec != cudaSuccess) return ec;
     int splits = 1;
     if (allow_cluster) {
       // split the keys while every cluster of the grid is resident at once and

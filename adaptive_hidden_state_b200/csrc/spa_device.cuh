@@ -8,6 +8,8 @@
 #pragma once
 #include <cstdint>
 #include <cstdlib>
+#include <mutex>
+#include <set>
 #include <utility>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -100,10 +102,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Gives up when
-// *abort is set by another thread or after kWaitLimitNs; on its own time-out
-// it sets *abort and records the error.  Returns true when the phase completed.
+// *abort is set by another thread or after limit_ns; on its own time-out it
+// sets *abort and records the error.  Returns true when the phase completed.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int* err, int site) {
+                                          int* err, int site,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer();
@@ -112,8 +115,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(a, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort = 1;
+      report_error(err, DEVERR_TIMEOUT, site);
+      return false;
+    }
+  }
+}
+
+// Wait until the global int *flag equals `expect` (acquire: what the writer
+// stored before releasing the flag is visible afterwards).  Gives up after
+// limit_ns and records the error.  Returns true when the flag was seen.
+__device__ __forceinline__ bool flag_wait(const int* flag, int expect, int* err, int site,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
+  auto load = [flag] {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    return v;
+  };
+  if (load() == expect) return true;
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i)
+      if (load() == expect) return true;
+    if (globaltimer() - t0 > limit_ns) {
       report_error(err, DEVERR_TIMEOUT, site);
       return false;
     }
@@ -275,6 +301,36 @@ inline bool pdl_enabled() {
   }();
   return on;
 }
+
+// Host: sets a kernel's dynamic shared-memory limit (and, when asked, the
+// permission for clusters beyond the portable size) once per (kernel,
+// device), under a lock, with that device current.  Function attributes are
+// per device, so a process that launches on several devices configures each.
+inline cudaError_t configure_kernel(const void* func, int smem, bool nonportable_cluster) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  if (done.count({func, dev})) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess && nonportable_cluster)
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess) done.insert({func, dev});
+  return e;
+}
+
+// Host: the current device's ordinal (0 when the query fails).
+inline int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return dev;
+}
+constexpr int kMaxDevices = 64;  // per-device host caches (occupancy tables)
 
 // Host: launches `kern` on `stream` with the programmatic-serialization attribute.
 template <typename... KArgs, typename... Args>

@@ -482,14 +482,8 @@ static cudaError_t launch_tc_typed(const TcGemmParams& p, int m_tiles, int n_til
                                    cudaStream_t stream) {
   auto kern = tc_gemm_kernel<MODE, BN>;
   const int smem = tc_smem_bytes(BN);
-  static bool configured = false;  // per instantiation
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  cudaError_t ec = configure_kernel((const void*)kern, smem, true);
+  if (ec != cudaSuccess) return ec;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(splits, n_tiles, m_tiles);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -781,12 +775,8 @@ template <int MODE, int NACC>
 static cudaError_t launch_ws_typed(const TcWsParams& p, int n_tiles, int splits,
                                    cudaStream_t stream) {
   auto kern = tc_ws_kernel<MODE, NACC>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kWsSmem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  cudaError_t ec = configure_kernel((const void*)kern, kWsSmem, false);
+  if (ec != cudaSuccess) return ec;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(splits, n_tiles, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -806,11 +796,14 @@ static cudaError_t launch_ws_typed(const TcWsParams& p, int n_tiles, int splits,
 
 template <int MODE, int NACC>
 static int ws_max_clusters(int splits) {
-  static int cache[9] = {0};
+  static int cache_all[kMaxDevices][9] = {{0}};  // per device, filled once (benign race: same value)
   if (splits < 1 || splits > 8) return 0;
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 0;
+  int* cache = cache_all[dev];
   if (cache[splits] == 0) {
     auto kern = tc_ws_kernel<MODE, NACC>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kWsSmem) != cudaSuccess) {
+    if (configure_kernel((const void*)kern, kWsSmem, false) != cudaSuccess) {
       cudaGetLastError();
       return 0;
     }

@@ -166,6 +166,10 @@ cudaError_t launch_argmax_reduce(const float* val, const int32_t* idx, int rows,
 // 1 / sum_v exp(l_v - max) from per-tile (max, argmax, sum of exp) partials.
 cudaError_t launch_confidence_reduce(const float* val, const int32_t* idx, const float* sum, int rows,
                                      int n_tiles, int32_t* tok, float* conf, cudaStream_t stream);
+// A bounded wait that nothing completes (flag == null: an mbarrier no thread
+// arrives on; else until *flag == expect), for tests of the time-out path.
+cudaError_t launch_wait_probe(const int* flag, int expect, unsigned long long limit_ns, int* err,
+                              cudaStream_t stream);
 // Copies a [rows] int32 array (device) element-wise.
 cudaError_t launch_copy_i32(const int32_t* src, int32_t* dst, int n, cudaStream_t stream);
 

@@ -596,4 +596,31 @@ cudaError_t launch_copy_i32(const int32_t* src, int32_t* dst, int n, cudaStream_
   return launch_k(copy_i32_kernel, dim3((n + 255) / 256), dim3(256), 0, stream, src, dst, n);
 }
 
+// ---------------------------------------------------------------------------
+// Bounded waits that nothing completes, for tests of the time-out path: with
+// flag == null an mbarrier of count 1 that no thread arrives on, otherwise
+// the global flag compared with `expect`.  Either way the wait gives up
+// after limit_ns and records DEVERR_TIMEOUT in the error word; no copy or
+// tensor-core operation is in flight, so the kernel then simply returns.
+// ---------------------------------------------------------------------------
+__global__ void wait_probe_kernel(const int* flag, int expect, unsigned long long limit_ns, int* err) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  if (flag == nullptr) mbar_wait(&bar, 0, &abort_flag, err, 901, limit_ns);
+  else flag_wait(flag, expect, err, 902, limit_ns);
+}
+
+cudaError_t launch_wait_probe(const int* flag, int expect, unsigned long long limit_ns, int* err,
+                              cudaStream_t stream) {
+  wait_probe_kernel<<<1, 32, 0, stream>>>(flag, expect, limit_ns, err);
+  return cudaPeekAtLastError();
+}
+
 }  // namespace spa

@@ -33,10 +33,11 @@ EXPORTS = [
     "spa_workspace_status", "spa_workspace_intermediates", "spa_profile_enable",
     "spa_profile_read", "spa_launch_count", "spa_init_layer", "spa_free_layer", "spa_layer_proxy_weights",
     "spa_proxy_select", "spa_partial_block", "spa_layer_step", "spa_full_block",
-    "spa_model_create", "spa_model_free", "spa_model_layer_k", "spa_model_embed",
+    "spa_model_create", "spa_model_free", "spa_model_layer_k", "spa_model_index_set", "spa_model_embed",
     "spa_decode_step", "spa_decode_layers", "spa_decode_confidence", "spa_model_write_tokens",
     "spa_decode_graph_capture", "spa_decode_graph_launch",
-    "spa_model_set_incremental_proxy", "spa_attention_noalloc",
+    "spa_model_set_incremental_proxy", "spa_debug_fail_alloc_after", "spa_debug_bounded_wait",
+    "spa_attention_noalloc", "spa_attention_noalloc_status",
 ]
 
 
@@ -114,6 +115,7 @@ _sig("spa_model_create", c_int, POINTER(ModelDesc), POINTER(c_void_p), POINTER(L
      c_void_p, c_void_p, c_void_p, c_void_p, POINTER(c_void_p))
 _sig("spa_model_free", None, c_void_p)
 _sig("spa_model_layer_k", c_int, c_void_p, c_int)
+_sig("spa_model_index_set", c_int, c_void_p, c_int, c_void_p, c_void_p)
 _sig("spa_model_set_incremental_proxy", c_int, c_void_p, c_int)
 _sig("spa_model_embed", c_int, c_void_p, c_void_p, c_void_p)
 _sig("spa_decode_step", c_int, c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p)
@@ -124,6 +126,9 @@ _sig("spa_decode_graph_capture", c_int, c_void_p, c_void_p, c_void_p, c_int, c_v
 _sig("spa_decode_graph_launch", c_int, c_void_p, c_void_p)
 _sig("spa_attention_noalloc", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
      c_int, c_int, c_void_p)
+_sig("spa_attention_noalloc_status", c_int, c_void_p)
+_sig("spa_debug_fail_alloc_after", c_int, ctypes.c_longlong)
+_sig("spa_debug_bounded_wait", c_int, c_void_p, c_void_p, c_int, c_double, c_void_p)
 
 
 def _check(status: int, where: str):
@@ -310,6 +315,7 @@ class Model:
                  B: int, N: int, rho_p: float, l_p: int, rho_1: float, rho_L: float):
         self.layers, self.caches = layers, caches
         self.h0, self.embed, self.final_norm, self.lm_head = h0, embed, final_norm, lm_head
+        self.B, self.N = B, N
         L = len(layers)
         desc = ModelDesc(L, vocab, B, N, rho_p, rho_1, rho_L, l_p)
         handles = (c_void_p * L)(*[ly.handle.value for ly in layers])
@@ -323,6 +329,13 @@ class Model:
 
     def embed_tokens(self, tokens, stream=None):
         _check(lib.spa_model_embed(self.handle, _ptr(tokens), _stream(stream)), "spa_model_embed")
+
+    def index_set(self, layer: int, stream=None) -> torch.Tensor:
+        """[B, k_l] int32 device copy of layer `layer`'s index set from the last cached step."""
+        out = torch.empty((self.B, self.k[layer]), dtype=torch.int32, device="cuda")
+        _check(lib.spa_model_index_set(self.handle, layer, _ptr(out), _stream(stream)),
+               "spa_model_index_set")
+        return out
 
     def set_incremental_proxy(self, enable: bool = True):
         _check(lib.spa_model_set_incremental_proxy(self.handle, 1 if enable else 0),
@@ -374,3 +387,9 @@ def spa_attention_noalloc(Q, k_cache, v_cache, O, B: int, k: int, N: int, n_head
     library's fixed scratch instead of allocated memory (see include/spa.h)."""
     _check(lib.spa_attention_noalloc(_ptr(Q), _ptr(k_cache), _ptr(v_cache), _ptr(O), B, k, N,
                                      n_heads, head_dim, _stream(stream)), "spa_attention_noalloc")
+
+
+def spa_attention_noalloc_status(stream=None) -> int:
+    """Reads and clears the allocation-free attention's device error word
+    (synchronises the stream): 0, or the negative status of what failed."""
+    return lib.spa_attention_noalloc_status(_stream(stream))

@@ -215,6 +215,12 @@ int spa_model_create(const spa_model_desc *desc, spa_layer *const *layers,
 void spa_model_free(spa_model *model);
 /* k_l of layer l (0-based), or -1. */
 int spa_model_layer_k(const spa_model *model, int layer);
+/* The index set I of layer `layer` (0-based) from the last cached decode
+ * step (Algorithm 1, phase 1: the k_l tokens per sequence whose proxy drifted
+ * most, ascending): copies B * k_l int32 values, [B, k_l], into idx_out
+ * (device), asynchronously on `stream`.  Undefined before the first cached
+ * step (a rho = 1 step selects every row and does not write it). */
+int spa_model_index_set(const spa_model *model, int layer, int32_t *idx_out, void *stream);
 /* h0[b, i] <- embed[tokens[b, i]] for every position (tokens: [B, N] int32 device). */
 int spa_model_embed(spa_model *model, const int32_t *tokens, void *stream);
 
@@ -281,6 +287,28 @@ int spa_decode_graph_launch(spa_model *model, void *stream);
  * (null model), SPA_ERR_NOMEM. */
 int spa_model_set_incremental_proxy(spa_model *model, int enable);
 
+/* ------------------------------------------------------- testing hooks --
+ * No counterpart on the pages: hooks that let tests drive the failure paths
+ * without faulting or hanging a GPU.
+ *
+ * spa_debug_fail_alloc_after(n): after n more successful device allocations
+ * made by the library (workspaces, layer proxy weights, model buffers, the
+ * incremental-proxy state), the next one fails once, as if the device were
+ * out of memory; the call that made it returns SPA_ERR_NOMEM having freed
+ * what it had allocated.  n < 0 switches the injection off.  Process-wide;
+ * returns SPA_OK.
+ *
+ * spa_debug_bounded_wait(ws, flag, expect, limit_us, stream): launches one
+ * bounded device-side wait that records a time-out in the workspace's error
+ * word (spa_workspace_status then returns SPA_ERR_TIMEOUT) if it has not
+ * completed after limit_us microseconds (0 <= limit_us <= 1e6).  flag NULL:
+ * the wait is on a shared-memory barrier that nothing completes, the kind of
+ * wait every pipelined kernel of the library bounds; otherwise it waits
+ * until the device int *flag equals expect.  Errors: SPA_ERR_INVALID,
+ * SPA_ERR_CUDA. */
+int spa_debug_fail_alloc_after(long long n);
+int spa_debug_bounded_wait(spa_workspace *ws, const int *flag, int expect, double limit_us, void *stream);
+
 /* ------------------------------------------------- allocation-free variant --
  * No counterpart on the pages: an engineering addition for callers that may
  * not allocate device memory (custom memory managers and allocator hooks that
@@ -293,18 +321,31 @@ int spa_model_set_incremental_proxy(spa_model *model, int enable);
  * rows.  Q [B, k, n_heads * 128] (the compact selected queries, post-RoPE),
  * k_cache, v_cache [B, N, n_heads * 128], O [B, k, n_heads * 128]: device,
  * bf16, row-major, caller-owned.  It allocates nothing: the split-over-keys
- * partials live in one fixed 8 MiB array inside the library (held on every
- * GPU that loads it until the process exits), so B * k * (n_heads * 130)
- * fp32 values must fit in 2 Mi floats; larger calls return SPA_ERR_SHAPE and
- * launch nothing.  The first call on each device looks up the array's device
- * address (cudaGetSymbolAddress) with that device current; make that first
- * call before any stream capture.  Every call on a device shares the array:
- * calls whose work overlaps on the GPU (other streams, other host threads)
- * race, so order them on one stream.  Errors: SPA_ERR_INVALID (null
- * pointer), SPA_ERR_SHAPE, SPA_ERR_UNSUPPORTED (head_dim != 128),
- * SPA_ERR_CUDA; details in spa_last_error(). */
+ * partials, the per-query-tile split counters and a device error word live
+ * in one fixed 8 MiB array inside the library (held on every GPU that loads
+ * it until the process exits).  The keys of a query tile are split across
+ * CTAs only as far as that array holds the partials (B * k * (n_heads * 130)
+ * fp32 values within 2 Mi floats, and B * n_heads * ceil(k / 128) query tiles
+ * within 4096 counters); a larger call is not refused but splits less, down to
+ * no split, which needs no scratch (it is then slower for long caches).  The
+ * first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call on a device shares the array: calls
+ * whose work overlaps on the GPU (other streams, other host threads) race, so
+ * order them on one stream.  Errors: SPA_ERR_INVALID (null pointer),
+ * SPA_ERR_SHAPE (k > N, or B, n_heads or the cache beyond the launch limits:
+ * B, n_heads <= 65535 and fewer than 2^31 elements per cache),
+ * SPA_ERR_UNSUPPORTED (head_dim != 128), SPA_ERR_CUDA; details in
+ * spa_last_error().  Device-side failures (a bounded wait that ran out) are
+ * kept in the error word until spa_attention_noalloc_status reads them. */
 int spa_attention_noalloc(const void *Q, const void *k_cache, const void *v_cache, void *O, int B,
                           int k, int N, int n_heads, int head_dim, void *stream);
+/* Synchronises `stream`, then reads and clears the error word of the
+ * allocation-free attention on the current device (into host stack memory:
+ * it allocates nothing either): SPA_OK, SPA_ERR_TIMEOUT (a bounded wait of
+ * some call since the last read ran out; that call's O rows are not valid)
+ * or SPA_ERR_DEVICE; SPA_ERR_CUDA if the stream or the copy failed. */
+int spa_attention_noalloc_status(void *stream);
 
 #ifdef __cplusplus
 }

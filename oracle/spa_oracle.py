@@ -366,10 +366,14 @@ def init_decode_state(model: OracleModel, tokens: np.ndarray) -> DecodeState:
     return DecodeState(tokens=tokens, H0=H0, caches=[None] * len(model.layers), step=0)
 
 
-def lm_head_argmax(model: OracleModel, h: np.ndarray) -> tuple:
+def lm_head_argmax(model: OracleModel, h: np.ndarray, bf16_input: bool = False) -> tuple:
     """Final RMSNorm, logits over the vocabulary, argmax with the lowest
-    index on ties (reading A14/A15: only the positions being unmasked)."""
+    index on ties (reading A14/A15: only the positions being unmasked).
+    bf16_input rounds the normalised rows to bf16 before the LM head, the
+    rounding point of a bf16 model (reading A18)."""
     x = rmsnorm(h, model.final_norm, model.eps)
+    if bf16_input:
+        x = round_bf16(x)
     logits = x @ np.asarray(model.lm_head, dtype=np.float64).T
     return np.argmax(logits, axis=-1).astype(np.int64), logits
 
@@ -405,10 +409,12 @@ def decode_step(model: OracleModel, state: DecodeState, positions: np.ndarray,
     tokens; the tokens written are `forced` when given (teacher forcing),
     else the argmax.  The next step's layer-0 input changes only at those rows
     [NOTES 研究背景与动机; reading A14].  Updates `state`; returns the argmax
-    ids, the written ids and per-layer index sets."""
+    ids, the written ids, per-layer index sets and per-layer drift scores
+    (None for a full step)."""
     B = state.tokens.shape[0]
     Ls = len(model.layers)
     index_sets = [[None] * B for _ in range(Ls)]
+    scores = [[None] * B for _ in range(Ls)]
     h_final = np.zeros((B, positions.shape[1], state.H0.shape[2]))
     for b in range(B):
         H = state.H0[b]
@@ -423,6 +429,7 @@ def decode_step(model: OracleModel, state: DecodeState, positions: np.ndarray,
                 cache = state.caches[l][b]
                 out = layer_step(layer, H, cache, k_per_layer[l])
                 index_sets[l][b] = out["I"]
+                scores[l][b] = out["s"]
             H = state.caches[l][b].H_c
         h_final[b] = H[positions[b]]
     argmax, logits = lm_head_argmax(model, h_final)
@@ -432,4 +439,4 @@ def decode_step(model: OracleModel, state: DecodeState, positions: np.ndarray,
         state.tokens[b, positions[b]] = written[b]
         state.H0[b, positions[b]] = emb[written[b]]
     state.step += 1
-    return {"argmax": argmax, "written": written, "logits": logits, "I": index_sets}
+    return {"argmax": argmax, "written": written, "logits": logits, "I": index_sets, "s": scores}

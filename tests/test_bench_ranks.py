@@ -3,6 +3,7 @@ process groups over 127.0.0.1, the max-over-ranks timing every rank joins,
 the whole-job throughput, and the reference arm leaving non-zero ranks
 without work.  The GPU path replicates the model per GPU with no data-path
 collective, so these are the only cross-rank steps."""
+import json
 import os
 import socket
 import subprocess
@@ -55,3 +56,30 @@ def test_reference_arm_nonzero_rank_exits_without_work():
                        capture_output=True, text=True, env=env, timeout=120)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_world_size_must_match_gpus():
+    assert bench.check_world(1, {}) == 1
+    assert bench.check_world(2, {}) == 0            # outside a launcher: start the ranks
+    assert bench.check_world(2, {"WORLD_SIZE": "2"}) == 2
+    with pytest.raises(SystemExit):
+        bench.check_world(8, {"WORLD_SIZE": "1"})
+    argv = bench.launch_argv(2, ["--gpus", "2"], 29512)
+    assert argv[1:4] == ["-m", "torch.distributed.run", "--nnodes=1"]
+    assert "--nproc-per-node=2" in argv and "127.0.0.1" in argv and argv[-2:] == ["--gpus", "2"]
+
+
+def test_gpus_2_without_launcher_starts_two_ranks():
+    # the reference arm needs no GPU: run as `bench.py --gpus 2` outside any
+    # launcher, it relaunches itself as two gloo-free ranks; rank 0 prints the
+    # one line (n_gpus = 2), rank 1 exits without work, and the status is 0
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "1", "--warmup", "0"],
+                       capture_output=True, text=True, env=env, timeout=900)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["n_gpus"] == 2
+    assert rec["extrapolated_x32"] is True and rec["steps"] == 1

@@ -42,10 +42,48 @@ def _tiny_model(dtype, shape, L, vocab, B, N, rho, seed, N_max=None):
     return model, om, lps, caches, h0, keep
 
 
-def test_tiny_decode_loop_teacher_forced():
+def _check_index_sets(model, ref, B, what):
+    """Every layer's index set of the cached step the GPU has just run against
+    the oracle's (exact, or valid within the score margin)."""
+    for l in range(len(model.k)):
+        I_gpu = model.index_set(l).cpu().numpy()
+        for b in range(B):
+            assert_index_set(I_gpu[b], ref["s"][l][b], model.k[l], ref["I"][l][b], f"{what} layer {l} seq {b} I")
+
+
+def _check_lm_head(model, om, caches, pos, u, B, bf16, tok_step, what):
+    """The LM head on the GPU's own final-layer rows at pos, through the
+    confidence pass (the argmax GEMM epilogue that also keeps per-tile sums
+    of exp), against the oracle's logits on the same rows: the argmax ids
+    where the oracle's top-2 gap is clear, every softmax probability of the
+    argmax within 1e-3 relative, and the step's own ids equal to these."""
+    tok = torch.empty((B, u), dtype=torch.int32, device="cuda")
+    conf = torch.empty((B, u), dtype=torch.float32, device="cuda")
+    spa.spa_decode_confidence(model, pos, u, tok, conf)
+    torch.cuda.synchronize()
+    p = pos.cpu().numpy()
+    hrows = np.stack([np64(caches[-1].h[b])[p[b]] for b in range(B)])
+    _, logits = O.lm_head_argmax(om, hrows, bf16_input=bf16)
+    got_tok, got_conf = tok.cpu().numpy(), conf.cpu().numpy().astype(np.float64)
+    assert np.array_equal(got_tok, tok_step.cpu().numpy()), what + ": confidence pass ids differ from the step's"
+    for b in range(B):
+        ids_ref, conf_ref = O.confidence(logits[b])
+        assert np.max(np.abs(got_conf[b] - conf_ref) / conf_ref) < 1e-3, f"{what} seq {b} confidence"
+        for j in range(u):
+            top2 = np.sort(logits[b, j])[-2:]
+            if top2[1] - top2[0] > 1e-4 * max(1.0, abs(top2[1])):
+                assert got_tok[b, j] == ids_ref[j], f"{what} seq {b} position {p[b, j]} argmax"
+
+
+@pytest.mark.parametrize("inc", [False, True])
+def test_tiny_decode_loop_teacher_forced(inc):
+    """Teacher-forced decode steps against the oracle, with the plain proxy
+    (every row projected at every layer) and the incremental proxy (only rows
+    whose layer input changed): ids, index sets of every layer, K^c, H^c, h0."""
     B, N, vocab, steps, u = 1, 64, 1024, 8, 2
     model, om, lps, caches, h0, keep = _tiny_model(spa.SPA_F32, synth.TINY_LAYER, 2, vocab, B, N,
                                                    0.25, seed=0)
+    model.set_incremental_proxy(inc)
     assert model.k == [16, 16]
     job = synth.decode_inputs(B=B, N=N, n_prompt=32, vocab=vocab, steps=steps, u=u, seed=5)
     toks = torch.from_numpy(job.tokens.astype(np.int32)).cuda()
@@ -59,6 +97,9 @@ def test_tiny_decode_loop_teacher_forced():
         lps[0].ws.check()
         ref = O.decode_step(om, state, job.positions[t], model.k, full=(t == 0),
                             forced=job.forced[t])
+        if t > 0:
+            _check_index_sets(model, ref, B, f"step {t}")
+        _check_lm_head(model, om, caches, pos, u, B, False, tok_out, f"step {t}")
         # argmax ids: equal wherever the oracle's top-2 logit gap is clear
         got = tok_out.cpu().numpy()
         lg = ref["logits"]
@@ -105,14 +146,18 @@ def test_tiny_decode_full_k_matches_vanilla():
 SMALL_BF16 = synth.LayerShape(d=256, n_heads=2, head_dim=128, ffn=384, r=16)
 
 
-def test_bf16_decode_loop_and_graph_replay():
+@pytest.mark.parametrize("inc", [False, True])
+def test_bf16_decode_loop_and_graph_replay(inc):
     """bf16 model (2 layers of d=256, vocab 8192 so the LM head uses wide
-    weight tiles): teacher-forced steps against the oracle, then the same
-    steps replayed from a captured CUDA graph must reproduce the directly
-    launched steps bit for bit."""
+    weight tiles), plain or incremental proxy: teacher-forced steps against
+    the oracle (index sets of every layer, H^c, and the tensor-core LM head
+    with its argmax and softmax-probability epilogue on the GPU's final rows),
+    then the same steps replayed from a captured CUDA graph must reproduce the
+    directly launched steps bit for bit."""
     B, N, vocab, steps, u = 2, 96, 8192, 4, 2
     model, om, lps, caches, h0, keep = _tiny_model(spa.SPA_BF16, SMALL_BF16, 2, vocab, B, N,
                                                    0.3, seed=50)
+    model.set_incremental_proxy(inc)
     job = synth.decode_inputs(B=B, N=N, n_prompt=32, vocab=vocab, steps=steps, u=u, seed=51)
     toks = torch.from_numpy(job.tokens.astype(np.int32)).cuda()
     model.embed_tokens(toks)
@@ -126,6 +171,9 @@ def test_bf16_decode_loop_and_graph_replay():
         lps[0].ws.check()
         ref = O.decode_step(om, state, job.positions[t], model.k, full=(t == 0),
                             forced=job.forced[t])
+        if t > 0:
+            _check_index_sets(model, ref, B, f"bf16 step {t}")
+        _check_lm_head(model, om, caches, pos, u, B, True, tok_out[t], f"bf16 step {t}")
         got = tok_out[t].cpu().numpy()
         lg = ref["logits"]
         for b in range(B):

@@ -16,6 +16,9 @@ and by property:
   them are compared with the GPU's: the index set (exact, or valid within the
   score margin), Q, O, H1, A and the rewritten K^c, V^c, H^c, P^c rows, with
   the bf16 tolerance; the rows outside I stay bit-identical.
+- the full-vocabulary LM head of that step (argmax ids and their softmax
+  probabilities through the confidence pass) against the oracle's logits on
+  the GPU's final-layer rows.
 Layers run through spa_layer_step, the call spa_decode_step makes."""
 import gc
 
@@ -71,6 +74,39 @@ def _build(B, N, seed):
     return model, ws, layers, caches, weights, (embed, lm_head, h0, ones)
 
 
+def _check_lm_head(model, caches, lm_head, pos, u, B, tok_step):
+    """The full-vocabulary LM head (126464 x 4096, the tensor-core argmax
+    GEMM with per-tile sums of exp) on the GPU's final-layer rows at pos,
+    through the confidence pass, against the oracle's logits on the same rows
+    (the normalised rows rounded to bf16, the bf16 model's rounding point):
+    every argmax id whose top-2 gap is clear, every softmax probability of the
+    argmax within 1e-3 relative, and the step's ids equal to the pass's.  The
+    oracle runs over row blocks of the LM head (logits of different vocabulary
+    rows are independent), which keeps its fp64 copy small."""
+    tok = torch.empty((B, u), dtype=torch.int32, device="cuda")
+    conf = torch.empty((B, u), dtype=torch.float32, device="cuda")
+    spa.spa_decode_confidence(model, pos, u, tok, conf)
+    torch.cuda.synchronize()
+    p = pos.cpu().numpy()
+    h = np.stack([caches[-1].h[b][pos[b].long()].float().cpu().numpy() for b in range(B)]).astype(np.float64)
+    ones = np.ones(D)
+    parts = []
+    for v0 in range(0, VOCAB, 16384):
+        chunk = lm_head[v0:v0 + 16384].float().cpu().numpy()
+        om = O.OracleModel(layers=[], embed=None, final_norm=ones, lm_head=chunk, eps=1e-5)
+        parts.append(O.lm_head_argmax(om, h, bf16_input=True)[1])
+    logits = np.concatenate(parts, axis=-1)
+    got_tok, got_conf = tok.cpu().numpy(), conf.cpu().numpy().astype(np.float64)
+    assert np.array_equal(got_tok, tok_step.cpu().numpy()), "confidence pass ids differ from the step's"
+    for b in range(B):
+        ids_ref, conf_ref = O.confidence(logits[b])
+        assert np.max(np.abs(got_conf[b] - conf_ref) / conf_ref) < 1e-3, f"seq {b} confidence"
+        for j in range(u):
+            top2 = np.sort(logits[b, j])[-2:]
+            if top2[1] - top2[0] > 1e-4 * max(1.0, abs(top2[1])):
+                assert got_tok[b, j] == ids_ref[j], f"seq {b} position {p[b, j]} argmax"
+
+
 def _run(B, N, n_prompt, u, sample_layers, seqs, check_graph):
     stream = torch.cuda.Stream()
     with torch.cuda.stream(stream):
@@ -122,6 +158,7 @@ def _run_on_stream(B, N, n_prompt, u, sample_layers, seqs, check_graph):
         spa.spa_decode_step(model, pos[2], None, u, 0, tok_out[2])
         ws.check()
     torch.cuda.synchronize()
+    _check_lm_head(model, caches, keep[1], pos[2], u, B, tok_out[2])
 
     # step 3, layer by layer, with sampled oracle checks
     for l in range(L):

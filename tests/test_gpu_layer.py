@@ -34,9 +34,25 @@ def _compare_cache(lp, cache, ocs, what):
     assert np.max(np.abs(p - np.stack([c.P_c for c in ocs]))) < (2e-3 if bf else 1e-5), what + " P^c"
 
 
+def _compare_rewritten_rows(lp, cache, ocs, I_gpu, before, what):
+    """After a cached step: the rewritten rows K^c/V^c/H^c[I] against the
+    oracle's, each on its own (so the N - k untouched rows cannot dilute the
+    error of the k rewritten ones), and every other row bit-identical to the
+    cache before the step."""
+    after = [np64(t) for t in (cache.k, cache.v, cache.h)]
+    for b in range(I_gpu.shape[0]):
+        I = I_gpu[b].astype(np.int64)
+        keep = np.ones(after[0].shape[1], bool)
+        keep[I] = False
+        for j, (name, ref) in enumerate((("K^c", ocs[b].K_c), ("V^c", ocs[b].V_c), ("H^c", ocs[b].H_c))):
+            assert_close(after[j][b][I], ref[I], lp.bf16, f"{what} seq {b} {name}[I]")
+            assert np.array_equal(after[j][b][keep], before[j][b][keep]), f"{what} seq {b} {name} outside I"
+
+
 def _step(lp, cache, ocs, H2, k, check_intermediates=True):
     """Cached step on both sides, compared phase by phase."""
     B, N, d = H2.shape
+    before = [np64(t) for t in (cache.k, cache.v, cache.h)]
     H2d = lp.to_dev(H2)
     idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
     score = torch.empty((B, N), dtype=torch.float32, device="cuda")
@@ -64,6 +80,7 @@ def _step(lp, cache, ocs, H2, k, check_intermediates=True):
             got = lp.ws.view(name, (M, width), dt)
             ref = np.concatenate([outs[b][key] for b in range(B)])
             assert_close(got, ref, lp.bf16, "step " + key)
+    _compare_rewritten_rows(lp, cache, ocs, I_gpu, before, "step")
     _compare_cache(lp, cache, ocs, "step")
     return I_gpu, outs
 

@@ -76,9 +76,13 @@ def test_pages_facts_fixture():
     rp = facts["rho_p_default"]["value"]
     assert O.rho(12, 32, rp, 12, .06, .06) == rp
     assert facts["r_default"]["value"] == 128
-    # the adaptive curve lowers the mean budget below the peak (25% -> ~16%)
+    # the adaptive curve lowers the mean budget below the peak (25% -> ~16%):
+    # with the decode workload's curve (rho_1 = rho_L = 6%, peak at layer 12
+    # of 32) the mean of k_l / N is 16% to within one percentage point
     ks = O.budget_table(1024, 32, rp, 12, .06, .06)
-    assert sum(ks) / (32 * 1024) < rp
+    mean = sum(ks) / (32 * 1024)
+    assert mean < rp
+    assert abs(mean - facts["mean_rho_adaptive"]["value"]) < 0.01
 
 
 # ------------------------------------------------------------------ SVD proxy
@@ -525,3 +529,23 @@ def test_lm_head_argmax_matches_torch():
     ref = x @ torch.from_numpy(model.lm_head).T
     assert np.max(np.abs(logits - ref.numpy())) < 1e-10
     assert np.array_equal(ids, ref.argmax(-1).numpy())
+
+
+def test_lm_head_bf16_input_rounds_the_normalised_rows():
+    # with the identity as LM head the logits are the normalised rows
+    # themselves: with bf16_input they are those rows rounded to bf16 (each
+    # representable in bf16 and within half a bf16 ulp, 2^-8 relative, of the
+    # unrounded row), and rows already exact in bf16 are left unchanged
+    rng = np.random.default_rng(63)
+    d = 64
+    model = O.OracleModel(layers=[], embed=None, final_norm=np.ones(d), lm_head=np.eye(d), eps=0.0)
+    h = rng.standard_normal((3, d))
+    _, x = O.lm_head_argmax(model, h)
+    _, xr = O.lm_head_argmax(model, h, bf16_input=True)
+    assert np.array_equal(xr.astype(np.float32), synth.bf16_round(xr.astype(np.float32)))
+    assert np.all(np.abs(xr - x) <= 2.0 ** -8 * np.abs(x))
+    assert np.any(xr != x)
+    signs = rng.choice([-1.0, 1.0], size=(2, d))      # rms 1: the normalised row is exactly +-1
+    _, a = O.lm_head_argmax(model, 3.0 * signs)
+    _, b = O.lm_head_argmax(model, 3.0 * signs, bf16_input=True)
+    assert np.array_equal(a, b) and np.allclose(np.abs(a), 1.0)
