@@ -37,7 +37,8 @@ __all__ = [
     "truncation_bound", "proxy_identify", "select_topk", "rmsnorm", "rope",
     "attention", "swiglu_ffn", "OracleLayer", "LayerCache", "empty_cache",
     "phase2_attention", "phase3_ffn_scatter", "partial_block", "layer_step",
-    "full_block", "vanilla_block", "OracleModel", "DecodeState",
+    "full_block", "vanilla_block", "attn_output_identify", "attn_output_layer_step",
+    "attn_output_fill", "OracleModel", "DecodeState",
     "init_decode_state", "decode_step", "lm_head_argmax", "confidence", "confident_positions",
 ]
 
@@ -319,6 +320,55 @@ def full_block(layer: OracleLayer, H: np.ndarray, r: int | None = None) -> tuple
     cache.P_c[:] = a_hat
     out = partial_block(layer, H, np.arange(N), cache)
     return cache, out
+
+
+def attn_output_identify(layer: OracleLayer, H: np.ndarray, cache: LayerCache):
+    """The attention-output identifier, one of the identifiers the pages
+    compare with the Value proxy [NOTES 关键设计 1, Table 1: Query, Key,
+    Value, attention output; GIST Key Findings, identifier ablation].
+
+    Every token's attention output is computed from fresh projections of
+    every row (reading A24): x = RMSNorm(H); Q, K, V = x W_{q,k,v}ᵀ for all N
+    rows, RoPE on Q and K; K^c, V^c ← K, V at every row (the identifier needs
+    them); O = softmax(Q K^cᵀ/√d_h) V^c; ô_i = O_i/‖O_i‖ (0 for a zero row);
+    s_i = ½‖ô_i − P^c_i‖² with P^c holding the cached unit attention outputs
+    (r = d).  Updates K^c and V^c in place; returns (O [N, d], ô, s)."""
+    H = np.asarray(H, dtype=np.float64)
+    N = H.shape[0]
+    _, O = phase2_attention(layer, H, np.arange(N), cache)
+    norm = np.sqrt(np.sum(O * O, axis=1))
+    o_hat = np.zeros_like(O)
+    nz = norm > 0
+    o_hat[nz] = O[nz] / norm[nz, None]
+    diff = o_hat - np.asarray(cache.P_c, dtype=np.float64)
+    return O, o_hat, 0.5 * np.sum(diff * diff, axis=1)
+
+
+def attn_output_layer_step(layer: OracleLayer, H: np.ndarray, cache: LayerCache, k: int) -> dict:
+    """Cached layer step with the attention-output identifier (reading A24):
+    phase 1 scores every token by the drift of its attention output (which
+    refreshes K^c, V^c at every row), selects the k most drifted (lowest index
+    on ties, ascending) and writes P^c[I] ← ô[I]; phase 2 is the attention
+    already computed; phase 3 runs the FFN on the selected rows and scatters
+    into H^c [NOTES 整体框架, Phase 3].  Cache updated in place."""
+    H = np.asarray(H, dtype=np.float64)
+    O, o_hat, s = attn_output_identify(layer, H, cache)
+    I = select_topk(s, k)
+    cache.P_c[I] = o_hat[I]
+    H1, A = phase3_ffn_scatter(layer, H, I, O[I], cache)
+    return {"I": I, "s": s, "O": O[I], "H1": H1, "A": A}
+
+
+def attn_output_fill(layer: OracleLayer, H: np.ndarray) -> tuple:
+    """ρ = 1 fill for the attention-output identifier: the full block, with
+    P^c = ô of every row (r = d)."""
+    H = np.asarray(H, dtype=np.float64)
+    N, d = H.shape
+    cache = empty_cache(N, d, d)
+    O, o_hat, _ = attn_output_identify(layer, H, cache)
+    cache.P_c[:] = o_hat
+    H1, A = phase3_ffn_scatter(layer, H, np.arange(N), O, cache)
+    return cache, {"O": O, "H1": H1, "A": A}
 
 
 def vanilla_block(layer: OracleLayer, H: np.ndarray) -> np.ndarray:

@@ -549,3 +549,73 @@ def test_lm_head_bf16_input_rounds_the_normalised_rows():
     _, a = O.lm_head_argmax(model, 3.0 * signs)
     _, b = O.lm_head_argmax(model, 3.0 * signs, bf16_input=True)
     assert np.array_equal(a, b) and np.allclose(np.abs(a), 1.0)
+
+
+# ------------------------------------------------------- attention-output identifier
+
+def _torch_attention_rows(layer, H):
+    """Every row's attention output and post-RoPE keys / values from torch
+    routines (the first half of _torch_block)."""
+    N, d = H.shape
+    nh, hd = layer.n_heads, layer.head_dim
+    x = F.rms_norm(_t(H), (d,), weight=_t(layer.attn_norm), eps=layer.eps)
+    freq = 10000.0 ** (-torch.arange(hd // 2, dtype=torch.float64) * 2.0 / hd)
+    rot = torch.polar(torch.ones(N, hd // 2, dtype=torch.float64),
+                      torch.arange(N, dtype=torch.float64)[:, None] * freq[None, :])
+
+    def rope_t(t):
+        t = t.view(N, nh, hd)
+        z = torch.complex(t[..., :hd // 2], t[..., hd // 2:]) * rot[:, None, :]
+        return torch.cat([z.real, z.imag], dim=-1)
+
+    q, k = rope_t(F.linear(x, _t(layer.wq))), rope_t(F.linear(x, _t(layer.wk)))
+    v = F.linear(x, _t(layer.wv)).view(N, nh, hd)
+    o = F.scaled_dot_product_attention(q.transpose(0, 1), k.transpose(0, 1), v.transpose(0, 1))
+    return o.transpose(0, 1).reshape(N, d).numpy(), k.reshape(N, d).numpy(), v.reshape(N, d).numpy()
+
+
+def test_attn_output_fill_is_vanilla_with_unit_outputs_cached():
+    layer = _tiny_layer(70)
+    H = np.random.default_rng(71).standard_normal((9, 32))
+    cache, _ = O.attn_output_fill(layer, H)
+    o, k, v = _torch_attention_rows(layer, H)
+    assert np.max(np.abs(cache.H_c - _torch_block(layer, H))) < 1e-12
+    assert np.max(np.abs(cache.P_c - o / np.linalg.norm(o, axis=1, keepdims=True))) < 1e-12
+    assert np.max(np.abs(cache.K_c - k)) < 1e-12 and np.max(np.abs(cache.V_c - v)) < 1e-12
+
+
+def test_attn_output_step_scores_refreshes_and_selects():
+    # the score is the cosine distance of every row's fresh attention output
+    # to the one cached at the fill; every K/V row is refreshed; only the k
+    # selected rows of H^c change; with k = N the step is the vanilla block
+    layer = _tiny_layer(72)
+    rng = np.random.default_rng(73)
+    N, k = 12, 5
+    H = rng.standard_normal((N, 32))
+    H2 = H.copy()
+    H2[[2, 7, 9]] += 0.7 * rng.standard_normal((3, 32))
+    cache, _ = O.attn_output_fill(layer, H)
+    o_old = _torch_attention_rows(layer, H)[0]
+    before = cache.copy()
+    out = O.attn_output_layer_step(layer, H2, cache, k)
+    o_new, k_new, v_new = _torch_attention_rows(layer, H2)
+    ref = np.array([scipy_cosine_distance(o_new[i], o_old[i]) for i in range(N)])
+    assert np.max(np.abs(out["s"] - ref)) < 1e-12
+    assert out["I"].tolist() == sorted(np.lexsort((np.arange(N), -out["s"]))[:k].tolist())
+    assert np.max(np.abs(cache.K_c - k_new)) < 1e-12 and np.max(np.abs(cache.V_c - v_new)) < 1e-12
+    keep = np.setdiff1d(np.arange(N), out["I"])
+    assert np.array_equal(cache.H_c[keep], before.H_c[keep])
+    assert np.max(np.abs(cache.H_c[out["I"]] - _torch_block(layer, H2)[out["I"]])) < 1e-12
+    full = O.attn_output_fill(layer, H)[0]
+    O.attn_output_layer_step(layer, H2, full, N)
+    assert np.max(np.abs(full.H_c - _torch_block(layer, H2))) < 1e-12
+
+
+def test_attn_output_zero_drift_selects_lowest_indices():
+    layer = _tiny_layer(74)
+    H = np.random.default_rng(75).standard_normal((10, 32))
+    cache, _ = O.attn_output_fill(layer, H)
+    before = cache.copy()
+    out = O.attn_output_layer_step(layer, H, cache, 3)
+    assert np.all(out["s"] == 0.0) and out["I"].tolist() == [0, 1, 2]
+    assert np.max(np.abs(cache.H_c - before.H_c)) < 1e-12
