@@ -193,6 +193,9 @@ struct spa_workspace {
   int* attn_sync = nullptr;  // per query tile: attention key splits finished
   int attn_sync_len = 0;
   int* err = nullptr;       // [2]
+  float* sk_part = nullptr;  // stream-K GEMM: partial tiles [2 * num_sms, 128, 256] fp32
+  int* sk_count = nullptr;   // stream-K GEMM: per tile, segments counted
+  int sk_count_len = 0;
   float* rope_cos = nullptr;  // [max_N, hd/2]
   float* rope_sin = nullptr;
   CUtensorMap tmX, tmO, tmX2, tmA;
@@ -207,6 +210,7 @@ struct spa_layer {
   spa_workspace* ws = nullptr;
   void* w_r = nullptr;      // [r, d] dtype
   CUtensorMap tm_wq, tm_wk, tm_wv, tm_wo, tm_wg, tm_wu, tm_wd, tm_wr;
+  CUtensorMap tm_wg64, tm_wu64;  // W_gate, W_up with 64-row boxes (stream-K gate/up tiles)
 };
 
 struct spa_model {
@@ -342,6 +346,11 @@ extern "C" int spa_workspace_create(const spa_layer_desc* desc, int max_B, int m
   ws->attn_sync_len = max_B * desc->n_heads * ((max_N + 127) / 128);
   WS_ALLOC(attn_sync, (size_t)ws->attn_sync_len * sizeof(int))
   WS_ALLOC(err, 2 * sizeof(int))
+  if (desc->dtype == SPA_BF16) {
+    ws->sk_count_len = (int)std::max<size_t>(3 * d / 128, std::max<size_t>(F / 64, d / 128));
+    WS_ALLOC(sk_part, (size_t)2 * ws->num_sms * 128 * 256 * 4)
+    WS_ALLOC(sk_count, (size_t)ws->sk_count_len * sizeof(int))
+  }
   WS_ALLOC(rope_cos, (size_t)max_N * (desc->head_dim / 2) * 4)
   WS_ALLOC(rope_sin, (size_t)max_N * (desc->head_dim / 2) * 4)
 #undef WS_ALLOC
@@ -362,7 +371,8 @@ extern "C" int spa_workspace_create(const spa_layer_desc* desc, int max_B, int m
   if (cudaMemcpy(ws->rope_cos, cs.data(), cs.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
       cudaMemcpy(ws->rope_sin, sn.data(), sn.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
       cudaMemset(ws->err, 0, 2 * sizeof(int)) != cudaSuccess ||
-      cudaMemset(ws->attn_sync, 0, (size_t)ws->attn_sync_len * sizeof(int)) != cudaSuccess) {
+      cudaMemset(ws->attn_sync, 0, (size_t)ws->attn_sync_len * sizeof(int)) != cudaSuccess ||
+      (ws->sk_count && cudaMemset(ws->sk_count, 0, (size_t)ws->sk_count_len * sizeof(int)) != cudaSuccess)) {
     spa_workspace_free(ws);
     return fail(SPA_ERR_CUDA, "workspace initialisation copy failed");
   }
@@ -384,6 +394,9 @@ extern "C" int spa_workspace_status(spa_workspace* ws, void* stream) {
   SPA_CK(cudaMemcpy(h, ws->err, sizeof(h), cudaMemcpyDeviceToHost));
   if (h[0] == 0) return SPA_OK;
   SPA_CK(cudaMemset(ws->err, 0, sizeof(h)));
+  // a kernel that gave up may have left split counters behind: start them afresh
+  SPA_CK(cudaMemset(ws->attn_sync, 0, (size_t)ws->attn_sync_len * sizeof(int)));
+  if (ws->sk_count) SPA_CK(cudaMemset(ws->sk_count, 0, (size_t)ws->sk_count_len * sizeof(int)));
   if (h[0] & DEVERR_TIMEOUT) return fail(SPA_ERR_TIMEOUT, "device wait timed out (site %d)", h[1]);
   return fail(SPA_ERR_DEVICE, "device check failed: bits 0x%x site %d", h[0], h[1]);
 }
@@ -503,7 +516,8 @@ extern "C" int spa_init_layer(const spa_layer_desc* desc, const spa_layer_weight
         (encode_bf16_map(&L->tm_wq, w->wq, D, D) || encode_bf16_map(&L->tm_wk, w->wk, D, D) ||
          encode_bf16_map(&L->tm_wv, w->wv, D, D) || encode_bf16_map(&L->tm_wo, w->wo, D, D) ||
          encode_bf16_map(&L->tm_wg, w->w_gate, F, D) || encode_bf16_map(&L->tm_wu, w->w_up, F, D) ||
-         encode_bf16_map(&L->tm_wd, w->w_down, D, F) || encode_bf16_map(&L->tm_wr, L->w_r, r, D)))
+         encode_bf16_map(&L->tm_wd, w->w_down, D, F) || encode_bf16_map(&L->tm_wr, L->w_r, r, D) ||
+         encode_bf16_map_box(&L->tm_wg64, w->w_gate, F, D, 64) || encode_bf16_map_box(&L->tm_wu64, w->w_up, F, D, 64)))
       st = fail(SPA_ERR_CUDA, "tensor map encoding failed (weights must be 16-byte aligned)");
   } else {
     if (cudaMemcpy(L->w_r, wr.data(), wr.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess)
@@ -626,6 +640,47 @@ static int run_ws(int mode, bool gateup, TcWsParams& p, const void* X, int M, in
   return SPA_OK;
 }
 
+// Stream-K weight-streaming GEMM (M <= 256 tokens): `tiles` weight tiles of
+// 128 output features (gate/up: 64 features, 64 gate + 64 up rows) times the
+// [M, K] bf16 token operand X, K / 64 k-blocks each, over one CTA per SM.
+static bool streamk_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("SPA_STREAMK");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+static int run_sk(int mode, SkParams& p, spa_workspace* ws, const void* X, int M, int K, int tiles,
+                  cudaStream_t s, Profiler* prof, Work w) {
+  if (M <= 0) return SPA_OK;
+  if (M > 256) return fail(SPA_ERR_SHAPE, "stream-K GEMM takes at most 256 tokens");
+  const int NT = ((M + 31) / 32) * 32;
+  if (encode_bf16_map_box(&p.tmX, X, (uint64_t)M, (uint64_t)K, (uint32_t)NT))
+    return fail(SPA_ERR_CUDA, "tensor map for the token operand failed");
+  int cols = 32;
+  while (cols < 2 * NT) cols *= 2;
+  p.K = K;
+  p.KB = K / 64;
+  p.NT = NT;
+  p.n_tiles = tiles;
+  p.units = tiles * p.KB;
+  p.tmem_cols = cols;
+  p.part = ws->sk_part;
+  p.count = ws->sk_count;
+  if (tiles > ws->sk_count_len) return fail(SPA_ERR_SHAPE, "stream-K GEMM: more tiles than counters");
+  // one CTA per SM, at least four k-blocks each
+  int grid = std::max(1, std::min(ws->num_sms, p.units / 4));
+  if (const char* env = std::getenv("SPA_SK_GRID")) {  // tuning / test override, 1..SMs and <= units
+    const int v = std::atoi(env);
+    if (v >= 1 && v <= ws->num_sms && v <= p.units) grid = v;
+  }
+  ProfScope ps(prof, w.cls, w.bytes, w.flops, s);
+  cudaError_t e = launch_tc_sk(mode, p, grid, s);
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "stream-K GEMM launch (mode %d): %s", mode, cudaGetErrorString(e));
+  return SPA_OK;
+}
+
 static int run_simt(int mode, SimtGemmParams& p, int M, int n_tiles, cudaStream_t s, Profiler* prof,
                     Work w) {
   const int m_tiles = (M + 63) / 64;
@@ -709,12 +764,14 @@ static int run_proxy(spa_layer* L, const void* H, const spa_layer_cache* c, floa
 }
 
 // Phases 2 and 3 for M = B * tps tokens; idx == null means every row (rho = 1).
-static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
-                     const spa_layer_cache* c, cudaStream_t s, bool x_ready = false,
-                     void* row_copy = nullptr, float* score_zero = nullptr) {
+// Phase 2: x = RMSNorm(H[I]), Q/K/V with RoPE, K^c/V^c[I] <- K, V, and the
+// attention of the M = B * tps selected queries over the whole cache into
+// ws->O (compact rows); idx == null means every row (rho = 1).
+static int run_attn_half(spa_layer* L, const void* H, const int32_t* idx, int tps,
+                         const spa_layer_cache* c, cudaStream_t s, bool x_ready) {
   spa_workspace* ws = L->ws;
   const spa_layer_desc& D = L->desc;
-  const int d = D.d, F = D.ffn, M = c->B * tps, N = c->N;
+  const int d = D.d, M = c->B * tps, N = c->N;
   const bool bf = D.dtype == SPA_BF16;
   const double es = bf ? 2.0 : 4.0, Md = (double)M * d, Bn = (double)c->B * N;
   Profiler* prof = &ws->prof;
@@ -734,7 +791,15 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
     ep.out = ws->Q;
     ep.k_cache = c->k_cache;
     ep.v_cache = c->v_cache;
-    if (bf && M <= 256) {
+    const int hd = D.head_dim;
+    if (bf && M <= 256 && streamk_enabled() && (hd == 32 || hd == 64 || hd == 128)) {
+      SkParams p;
+      std::memset(&p, 0, sizeof(p));
+      p.tmW[0] = L->tm_wq; p.tmW[1] = L->tm_wk; p.tmW[2] = L->tm_wv;
+      p.b_mode = B_CONCAT3; p.b_rows_per_src = d; p.ep = ep;
+      SPA_TRY(run_sk(EPI_QKV, p, ws, ws->X, M, d, 3 * d / 128, s, prof,
+                     Work{SPA_PROF_QKV, 3.0 * d * d * es + Md * es + 3.0 * Md * es, 6.0 * Md * d}));
+    } else if (bf && M <= 256) {
       TcWsParams p;
       std::memset(&p, 0, sizeof(p));
       p.tmW[0] = L->tm_wq; p.tmW[1] = L->tm_wk; p.tmW[2] = L->tm_wv;
@@ -768,22 +833,44 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
                          ws->attn_sync_len, ws->err, 1, s);
   }
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
+  return SPA_OK;
+}
+
+// Phase 3 for the M = B * tps selected rows whose attention outputs are the
+// compact rows of Ob (tmOb: its tensor map, bf16): H1 = H[I] + O W_o^T,
+// x2 = RMSNorm(H1), A = SwiGLU, H^c[I] = H1 + A W_down^T.
+static int run_ffn_half(spa_layer* L, const void* H, const int32_t* idx, int tps,
+                        const spa_layer_cache* c, cudaStream_t s, const void* Ob, const CUtensorMap* tmOb,
+                        void* row_copy, float* score_zero) {
+  spa_workspace* ws = L->ws;
+  const spa_layer_desc& D = L->desc;
+  const int d = D.d, F = D.ffn, M = c->B * tps, N = c->N;
+  const bool bf = D.dtype == SPA_BF16;
+  const double es = bf ? 2.0 : 4.0, Md = (double)M * d;
+  Profiler* prof = &ws->prof;
+  cudaError_t e;
   // H1 = H[I] + O W_o^T
   {
     EpiParams ep = base_epi(L, M, tps, N, idx);
     ep.n_out = d;
     ep.out = ws->H1;
     ep.resid = H;
-    if (bf && M <= 256) {
+    if (bf && M <= 256 && streamk_enabled()) {
+      SkParams p;
+      std::memset(&p, 0, sizeof(p));
+      p.tmW[0] = L->tm_wo; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
+      SPA_TRY(run_sk(EPI_RESID, p, ws, Ob, M, d, d / 128, s, prof,
+                     Work{SPA_PROF_OPROJ, (double)d * d * es + 3.0 * Md * es, 2.0 * Md * d}));
+    } else if (bf && M <= 256) {
       TcWsParams p;
       std::memset(&p, 0, sizeof(p));
       p.tmW[0] = L->tm_wo; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
-      SPA_TRY(run_ws(EPI_RESID, false, p, ws->O, M, d, d, s, prof,
+      SPA_TRY(run_ws(EPI_RESID, false, p, Ob, M, d, d, s, prof,
                      Work{SPA_PROF_OPROJ, (double)d * d * es + 3.0 * Md * es, 2.0 * Md * d}));
     } else if (bf) {
       TcGemmParams p;
       std::memset(&p, 0, sizeof(p));
-      p.tmA = ws->tmO; p.tmB[0] = L->tm_wo;
+      p.tmA = *tmOb; p.tmB[0] = L->tm_wo;
       p.K = d; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
       const int nt = d / 256, mt = (M + 127) / 128;
       SPA_TRY(run_tc(EPI_RESID, 256, p, M, nt, choose_splits(nt * mt, d / 64, ws->num_sms), s, prof,
@@ -791,7 +878,7 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
     } else {
       SimtGemmParams p;
       std::memset(&p, 0, sizeof(p));
-      p.A = (const float*)ws->O; p.B[0] = (const float*)L->w.wo;
+      p.A = (const float*)Ob; p.B[0] = (const float*)L->w.wo;
       p.K = d; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
       SPA_TRY(run_simt(EPI_RESID, p, M, (d + 127) / 128, s, prof,
                        Work{SPA_PROF_OPROJ, (double)d * d * es + 3.0 * Md * es, 2.0 * Md * d}));
@@ -808,7 +895,13 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
     EpiParams ep = base_epi(L, M, tps, N, idx);
     ep.n_out = F;
     ep.out = ws->A;
-    if (bf && M <= 256) {
+    if (bf && M <= 256 && streamk_enabled()) {
+      SkParams p;
+      std::memset(&p, 0, sizeof(p));
+      p.tmW[0] = L->tm_wg64; p.tmW[1] = L->tm_wu64; p.b_mode = B_GATEUP; p.b_rows_per_src = F; p.ep = ep;
+      SPA_TRY(run_sk(EPI_SWIGLU, p, ws, ws->X2, M, d, F / 64, s, prof,
+                     Work{SPA_PROF_GATEUP, 2.0 * F * d * es + Md * es + (double)M * F * es, 4.0 * Md * F}));
+    } else if (bf && M <= 256) {
       TcWsParams p;
       std::memset(&p, 0, sizeof(p));
       p.tmW[0] = L->tm_wg; p.tmW[1] = L->tm_wu; p.b_mode = B_GATEUP; p.b_rows_per_src = F; p.ep = ep;
@@ -839,7 +932,13 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
     ep.resid = ws->H1;
     ep.row_copy = row_copy;
     ep.score_zero = score_zero;
-    if (bf && M <= 256) {
+    if (bf && M <= 256 && streamk_enabled()) {
+      SkParams p;
+      std::memset(&p, 0, sizeof(p));
+      p.tmW[0] = L->tm_wd; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
+      SPA_TRY(run_sk(EPI_RESID_SCATTER, p, ws, ws->A, M, F, d / 128, s, prof,
+                     Work{SPA_PROF_DOWN, (double)d * F * es + (double)M * F * es + 2.0 * Md * es, 2.0 * Md * F}));
+    } else if (bf && M <= 256) {
       TcWsParams p;
       std::memset(&p, 0, sizeof(p));
       p.tmW[0] = L->tm_wd; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
@@ -863,6 +962,14 @@ static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
     }
   }
   return SPA_OK;
+}
+
+// Phases 2 and 3 for M = B * tps tokens; idx == null means every row (rho = 1).
+static int run_block(spa_layer* L, const void* H, const int32_t* idx, int tps,
+                     const spa_layer_cache* c, cudaStream_t s, bool x_ready = false,
+                     void* row_copy = nullptr, float* score_zero = nullptr) {
+  SPA_TRY(run_attn_half(L, H, idx, tps, c, s, x_ready));
+  return run_ffn_half(L, H, idx, tps, c, s, L->ws->O, &L->ws->tmO, row_copy, score_zero);
 }
 
 static int check_H(const void* H) {
@@ -951,14 +1058,67 @@ extern "C" int spa_layer_step(spa_layer* L, const void* H, const spa_layer_cache
                          nullptr);
 }
 
+// Unit rows of the attention outputs ws->O (M rows of r = d elements) into
+// P^c (fill) or into a_hat with their drift scores against P^c.
+static int score_attn_rows(spa_layer* L, const spa_layer_cache* c, int fill, cudaStream_t s) {
+  spa_workspace* ws = L->ws;
+  const int M = c->B * c->N, d = L->desc.d;
+  const double e = L->desc.dtype == SPA_BF16 ? 2.0 : 4.0;
+  ProfScope ps(&ws->prof, SPA_PROF_PROXY, (double)M * d * e + (fill ? 1.0 : 3.0) * M * d * 4, 0.0, s);
+  const cudaError_t er = launch_unit_rows_score(L->desc.dtype, ws->O, M, d, c->N, c->N, nullptr,
+                                                fill ? nullptr : ws->a_hat, c->p_cache, fill ? nullptr : ws->score,
+                                                fill, ws->err, s);
+  if (er != cudaSuccess) return fail(SPA_ERR_CUDA, "attention-output score launch: %s", cudaGetErrorString(er));
+  return SPA_OK;
+}
+
 extern "C" int spa_full_block(spa_layer* L, const void* H, const spa_layer_cache* c, int fill_proxy,
                               void* stream) {
   if (!L) return fail(SPA_ERR_INVALID, "null layer");
   SPA_TRY(check_H(H));
   SPA_TRY(check_cache(L, c));
+  if (fill_proxy < 0 || fill_proxy > 2) return fail(SPA_ERR_INVALID, "fill_proxy must be 0, 1 or 2");
   cudaStream_t s = (cudaStream_t)stream;
+  if (fill_proxy == 2) {
+    // the attention-output identifier's fill: P^c = unit attention output of every row
+    if (L->desc.r != L->desc.d) return fail(SPA_ERR_SHAPE, "the attention-output identifier needs r = d");
+    SPA_TRY(run_attn_half(L, H, nullptr, c->N, c, s, false));
+    SPA_TRY(score_attn_rows(L, c, 1, s));
+    return run_ffn_half(L, H, nullptr, c->N, c, s, L->ws->O, &L->ws->tmO, nullptr, nullptr);
+  }
   if (fill_proxy) SPA_TRY(run_proxy(L, H, c, nullptr, 1, s));
   return run_block(L, H, nullptr, c->N, c, s);
+}
+
+extern "C" int spa_layer_step_attn_identifier(spa_layer* L, const void* H, const spa_layer_cache* c, int k,
+                                              int32_t* idx, void* stream) {
+  if (!L) return fail(SPA_ERR_INVALID, "null layer");
+  SPA_TRY(check_H(H));
+  SPA_TRY(check_cache(L, c));
+  if (!idx) return fail(SPA_ERR_INVALID, "null idx");
+  if (k < 1 || k > c->N) return fail(SPA_ERR_SHAPE, "k=%d outside [1, N=%d]", k, c->N);
+  if (L->desc.r != L->desc.d) return fail(SPA_ERR_SHAPE, "the attention-output identifier needs r = d");
+  cudaStream_t s = (cudaStream_t)stream;
+  spa_workspace* ws = L->ws;
+  const spa_layer_desc& D = L->desc;
+  // phase 1: every row's attention output from fresh Q/K/V (K^c, V^c rewritten
+  // at every row), its drift score, the top-k and P^c[I] <- unit output
+  SPA_TRY(run_attn_half(L, H, nullptr, c->N, c, s, false));
+  SPA_TRY(score_attn_rows(L, c, 0, s));
+  cudaError_t e;
+  const double Bn = (double)c->B * c->N, Bk = (double)c->B * k, es = D.dtype == SPA_BF16 ? 2.0 : 4.0;
+  {
+    ProfScope ps(&ws->prof, SPA_PROF_TOPK, 4.0 * Bn + 8.0 * Bk * D.r + 4.0 * Bk, 0.0, s);
+    e = launch_topk_select(ws->score, c->B, c->N, k, idx, ws->a_hat, c->p_cache, D.r, ws->err, s);
+  }
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "select launch: %s", cudaGetErrorString(e));
+  // phase 2 is done: the selected rows' outputs, compact, feed phase 3
+  {
+    ProfScope ps(&ws->prof, SPA_PROF_MISC, 2.0 * Bk * D.d * es, 0.0, s);
+    e = launch_gather_rows(D.dtype, ws->O, idx, c->B, k, c->N, D.d, ws->X, ws->err, s);
+  }
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "gather launch: %s", cudaGetErrorString(e));
+  return run_ffn_half(L, H, idx, k, c, s, ws->X, &ws->tmX, nullptr, nullptr);
 }
 
 // ---------------------------------------------------------------------------

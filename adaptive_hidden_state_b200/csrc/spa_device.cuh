@@ -123,6 +123,33 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Plain arrive (count one) on an mbarrier of this CTA.
+__device__ __forceinline__ void mbar_arrive_cta(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Bounded wait that ignores any abort flag: for copies and tensor-core
+// operations already in flight, which must land before shared memory or
+// TMEM is released.  Records a time-out and returns false after limit_ns.
+__device__ __forceinline__ bool mbar_drain_bounded(uint64_t* bar, uint32_t parity, int* err, int site,
+                                                   unsigned long long limit_ns = kWaitLimitNs) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer() - t0 > limit_ns) {
+      report_error(err, DEVERR_TIMEOUT, site);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Named barrier `id` over `n` threads (whole warps).
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 // Wait until the global int *flag equals `expect` (acquire: what the writer
 // stored before releasing the flag is visible afterwards).  Gives up after
 // limit_ns and records the error.  Returns true when the flag was seen.

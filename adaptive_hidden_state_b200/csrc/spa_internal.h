@@ -81,6 +81,24 @@ struct alignas(64) TcWsParams {
   EpiParams ep;
 };
 
+// Stream-K weight-streaming GEMM (spa_streamk.cu): tiles of 128 output
+// features (gate/up: 64 gate + the same 64 up rows), units (tile, 64-column
+// k-block) split evenly over the grid's CTAs.
+struct alignas(64) SkParams {
+  CUtensorMap tmW[3];  // weight sources, box 64 x 128 rows (B_GATEUP: 64 rows)
+  CUtensorMap tmX;     // token rows [M, K], box 64 x NT, 128-byte swizzle
+  int K, KB;           // reduction length and its 64-column blocks
+  int NT;              // tokens per MMA (multiple of 32, <= 256)
+  int n_tiles;         // 128-row weight tiles
+  int units;           // n_tiles * KB
+  int tmem_cols;       // power of two >= 2 * NT (two accumulators)
+  int b_mode;
+  int b_rows_per_src;
+  float* part;         // [2 * grid, 128, NT] fp32 partial tiles of split tiles
+  int* count;          // [n_tiles] segments counted (zero between launches)
+  EpiParams ep;
+};
+
 struct SimtGemmParams {
   const float* A;      // [M, K]
   const float* B[3];
@@ -100,6 +118,9 @@ cudaError_t launch_tc_gemm(int mode, int BN, const TcGemmParams& p, int m_tiles,
 cudaError_t launch_tc_ws(int mode, int nacc, const TcWsParams& p, int n_tiles, int splits,
                          cudaStream_t stream);
 int plan_ws_splits(int mode, int nacc, int n_tiles, int KB);
+// Stream-K weight-streaming GEMM over `grid` CTAs (one per SM).
+cudaError_t launch_tc_sk(int mode, const SkParams& p, int grid, cudaStream_t stream);
+int sk_stages(int NT);
 // Encodes a 2D bf16 tensor map with a 64 x box_rows box.
 int encode_bf16_map_box(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                         uint32_t box_rows);
@@ -136,6 +157,14 @@ cudaError_t launch_topk_select(const float* score, int B, int N, int k, int32_t*
 cudaError_t launch_proxy_finish(const float* raw, int M, int r, int tps, int N, const int32_t* idx,
                                 float* a_hat, float* p_cache, float* score, int fill, int* err,
                                 cudaStream_t stream);
+// The same per-row finish on rows of dtype elements (1 = bf16, 0 = fp32):
+// the attention-output identifier scores every row's attention output.
+cudaError_t launch_unit_rows_score(int dtype, const void* rows, int M, int r, int tps, int N,
+                                   const int32_t* idx, float* a_hat, float* p_cache, float* score, int fill,
+                                   int* err, cudaStream_t stream);
+// dst[b * k + j] = src[b * N + idx[b * k + j]] (rows of d dtype elements; d * size a multiple of 16 bytes).
+cudaError_t launch_gather_rows(int dtype, const void* src, const int32_t* idx, int B, int k, int N, int d,
+                               void* dst, int* err, cudaStream_t stream);
 bool select_norm_supported(int dtype, int N, int d);
 cudaError_t launch_select_norm(int dtype, const float* score, int B, int N, int k, int32_t* idx,
                                const float* a_hat, float* p_cache, int r, const void* H,

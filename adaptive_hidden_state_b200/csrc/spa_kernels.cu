@@ -410,7 +410,8 @@ cudaError_t launch_select_norm(int dtype, const float* score, int B, int N, int 
 // score (block sums in a fixed order), and writes them at the token's cache
 // row.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) proxy_finish_kernel(const float* raw, int M, int r, int tps, int N,
+template <typename T>
+__global__ void __launch_bounds__(256) proxy_finish_kernel(const T* raw, int M, int r, int tps, int N,
                                                            const int32_t* idx, float* a_hat,
                                                            float* p_cache, float* score, int fill,
                                                            int* err) {
@@ -426,7 +427,7 @@ __global__ void __launch_bounds__(256) proxy_finish_kernel(const float* raw, int
     return;
   }
   const size_t dst = ((size_t)b * N + pos) * r;
-  const float* a = raw + (size_t)t * r;
+  const T* a = raw + (size_t)t * r;
   auto block_sum = [&](float v) {
     v = warp_sum(v);
     __syncthreads();  // red[] is reused by the next sum
@@ -438,12 +439,15 @@ __global__ void __launch_bounds__(256) proxy_finish_kernel(const float* raw, int
     return s;
   };
   float ss = 0.f;
-  for (int c = threadIdx.x; c < r; c += 256) ss += a[c] * a[c];
+  for (int c = threadIdx.x; c < r; c += 256) {
+    const float x = to_f(a[c]);
+    ss += x * x;
+  }
   ss = block_sum(ss);
   const float nrm = sqrtf(ss);
   float sd = 0.f;
   for (int c = threadIdx.x; c < r; c += 256) {
-    const float ah = ss > 0.f ? a[c] / nrm : 0.f;
+    const float ah = ss > 0.f ? to_f(a[c]) / nrm : 0.f;
     if (fill) {
       p_cache[dst + c] = ah;
       if (a_hat) a_hat[dst + c] = ah;
@@ -465,8 +469,52 @@ cudaError_t launch_proxy_finish(const float* raw, int M, int r, int tps, int N, 
                                 float* a_hat, float* p_cache, float* score, int fill, int* err,
                                 cudaStream_t stream) {
   if (M <= 0) return cudaSuccess;
-  return launch_k(proxy_finish_kernel, dim3(M), dim3(256), 0, stream, raw, M, r, tps, N, idx, a_hat,
+  return launch_k(proxy_finish_kernel<float>, dim3(M), dim3(256), 0, stream, raw, M, r, tps, N, idx, a_hat,
                   p_cache, score, fill, err);
+}
+
+cudaError_t launch_unit_rows_score(int dtype, const void* rows, int M, int r, int tps, int N,
+                                   const int32_t* idx, float* a_hat, float* p_cache, float* score, int fill,
+                                   int* err, cudaStream_t stream) {
+  if (M <= 0) return cudaSuccess;
+  if (dtype == 1)
+    return launch_k(proxy_finish_kernel<__nv_bfloat16>, dim3(M), dim3(256), 0, stream,
+                    (const __nv_bfloat16*)rows, M, r, tps, N, idx, a_hat, p_cache, score, fill, err);
+  return launch_k(proxy_finish_kernel<float>, dim3(M), dim3(256), 0, stream, (const float*)rows, M, r, tps,
+                  N, idx, a_hat, p_cache, score, fill, err);
+}
+
+// ---------------------------------------------------------------------------
+// Gather: dst[t] = src[b * N + idx[t]] for the M = B * k selected rows
+// (t = b * k + j), 16 bytes per thread step.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(128) gather_rows_kernel(const T* src, const int32_t* idx, int k, int N,
+                                                         int M, int d, T* dst, int* err) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int t = blockIdx.x;
+  if (t >= M) return;
+  const int b = t / k, pos = idx[t];
+  if (pos < 0 || pos >= N) {
+    if (threadIdx.x == 0) report_error(err, DEVERR_INDEX, 702);
+    return;
+  }
+  const uint4* s4 = reinterpret_cast<const uint4*>(src + ((size_t)b * N + pos) * d);
+  uint4* d4 = reinterpret_cast<uint4*>(dst + (size_t)t * d);
+  const int nch = d * (int)sizeof(T) / 16;
+  for (int c = threadIdx.x; c < nch; c += 128) d4[c] = s4[c];
+}
+
+cudaError_t launch_gather_rows(int dtype, const void* src, const int32_t* idx, int B, int k, int N, int d,
+                               void* dst, int* err, cudaStream_t stream) {
+  const int M = B * k;
+  if (M <= 0) return cudaSuccess;
+  if (dtype == 1)
+    return launch_k(gather_rows_kernel<__nv_bfloat16>, dim3(M), dim3(128), 0, stream,
+                    (const __nv_bfloat16*)src, idx, k, N, M, d, (__nv_bfloat16*)dst, err);
+  return launch_k(gather_rows_kernel<float>, dim3(M), dim3(128), 0, stream, (const float*)src, idx, k, N, M,
+                  d, (float*)dst, err);
 }
 
 // ---------------------------------------------------------------------------

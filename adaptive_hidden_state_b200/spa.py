@@ -33,6 +33,7 @@ EXPORTS = [
     "spa_workspace_status", "spa_workspace_intermediates", "spa_profile_enable",
     "spa_profile_read", "spa_launch_count", "spa_init_layer", "spa_free_layer", "spa_layer_proxy_weights",
     "spa_proxy_select", "spa_partial_block", "spa_layer_step", "spa_full_block",
+    "spa_layer_step_attn_identifier",
     "spa_model_create", "spa_model_free", "spa_model_layer_k", "spa_model_index_set", "spa_model_embed",
     "spa_decode_step", "spa_decode_layers", "spa_decode_confidence", "spa_model_write_tokens",
     "spa_decode_graph_capture", "spa_decode_graph_launch",
@@ -111,6 +112,8 @@ _sig("spa_partial_block", c_int, c_void_p, c_void_p, c_void_p, c_int, POINTER(La
 _sig("spa_layer_step", c_int, c_void_p, c_void_p, POINTER(LayerCacheDesc), c_int, c_void_p,
      c_void_p)
 _sig("spa_full_block", c_int, c_void_p, c_void_p, POINTER(LayerCacheDesc), c_int, c_void_p)
+_sig("spa_layer_step_attn_identifier", c_int, c_void_p, c_void_p, POINTER(LayerCacheDesc), c_int, c_void_p,
+     c_void_p)
 _sig("spa_model_create", c_int, POINTER(ModelDesc), POINTER(c_void_p), POINTER(LayerCacheDesc),
      c_void_p, c_void_p, c_void_p, c_void_p, POINTER(c_void_p))
 _sig("spa_model_free", None, c_void_p)
@@ -303,9 +306,15 @@ def spa_layer_step(layer: Layer, H, cache: Cache, k: int, idx, stream=None):
                               _stream(stream)), "spa_layer_step")
 
 
-def spa_full_block(layer: Layer, H, cache: Cache, fill_proxy: bool = True, stream=None):
+def spa_full_block(layer: Layer, H, cache: Cache, fill_proxy: int = 1, stream=None):
+    """fill_proxy: 0 none, 1 (or True) the value proxy, 2 unit attention outputs."""
     _check(lib.spa_full_block(layer.handle, _ptr(H), ctypes.byref(cache.desc), int(fill_proxy),
                               _stream(stream)), "spa_full_block")
+
+
+def spa_layer_step_attn_identifier(layer: Layer, H, cache: Cache, k: int, idx, stream=None):
+    _check(lib.spa_layer_step_attn_identifier(layer.handle, _ptr(H), ctypes.byref(cache.desc), k, _ptr(idx),
+                                              _stream(stream)), "spa_layer_step_attn_identifier")
 
 
 class Model:

@@ -192,9 +192,28 @@ int spa_layer_step(spa_layer *layer, const void *H, const spa_layer_cache *cache
 
 /* rho = 1 pass (the uncached forward): every row of K^c, V^c and H^c is
  * recomputed from H.  fill_proxy = 1 also writes P^c = a_hat of every row
- * (the cache fill that starts a decode); 0 skips the proxy entirely. */
+ * (the cache fill that starts a decode); 0 skips the proxy entirely; 2 fills
+ * P^c with every row's unit attention output instead, the fill of the
+ * attention-output identifier below (needs r = d). */
 int spa_full_block(spa_layer *layer, const void *H, const spa_layer_cache *cache, int fill_proxy,
                    void *stream);
+
+/* A cached layer step with the attention output as the update identifier,
+ * the variant the pages compare with the Value proxy (papernotes.org, 关键设计
+ * 1 and Table 1: Query, Key, Value or attention output as identifier).  Its
+ * cost is the point: scoring a token by the drift of its attention output
+ * needs that output for every token, so phase 1 runs the attention
+ * sub-layer for all N rows: x = RMSNorm(H), Q/K/V of every row with RoPE,
+ * K^c, V^c rewritten at every row, O = softmax(Q K^cT / sqrt(d_h)) V^c; then
+ * o_hat = O / |O|, s = 1/2 |o_hat - P^c|^2 against the cached unit outputs
+ * P^c ([B, N, r] with r = d), I = the k largest s (ties to the lowest index,
+ * ascending) into idx ([B, k] int32 device), P^c[I] <- o_hat[I].  Phase 3 runs
+ * on the selected rows: H1 = H[I] + O[I] W_o^T, H^c[I] <- H1 + FFN(RMSNorm(H1)).
+ * The layer must have r = d (its W_r is not used); start from
+ * spa_full_block(..., fill_proxy = 2).  Errors: SPA_ERR_INVALID,
+ * SPA_ERR_SHAPE (k outside [1, N], r != d), SPA_ERR_CUDA. */
+int spa_layer_step_attn_identifier(spa_layer *layer, const void *H, const spa_layer_cache *cache, int k,
+                                   int32_t *idx, void *stream);
 
 /* ---------------------------------------------------------- decode loop -- */
 typedef struct {

@@ -344,16 +344,19 @@ def attn_output_identify(layer: OracleLayer, H: np.ndarray, cache: LayerCache):
     return O, o_hat, 0.5 * np.sum(diff * diff, axis=1)
 
 
-def attn_output_layer_step(layer: OracleLayer, H: np.ndarray, cache: LayerCache, k: int) -> dict:
+def attn_output_layer_step(layer: OracleLayer, H: np.ndarray, cache: LayerCache, k: int,
+                           I: np.ndarray | None = None) -> dict:
     """Cached layer step with the attention-output identifier (reading A24):
     phase 1 scores every token by the drift of its attention output (which
     refreshes K^c, V^c at every row), selects the k most drifted (lowest index
     on ties, ascending) and writes P^c[I] ← ô[I]; phase 2 is the attention
     already computed; phase 3 runs the FFN on the selected rows and scatters
-    into H^c [NOTES 整体框架, Phase 3].  Cache updated in place."""
+    into H^c [NOTES 整体框架, Phase 3].  Cache updated in place.  A given I
+    (ascending, k entries) replaces the top-k, for parity runs where several
+    index sets are equally valid (reading A22)."""
     H = np.asarray(H, dtype=np.float64)
     O, o_hat, s = attn_output_identify(layer, H, cache)
-    I = select_topk(s, k)
+    I = select_topk(s, k) if I is None else np.asarray(I, dtype=np.int64)
     cache.P_c[I] = o_hat[I]
     H1, A = phase3_ffn_scatter(layer, H, I, O[I], cache)
     return {"I": I, "s": s, "O": O[I], "H1": H1, "A": A}

@@ -147,6 +147,20 @@ def test_bf16_wide_weight_tiles(monkeypatch, nacc, B, N, k):
     _step(lp, cache, ocs, H2, k)
 
 
+@pytest.mark.parametrize("grid", ["1", "5", "24"])
+@pytest.mark.parametrize("B,N,k", [(1, 200, 96), (2, 160, 33)])
+def test_bf16_stream_k_partitions(monkeypatch, grid, B, N, k):
+    # the stream-K weight-streaming GEMMs over 1, 5 and 24 CTAs: one CTA for
+    # everything, ranges that split tiles unevenly, and (QKV, gate/up: 24
+    # units) one k-block per CTA, so every tile is fixed up from 4 partials
+    monkeypatch.setenv("SPA_SK_GRID", grid)
+    lp = LayerPair(spa, SMALL_BF16, seed=80 + k, dtype=spa.SPA_BF16, max_B=2, max_N=200, std=0.05)
+    H = synth.hidden_states(B, N, 256, seed=k + 3, bf16=True)
+    cache, ocs = _run_fill(lp, H)
+    H2, _ = synth.drift_rows(H, 0.2, 0.5, seed=k + 4, bf16=True)
+    _step(lp, cache, ocs, H2, k)
+
+
 @pytest.mark.parametrize("B,N,k", [(1, 2048, 200), (2, 1000, 62), (1, 1536, 129), (1, 3000, 200)])
 def test_bf16_split_key_attention(B, N, k):
     # long caches: the keys of each query tile are split over a cluster of 8,
