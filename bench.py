@@ -252,24 +252,34 @@ def cpu_cores():
 
 # ------------------------------------------------------------------ traffic record
 
+def kernel_source_sha(files) -> str:
+    """Hash of the library source files a kernel is built from."""
+    src = os.path.join(ROOT, "adaptive_hidden_state_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(files):
+        with open(os.path.join(src, name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def traffic_record(cls: str):
     """Per-launch DRAM bytes of `cls` from the committed ncu summary, or None
-    when the kernel source changed since the counters were taken."""
+    when the kernel's source files changed since the counters were taken.
+    A record line: `traffic <class> bytes_per_launch=<n> source_sha=<sha>
+    files=<f1,f2,...>`, the hash taken over those files."""
     path = os.path.join(ROOT, "profiles", "traffic_llada_decode.md")
     if not os.path.exists(path):
         return None
-    src = os.path.join(ROOT, "adaptive_hidden_state_b200", "csrc")
-    h = hashlib.sha256()
-    for name in sorted(os.listdir(src)):
-        if name.endswith((".cu", ".cuh", ".h", ".cpp")):
-            with open(os.path.join(src, name), "rb") as fh:
-                h.update(fh.read())
-    sha = h.hexdigest()[:16]
     with open(path) as fh:
         for line in fh:
-            m = re.match(r"^traffic\s+(\w+)\s+bytes_per_launch=(\d+)\s+source_sha=(\w+)", line.strip())
+            m = re.match(r"^traffic\s+(\w+)\s+bytes_per_launch=(\d+)\s+source_sha=(\w+)\s+files=(\S+)",
+                         line.strip())
             if m and m.group(1) == cls:
-                return int(m.group(2)) if m.group(3) == sha else None
+                try:
+                    ok = kernel_source_sha(m.group(4).split(",")) == m.group(3)
+                except OSError:
+                    ok = False
+                return int(m.group(2)) if ok else None
     return None
 
 
@@ -408,6 +418,50 @@ def measure_single_layer(spa, torch, layer, ws, seed, hbm, tf):
                         "5% of rows drifted by N(0, 0.3) between steps",
             "us_per_layer": us, "roofline_us": roof["ms"] * 1e3 / 4, "roofline_frac": roof["ms"] * 1e3 / 4 / us,
             "bound": roof["bound"], "rho1_recompute_us": rho1, "speedup_over_rho1": rho1 / us}
+
+
+def measure_identifiers(spa, torch, w, w_r128, seed):
+    """The identifier comparison at the single-layer shape (N=512, rho=0.25,
+    k=128, 5% drifted rows): us per cached layer step with the singular Value
+    proxy (r=128), the full-d Value identifier (r=d), the Query and Key
+    identifiers (W_r = W_q or W_k, r=d) and the attention-output identifier
+    (every row's attention output, r=d); the step with the identifier minus
+    the plain FFN part is each identifier's cost."""
+    c = CFG
+    d, N, k = c["d"], 512, 128
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    H, H2 = drift_pair(torch, g, 1, N, d)
+    out = {}
+    for name, r, w_r in (("value_proxy_r128", 128, w_r128), ("value_full_d", d, None),
+                         ("query", d, w["wq"].float().cpu()), ("key", d, w["wk"].float().cpu()),
+                         ("attention_output", d, w["wv"].float().cpu())):
+        desc = spa.LayerDesc(d=d, n_heads=c["n_heads"], head_dim=c["head_dim"], ffn=c["ffn"], r=r,
+                             dtype=spa.SPA_BF16, rms_eps=1e-5, rope_theta=1e4)
+        ws = spa.Workspace(desc, 1, N)
+        if w_r is None:  # the full-d Value identifier: W_v itself scores each token like its value vector
+            w_r = w["wv"].float().cpu()
+        layer = spa.Layer(desc, w, ws, w_r_host=w_r)
+        cache = spa.Cache(1, N, d, r, spa.SPA_BF16)
+        idx = torch.empty((1, k), dtype=torch.int32, device="cuda")
+        attn = name == "attention_output"
+        spa.spa_full_block(layer, H, cache, 2 if attn else 1)
+        step = (lambda h: spa.spa_layer_step_attn_identifier(layer, h, cache, k, idx)) if attn else \
+               (lambda h: spa.spa_layer_step(layer, h, cache, k, idx))
+        for t in range(2):
+            step(H2 if t % 2 == 0 else H)
+        torch.cuda.synchronize()
+        e0, e1 = _ev(torch), _ev(torch)
+        e0.record()
+        for t in range(10):
+            step(H2 if t % 2 == 0 else H)
+        e1.record()
+        torch.cuda.synchronize()
+        out[name] = {"r": r, "us_per_layer_step": e0.elapsed_time(e1) * 1e3 / 10}
+        ws.check()
+        layer.close()
+        ws.close()
+    return {"workload": "single LLaDA-8B-shaped bf16 layer, B=1, N=512, rho=0.25 (k=128), 5% drifted rows; "
+                        "cached layer step with each update identifier", "identifiers": out}
 
 
 def measure_sweep(spa, torch, wbase, seed, ranks=(64, 128, 256, 512), rhos=(0.1, 0.25, 1.0),
@@ -799,6 +853,8 @@ def main():
         extra["batched_b8_n2048"] = measure_batched_decode(spa, torch, layers, weights, keep, args.seed + 12,
                                                            5, hbm, tf_sus)
         extra["sweep"] = measure_sweep(spa, torch, weights[0], args.seed + 13)
+        extra["identifiers"] = measure_identifiers(spa, torch, weights[c["l_p"] - 1],
+                                                   layers[c["l_p"] - 1].proxy_weights(), args.seed + 14)
         ws.check()
 
     # ---- CPU oracle on a bounded sample (rank 0, one GPU only)
