@@ -348,7 +348,7 @@ extern "C" int spa_workspace_create(const spa_layer_desc* desc, int max_B, int m
   WS_ALLOC(err, 2 * sizeof(int))
   if (desc->dtype == SPA_BF16) {
     ws->sk_count_len = (int)std::max<size_t>(3 * d / 128, std::max<size_t>(F / 64, d / 128));
-    WS_ALLOC(sk_part, (size_t)2 * ws->num_sms * 128 * 256 * 4)
+    WS_ALLOC(sk_part, (size_t)2 * ws->num_sms * 2 * 128 * 256 * 4)
     WS_ALLOC(sk_count, (size_t)ws->sk_count_len * sizeof(int))
   }
   WS_ALLOC(rope_cos, (size_t)max_N * (desc->head_dim / 2) * 4)
@@ -658,13 +658,22 @@ static int run_sk(int mode, SkParams& p, spa_workspace* ws, const void* X, int M
   const int NT = ((M + 31) / 32) * 32;
   if (encode_bf16_map_box(&p.tmX, X, (uint64_t)M, (uint64_t)K, (uint32_t)NT))
     return fail(SPA_ERR_CUDA, "tensor map for the token operand failed");
+  // two 128-row tiles per unit halve the token-tile traffic per weight byte
+  int nacc = tiles % 2 == 0 && NT <= 128 ? 2 : 1;
+  if (const char* env = std::getenv("SPA_SK_NACC")) {  // tuning override, 1 or 2
+    const int v = std::atoi(env);
+    if ((v == 1 || v == 2) && tiles % v == 0) nacc = v;
+  }
+  const int nbuf = 2 * nacc * NT <= 512 ? 2 : 1;
   int cols = 32;
-  while (cols < 2 * NT) cols *= 2;
+  while (cols < nbuf * nacc * NT) cols *= 2;
   p.K = K;
   p.KB = K / 64;
   p.NT = NT;
-  p.n_tiles = tiles;
-  p.units = tiles * p.KB;
+  p.nacc = nacc;
+  p.nbuf = nbuf;
+  p.n_tiles = tiles / nacc;
+  p.units = p.n_tiles * p.KB;
   p.tmem_cols = cols;
   p.part = ws->sk_part;
   p.count = ws->sk_count;

@@ -89,12 +89,14 @@ struct alignas(64) SkParams {
   CUtensorMap tmX;     // token rows [M, K], box 64 x NT, 128-byte swizzle
   int K, KB;           // reduction length and its 64-column blocks
   int NT;              // tokens per MMA (multiple of 32, <= 256)
-  int n_tiles;         // 128-row weight tiles
+  int n_tiles;         // units' weight tiles (nacc x 128 rows each)
   int units;           // n_tiles * KB
-  int tmem_cols;       // power of two >= 2 * NT (two accumulators)
+  int tmem_cols;       // power of two >= nbuf * nacc * NT
+  int nacc;            // 128-row weight tiles per unit (1 or 2), sharing the token box
+  int nbuf;            // TMEM accumulator buffers (2: a segment's epilogue overlaps the next)
   int b_mode;
   int b_rows_per_src;
-  float* part;         // [2 * grid, 128, NT] fp32 partial tiles of split tiles
+  float* part;         // [2 * grid, nacc, 128, NT] fp32 partial tiles of split tiles
   int* count;          // [n_tiles] segments counted (zero between launches)
   EpiParams ep;
 };
@@ -120,7 +122,7 @@ cudaError_t launch_tc_ws(int mode, int nacc, const TcWsParams& p, int n_tiles, i
 int plan_ws_splits(int mode, int nacc, int n_tiles, int KB);
 // Stream-K weight-streaming GEMM over `grid` CTAs (one per SM).
 cudaError_t launch_tc_sk(int mode, const SkParams& p, int grid, cudaStream_t stream);
-int sk_stages(int NT);
+int sk_stages(int nacc, int NT);
 // Encodes a 2D bf16 tensor map with a 64 x box_rows box.
 int encode_bf16_map_box(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                         uint32_t box_rows);

@@ -18,6 +18,9 @@
 //   warp 1      one thread issues tcgen05.mma (D[f, t] += W[f, k] X[t, k]) into
 //               one of two TMEM accumulators (segment j uses j % 2), so the
 //               epilogue of a segment overlaps the main loop of the next.
+// A unit may also hold NACC = 2 consecutive 128-row tiles that share the
+// token box of the stage (half the token-tile traffic per weight byte); then
+// two accumulators per buffer, and one buffer when 4 * NT > 512 TMEM columns.
 //   warps 2-3   stage every token's (sequence, cache row), then idle.
 //   warps 4-7   epilogue: thread (quadrant q, lane) owns feature row
 //               f = 32 q + lane of the tile (its TMEM lane).
@@ -208,8 +211,10 @@ __global__ void __launch_bounds__(kSkThreads, 1) tc_sk_kernel(const __grid_const
   const int KB = p.KB, U = p.units, NT = p.NT;
   const int u0 = sk_start(g, G, U), u1 = sk_start(g + 1, G, U);
   const int n_units = u1 - u0;
+  const int NACC = p.nacc, NBUF = p.nbuf;
+  const int W_BYTES = NACC * kSkW;
   const int X_BYTES = NT * 128;
-  const int STAGE_BYTES = kSkW + X_BYTES;  // multiple of 1024
+  const int STAGE_BYTES = W_BYTES + X_BYTES;  // multiple of 1024
   int STAGES = kSkRing / STAGE_BYTES;
   if (STAGES > kSkMaxStages) STAGES = kSkMaxStages;
   int* err = p.ep.err;
@@ -245,11 +250,12 @@ __global__ void __launch_bounds__(kSkThreads, 1) tc_sk_kernel(const __grid_const
       for (int it = 0; it < pre; ++it) {
         const int u = u0 + it;
         mbar_arrive_expect_tx(&full_bar[it], (uint32_t)STAGE_BYTES);
-        sk_load_w(p, u / KB, u % KB, smem + it * STAGE_BYTES, &full_bar[it]);
+        for (int a = 0; a < NACC; ++a)
+          sk_load_w(p, (u / KB) * NACC + a, u % KB, smem + it * STAGE_BYTES + a * kSkW, &full_bar[it]);
       }
       griddep_wait();  // the token rows come from earlier kernels
       for (int it = 0; it < pre; ++it)
-        tma_load_2d(smem + it * STAGE_BYTES + kSkW, &p.tmX, &full_bar[it], ((u0 + it) % KB) * 64, 0);
+        tma_load_2d(smem + it * STAGE_BYTES + W_BYTES, &p.tmX, &full_bar[it], ((u0 + it) % KB) * 64, 0);
       int it = pre;
       for (; it < n_units; ++it) {
         const int s = it % STAGES;
@@ -257,8 +263,8 @@ __global__ void __launch_bounds__(kSkThreads, 1) tc_sk_kernel(const __grid_const
         const int u = u0 + it;
         uint8_t* sw = smem + s * STAGE_BYTES;
         mbar_arrive_expect_tx(&full_bar[s], (uint32_t)STAGE_BYTES);
-        sk_load_w(p, u / KB, u % KB, sw, &full_bar[s]);
-        tma_load_2d(sw + kSkW, &p.tmX, &full_bar[s], (u % KB) * 64, 0);
+        for (int a = 0; a < NACC; ++a) sk_load_w(p, (u / KB) * NACC + a, u % KB, sw + a * kSkW, &full_bar[s]);
+        tma_load_2d(sw + W_BYTES, &p.tmX, &full_bar[s], (u % KB) * 64, 0);
       }
       prod_issued = it;
     }
@@ -270,19 +276,23 @@ __global__ void __launch_bounds__(kSkThreads, 1) tc_sk_kernel(const __grid_const
       for (int u = u0; ok && u < u1; ++j) {
         const int kb0 = u % KB;
         const int kb1 = kb0 + (u1 - u < KB - kb0 ? u1 - u : KB - kb0);
-        const int a = j & 1;
-        if (j >= 2 && !mbar_wait(&acc_empty[a], ((j >> 1) - 1) & 1, &abort_flag, err, 802)) break;
+        const int a = j % NBUF;
+        if (j >= NBUF && !mbar_wait(&acc_empty[a], ((j / NBUF) - 1) & 1, &abort_flag, err, 802)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem + (uint32_t)(a * NT);
+        const uint32_t d_tmem = tmem + (uint32_t)(a * NACC * NT);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           if (!mbar_wait(&full_bar[s], (it / STAGES) & 1, &abort_flag, err, 803)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
-          const uint64_t dw = smem_desc_sw128(sa), dx = smem_desc_sw128(sa + kSkW);
+          const uint64_t dx = smem_desc_sw128(sa + W_BYTES);
+          for (int sub = 0; sub < NACC; ++sub) {
+            const uint64_t dw = smem_desc_sw128(sa + sub * kSkW);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16(d_tmem, dw + 2 * kk, dx + 2 * kk, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16(d_tmem + (uint32_t)(sub * NT), dw + 2 * kk, dx + 2 * kk, idesc,
+                        (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
           umma_commit(&empty_bar[s]);
         }
         if (!ok) break;
@@ -313,8 +323,8 @@ __global__ void __launch_bounds__(kSkThreads, 1) tc_sk_kernel(const __grid_const
       const int t = u / KB, kb0 = u % KB;
       const int kb1 = kb0 + (u1 - u < KB - kb0 ? u1 - u : KB - kb0);
       u += kb1 - kb0;
-      const int a = j & 1;
-      const bool got = mbar_wait(&acc_full[a], (j >> 1) & 1, &abort_flag, err, 804);
+      const int a = j % NBUF;
+      const bool got = mbar_wait(&acc_full[a], (j / NBUF) & 1, &abort_flag, err, 804);
       __syncwarp();
       // the four epilogue warps agree on whether to go on, so every named
       // barrier below is reached by all 128 threads or by none
@@ -323,7 +333,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) tc_sk_kernel(const __grid_const
       named_bar_sync(2, 128);
       if (!s_ok) break;
       tc_fence_after();
-      const uint32_t acc_tmem = lane_base + (uint32_t)(a * NT);
+      const uint32_t buf_tmem = lane_base + (uint32_t)(a * NACC * NT);
       // the tile's segments: CTAs g_first..g_last, own index own_s
       const int g_first = sk_owner(t * KB, G, U), g_last = sk_owner(t * KB + KB - 1, G, U);
       const int nseg = g_last - g_first + 1, own_s = g - g_first;
@@ -338,13 +348,16 @@ __global__ void __launch_bounds__(kSkThreads, 1) tc_sk_kernel(const __grid_const
         finisher = s_flag != 0;
         named_bar_sync(2, 128);
         if (!finisher) {
-          float* dst = p.part + ((size_t)sk_slot(g, t, G, U, KB) * 128 + f) * NT;
-          for (int c0 = 0; c0 < NT; c0 += 32) {
-            float v[32];
-            tmem_ld32(acc_tmem + (uint32_t)c0, v);
+          for (int sub = 0; sub < NACC; ++sub) {
+            float* dst = p.part + (((size_t)sk_slot(g, t, G, U, KB) * NACC + sub) * 128 + f) * NT;
+            const uint32_t acc_tmem = buf_tmem + (uint32_t)(sub * NT);
+            for (int c0 = 0; c0 < NT; c0 += 32) {
+              float v[32];
+              tmem_ld32(acc_tmem + (uint32_t)c0, v);
 #pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              __stcg(reinterpret_cast<float4*>(dst + c0 + i), make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+              for (int i = 0; i < 32; i += 4)
+                __stcg(reinterpret_cast<float4*>(dst + c0 + i), make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+            }
           }
           __threadfence();
           named_bar_sync(2, 128);
@@ -356,7 +369,10 @@ __global__ void __launch_bounds__(kSkThreads, 1) tc_sk_kernel(const __grid_const
       }
       if (finisher) {
         __threadfence();
+        for (int sub = 0; sub < NACC; ++sub)
         for (int c0 = 0; c0 < NT && c0 < M; c0 += 32) {
+          const uint32_t acc_tmem = buf_tmem + (uint32_t)(sub * NT);
+          const int vt = t * NACC + sub;  // 128-row tile of the weights
           float acc[32];
           tmem_ld32(acc_tmem + (uint32_t)c0, acc);  // own partial
           if (nseg > 1) {
@@ -368,7 +384,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) tc_sk_kernel(const __grid_const
                 for (int i = 0; i < 32; ++i) x[i] = acc[i];
               } else {
                 const float4* src = reinterpret_cast<const float4*>(
-                    p.part + ((size_t)sk_slot(g_first + s, t, G, U, KB) * 128 + f) * NT + c0);
+                    p.part + (((size_t)sk_slot(g_first + s, t, G, U, KB) * NACC + sub) * 128 + f) * NT + c0);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                   const float4 w = __ldcg(src + i);
@@ -397,7 +413,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) tc_sk_kernel(const __grid_const
             for (int i = 0; i < 32; ++i) partner[i] = theirs[i * kSkXLd + pl];
             named_bar_sync(3, 128);
           }
-          sk_store_chunk<MODE>(p, t, f, c0, acc, partner, s_rows);
+          sk_store_chunk<MODE>(p, vt, f, c0, acc, partner, s_rows);
         }
         if (nseg > 1 && et == 0) p.count[t] = 0;  // every segment has counted: ready for the next launch
       }
@@ -448,8 +464,8 @@ cudaError_t launch_tc_sk(int mode, const SkParams& p, int grid, cudaStream_t str
   return cudaLaunchKernelExC(&cfg, kern, args);
 }
 
-int sk_stages(int NT) {
-  const int st = kSkRing / (kSkW + NT * 128);
+int sk_stages(int nacc, int NT) {
+  const int st = kSkRing / (nacc * kSkW + NT * 128);
   return st < kSkMaxStages ? st : kSkMaxStages;
 }
 
