@@ -555,8 +555,8 @@ def measure_batched_decode(spa, torch, layers, weights, keep, seed, steps, hbm, 
         spa.spa_decode_step(model, pos[t], None, u, 0, out)
     prof = ws.profile_read()
     ws.profile_enable(False)
-    roof = roofline_of(prof, hbm, tf)
     n_prof = total - (1 + warm + steps)
+    roof = roofline_of(prof, hbm, tf)  # over the n_prof profiled steps
     gemm = [k for k in ("qkv", "oproj", "gateup", "down") if prof[k][0]]
     g_ms = sum(prof[k][1] for k in gemm)
     g_fl = sum(prof[k][3] for k in gemm)
@@ -572,7 +572,7 @@ def measure_batched_decode(spa, torch, layers, weights, keep, seed, steps, hbm, 
     res = {"workload": "LLaDA-8B-shaped 32-layer bf16 decode, B=8 x N=2048 (512 prompt + 1536 masked), "
                        "r=128, piecewise-Gaussian rho(l), 4 tokens unmasked per sequence per step",
            "tokens_per_s": B * u / (ms / 1e3), "ms_per_step": ms, "steps": steps,
-           "step_roofline_ms": roof["ms"] * 1.0, "step_roofline_frac": roof["ms"] / ms,
+           "step_roofline_ms": roof["ms"] / n_prof, "step_roofline_frac": roof["ms"] / n_prof / ms,
            "step_bound": roof["bound"], "budget_k": model.k,
            "layer_gemm_tflops": (g_fl / (g_ms / 1e3) / 1e12) if g_ms else None,
            "layer_gemm_tensor_frac_of_sustained": ((g_fl / (g_ms / 1e3) / 1e12) / tf) if g_ms else None,
