@@ -193,9 +193,8 @@ struct spa_workspace {
   int* attn_sync = nullptr;  // per query tile: attention key splits finished
   int attn_sync_len = 0;
   int* err = nullptr;       // [2]
-  float* sk_part = nullptr;  // stream-K GEMM: partial tiles [2 * num_sms, 128, 256] fp32
-  int* sk_count = nullptr;   // stream-K GEMM: per tile, segments counted
-  int sk_count_len = 0;
+  float* sk_part = nullptr;  // stream-K GEMM: the segments' partial tiles (fp32)
+  size_t sk_part_floats = 0;
   float* rope_cos = nullptr;  // [max_N, hd/2]
   float* rope_sin = nullptr;
   CUtensorMap tmX, tmO, tmX2, tmA;
@@ -301,6 +300,68 @@ static int ws_alloc(spa_workspace* ws, void** p, size_t bytes) {
   return SPA_OK;
 }
 
+// Stream-K plan of one weight-streaming GEMM: `tiles128` tiles of 128 weight
+// rows, K / 64 k-blocks, NT tokens per MMA, on `sms` SMs.
+struct SkPlan {
+  int nacc, nbuf, n_tiles, KB, grid, maxseg;
+};
+
+static SkPlan sk_plan(int tiles128, int K, int NT, int sms, bool overrides) {
+  SkPlan pl;
+  // two 128-row tiles per unit halve the token-box traffic and the stages per
+  // weight byte; GEMMs with few tiles keep one (their tiles split over more
+  // CTAs, and two per unit would double the partials to sum)
+  pl.nacc = (tiles128 % 2 == 0 && tiles128 >= 64) ? 2 : 1;
+  if (overrides)
+    if (const char* env = std::getenv("SPA_SK_NACC")) {  // tuning override, 1 or 2
+      const int v = std::atoi(env);
+      if ((v == 1 || v == 2) && tiles128 % v == 0) pl.nacc = v;
+    }
+  pl.nbuf = 2 * pl.nacc * NT <= 512 ? 2 : 1;
+  pl.n_tiles = tiles128 / pl.nacc;
+  pl.KB = K / 64;
+  const int units = pl.n_tiles * pl.KB;
+  // one CTA per SM, at least four k-blocks each
+  pl.grid = std::max(1, std::min(sms, units / 4));
+  if (overrides)
+    if (const char* env = std::getenv("SPA_SK_GRID")) {  // tuning / test override, 1..SMs and <= units
+      const int v = std::atoi(env);
+      if (v >= 1 && v <= sms && v <= units) pl.grid = v;
+    }
+  // the reduce kernel takes at most sk_reduce_max_seg() segments per tile
+  int mc = 0, mt = 0;
+  for (;;) {
+    sk_partition_bounds(pl.n_tiles, pl.KB, pl.grid, &mc, &mt);
+    if (mt <= sk_reduce_max_seg() || pl.grid == 1) break;
+    --pl.grid;
+  }
+  pl.maxseg = mc;
+  return pl;
+}
+
+// Scratch floats the stream-K GEMMs of a layer of width d and FFN width F need
+// at the widest token count (256) with either tile width.
+static size_t sk_scratch_floats(int sms, int d, int F) {
+  const int gemm[4][2] = {{3 * d / 128, d}, {d / 128, d}, {F / 64, d}, {d / 128, F}};
+  size_t need = 0;
+  for (const auto& gk : gemm)
+    for (int nacc = 1; nacc <= 2; ++nacc) {
+      if (gk[0] % nacc) continue;
+      for (int NT = 32; NT <= 256; NT += 32) {
+        SkPlan pl = sk_plan(gk[0], gk[1], NT, sms, false);
+        pl.nacc = nacc;  // both widths, whatever the default
+        pl.n_tiles = gk[0] / nacc;
+        const int units = pl.n_tiles * pl.KB;
+        for (int grid = 1; grid <= std::min(sms, units); ++grid) {
+          int mc = 0, mt = 0;
+          sk_partition_bounds(pl.n_tiles, pl.KB, grid, &mc, &mt);
+          need = std::max(need, (size_t)grid * mc * NT * nacc * 128);
+        }
+      }
+    }
+  return need;
+}
+
 extern "C" void spa_workspace_free(spa_workspace* ws) {
   if (!ws) return;
   for (void* p : ws->allocs) cudaFree(p);
@@ -347,9 +408,8 @@ extern "C" int spa_workspace_create(const spa_layer_desc* desc, int max_B, int m
   WS_ALLOC(attn_sync, (size_t)ws->attn_sync_len * sizeof(int))
   WS_ALLOC(err, 2 * sizeof(int))
   if (desc->dtype == SPA_BF16) {
-    ws->sk_count_len = (int)std::max<size_t>(3 * d / 128, std::max<size_t>(F / 64, d / 128));
-    WS_ALLOC(sk_part, (size_t)2 * ws->num_sms * 2 * 128 * 256 * 4)
-    WS_ALLOC(sk_count, (size_t)ws->sk_count_len * sizeof(int))
+    ws->sk_part_floats = sk_scratch_floats(ws->num_sms, (int)d, (int)F);
+    WS_ALLOC(sk_part, ws->sk_part_floats * 4)
   }
   WS_ALLOC(rope_cos, (size_t)max_N * (desc->head_dim / 2) * 4)
   WS_ALLOC(rope_sin, (size_t)max_N * (desc->head_dim / 2) * 4)
@@ -371,8 +431,7 @@ extern "C" int spa_workspace_create(const spa_layer_desc* desc, int max_B, int m
   if (cudaMemcpy(ws->rope_cos, cs.data(), cs.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
       cudaMemcpy(ws->rope_sin, sn.data(), sn.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
       cudaMemset(ws->err, 0, 2 * sizeof(int)) != cudaSuccess ||
-      cudaMemset(ws->attn_sync, 0, (size_t)ws->attn_sync_len * sizeof(int)) != cudaSuccess ||
-      (ws->sk_count && cudaMemset(ws->sk_count, 0, (size_t)ws->sk_count_len * sizeof(int)) != cudaSuccess)) {
+      cudaMemset(ws->attn_sync, 0, (size_t)ws->attn_sync_len * sizeof(int)) != cudaSuccess) {
     spa_workspace_free(ws);
     return fail(SPA_ERR_CUDA, "workspace initialisation copy failed");
   }
@@ -396,7 +455,6 @@ extern "C" int spa_workspace_status(spa_workspace* ws, void* stream) {
   SPA_CK(cudaMemset(ws->err, 0, sizeof(h)));
   // a kernel that gave up may have left split counters behind: start them afresh
   SPA_CK(cudaMemset(ws->attn_sync, 0, (size_t)ws->attn_sync_len * sizeof(int)));
-  if (ws->sk_count) SPA_CK(cudaMemset(ws->sk_count, 0, (size_t)ws->sk_count_len * sizeof(int)));
   if (h[0] & DEVERR_TIMEOUT) return fail(SPA_ERR_TIMEOUT, "device wait timed out (site %d)", h[1]);
   return fail(SPA_ERR_DEVICE, "device check failed: bits 0x%x site %d", h[0], h[1]);
 }
@@ -651,41 +709,49 @@ static bool streamk_enabled() {
   return on;
 }
 
-static int run_sk(int mode, SkParams& p, spa_workspace* ws, const void* X, int M, int K, int tiles,
-                  cudaStream_t s, Profiler* prof, Work w) {
+static int run_sk(int mode, SkParams& p, spa_workspace* ws, const void* X, int M, int K, int tiles128,
+                  cudaStream_t s, Profiler* prof, Work w, const void* gamma = nullptr, void* x2 = nullptr,
+                  float eps = 0.f) {
   if (M <= 0) return SPA_OK;
   if (M > 256) return fail(SPA_ERR_SHAPE, "stream-K GEMM takes at most 256 tokens");
   const int NT = ((M + 31) / 32) * 32;
   if (encode_bf16_map_box(&p.tmX, X, (uint64_t)M, (uint64_t)K, (uint32_t)NT))
     return fail(SPA_ERR_CUDA, "tensor map for the token operand failed");
-  // two 128-row tiles per unit halve the token-tile traffic per weight byte
-  int nacc = tiles % 2 == 0 && NT <= 128 ? 2 : 1;
-  if (const char* env = std::getenv("SPA_SK_NACC")) {  // tuning override, 1 or 2
-    const int v = std::atoi(env);
-    if ((v == 1 || v == 2) && tiles % v == 0) nacc = v;
-  }
-  const int nbuf = 2 * nacc * NT <= 512 ? 2 : 1;
+  const SkPlan pl = sk_plan(tiles128, K, NT, ws->num_sms, true);
+  if (pl.n_tiles > sk_reduce_max_tiles()) return fail(SPA_ERR_SHAPE, "stream-K GEMM: too many weight tiles");
+  const size_t slot_floats = (size_t)NT * pl.nacc * 128;
+  if ((size_t)pl.grid * pl.maxseg * slot_floats > ws->sk_part_floats)
+    return fail(SPA_ERR_SHAPE, "stream-K GEMM: scratch too small for the partition");
   int cols = 32;
-  while (cols < nbuf * nacc * NT) cols *= 2;
+  while (cols < pl.nbuf * pl.nacc * NT) cols *= 2;
   p.K = K;
-  p.KB = K / 64;
+  p.KB = pl.KB;
   p.NT = NT;
-  p.nacc = nacc;
-  p.nbuf = nbuf;
-  p.n_tiles = tiles / nacc;
-  p.units = p.n_tiles * p.KB;
+  p.nacc = pl.nacc;
+  p.nbuf = pl.nbuf;
+  p.n_tiles = pl.n_tiles;
+  p.units = pl.n_tiles * pl.KB;
   p.tmem_cols = cols;
+  p.maxseg = pl.maxseg;
   p.part = ws->sk_part;
-  p.count = ws->sk_count;
-  if (tiles > ws->sk_count_len) return fail(SPA_ERR_SHAPE, "stream-K GEMM: more tiles than counters");
-  // one CTA per SM, at least four k-blocks each
-  int grid = std::max(1, std::min(ws->num_sms, p.units / 4));
-  if (const char* env = std::getenv("SPA_SK_GRID")) {  // tuning / test override, 1..SMs and <= units
-    const int v = std::atoi(env);
-    if (v >= 1 && v <= ws->num_sms && v <= p.units) grid = v;
-  }
+  SkReduceParams r;
+  std::memset(&r, 0, sizeof(r));
+  r.part = ws->sk_part;
+  r.slot_floats = slot_floats;
+  r.feat = pl.nacc * 128;
+  r.nacc = pl.nacc;
+  r.n_tiles = pl.n_tiles;
+  r.KB = pl.KB;
+  r.G = pl.grid;
+  r.U = p.units;
+  r.maxseg = pl.maxseg;
+  r.gamma = gamma;
+  r.x2 = x2;
+  r.eps = eps;
+  r.ep = p.ep;
   ProfScope ps(prof, w.cls, w.bytes, w.flops, s);
-  cudaError_t e = launch_tc_sk(mode, p, grid, s);
+  g_launches += 1;  // the reduce kernel (the scope counts the GEMM)
+  cudaError_t e = launch_tc_sk(mode, p, pl.grid, r, s);
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "stream-K GEMM launch (mode %d): %s", mode, cudaGetErrorString(e));
   return SPA_OK;
 }
@@ -868,8 +934,10 @@ static int run_ffn_half(spa_layer* L, const void* H, const int32_t* idx, int tps
       SkParams p;
       std::memset(&p, 0, sizeof(p));
       p.tmW[0] = L->tm_wo; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
+      // the reduce kernel also takes the FFN RMSNorm of each row: x2 = RMSNorm(H1)
       SPA_TRY(run_sk(EPI_RESID, p, ws, Ob, M, d, d / 128, s, prof,
-                     Work{SPA_PROF_OPROJ, (double)d * d * es + 3.0 * Md * es, 2.0 * Md * d}));
+                     Work{SPA_PROF_OPROJ, (double)d * d * es + 4.0 * Md * es + d * es, 2.0 * Md * d + 4.0 * Md},
+                     L->w.ffn_norm, ws->X2, D.rms_eps));
     } else if (bf && M <= 256) {
       TcWsParams p;
       std::memset(&p, 0, sizeof(p));
@@ -893,12 +961,14 @@ static int run_ffn_half(spa_layer* L, const void* H, const int32_t* idx, int tps
                        Work{SPA_PROF_OPROJ, (double)d * d * es + 3.0 * Md * es, 2.0 * Md * d}));
     }
   }
-  // x2 = RMSNorm(H1)
-  {
-    ProfScope ps(prof, SPA_PROF_NORM, 2.0 * Md * es + d * es, 4.0 * Md, s);
-    e = launch_rmsnorm_rows(D.dtype, ws->H1, 0, nullptr, tps, N, M, d, L->w.ffn_norm, D.rms_eps, ws->X2, ws->err, s);
+  // x2 = RMSNorm(H1) (the stream-K O-proj's reduce kernel wrote it already)
+  if (!(bf && M <= 256 && streamk_enabled())) {
+    {
+      ProfScope ps(prof, SPA_PROF_NORM, 2.0 * Md * es + d * es, 4.0 * Md, s);
+      e = launch_rmsnorm_rows(D.dtype, ws->H1, 0, nullptr, tps, N, M, d, L->w.ffn_norm, D.rms_eps, ws->X2, ws->err, s);
+    }
+    if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "rmsnorm launch: %s", cudaGetErrorString(e));
   }
-  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "rmsnorm launch: %s", cudaGetErrorString(e));
   // A = silu(x2 W_gate^T) * (x2 W_up^T)
   {
     EpiParams ep = base_epi(L, M, tps, N, idx);

@@ -81,23 +81,36 @@ struct alignas(64) TcWsParams {
   EpiParams ep;
 };
 
-// Stream-K weight-streaming GEMM (spa_streamk.cu): tiles of 128 output
-// features (gate/up: 64 gate + the same 64 up rows), units (tile, 64-column
-// k-block) split evenly over the grid's CTAs.
+// Stream-K weight-streaming GEMM (spa_streamk.cu): units (tile of nacc x 128
+// output features, 64-column k-block) split evenly over the grid's CTAs; each
+// CTA writes every segment's fp32 partial tile to its scratch slots, and a
+// reduce kernel sums them per token row in k-block order and applies the
+// fused epilogue.
 struct alignas(64) SkParams {
   CUtensorMap tmW[3];  // weight sources, box 64 x 128 rows (B_GATEUP: 64 rows)
   CUtensorMap tmX;     // token rows [M, K], box 64 x NT, 128-byte swizzle
   int K, KB;           // reduction length and its 64-column blocks
   int NT;              // tokens per MMA (multiple of 32, <= 256)
-  int n_tiles;         // units' weight tiles (nacc x 128 rows each)
+  int n_tiles;         // unit tiles (nacc x 128 weight rows each)
   int units;           // n_tiles * KB
   int tmem_cols;       // power of two >= nbuf * nacc * NT
   int nacc;            // 128-row weight tiles per unit (1 or 2), sharing the token box
   int nbuf;            // TMEM accumulator buffers (2: a segment's epilogue overlaps the next)
+  int maxseg;          // scratch slots per CTA (its most segments)
   int b_mode;
   int b_rows_per_src;
-  float* part;         // [2 * grid, nacc, 128, NT] fp32 partial tiles of split tiles
-  int* count;          // [n_tiles] segments counted (zero between launches)
+  float* part;         // scratch: slot (g * maxseg + j) = [NT][nacc * 128] fp32
+  EpiParams ep;
+};
+
+struct SkReduceParams {
+  const float* part;   // the GEMM's scratch slots
+  size_t slot_floats;  // NT * feat
+  int feat;            // nacc * 128
+  int nacc, n_tiles, KB, G, U, maxseg;
+  const void* gamma;   // EPI_RESID: FFN RMSNorm gain [d] and output x2 [M, d] (null: no norm)
+  void* x2;
+  float eps;
   EpiParams ep;
 };
 
@@ -120,9 +133,14 @@ cudaError_t launch_tc_gemm(int mode, int BN, const TcGemmParams& p, int m_tiles,
 cudaError_t launch_tc_ws(int mode, int nacc, const TcWsParams& p, int n_tiles, int splits,
                          cudaStream_t stream);
 int plan_ws_splits(int mode, int nacc, int n_tiles, int KB);
-// Stream-K weight-streaming GEMM over `grid` CTAs (one per SM).
-cudaError_t launch_tc_sk(int mode, const SkParams& p, int grid, cudaStream_t stream);
+// Stream-K weight-streaming GEMM over `grid` CTAs (one per SM), then its
+// per-row reduce + epilogue kernel (M CTAs).
+cudaError_t launch_tc_sk(int mode, const SkParams& p, int grid, const SkReduceParams& r, cudaStream_t stream);
 int sk_stages(int nacc, int NT);
+// Segments of the busiest CTA and of the most split tile of a partition.
+void sk_partition_bounds(int n_tiles, int KB, int G, int* max_seg_per_cta, int* max_seg_per_tile);
+int sk_reduce_max_seg();    // segments per tile the reduce kernel takes
+int sk_reduce_max_tiles();  // unit tiles the reduce kernel takes
 // Encodes a 2D bf16 tensor map with a 64 x box_rows box.
 int encode_bf16_map_box(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                         uint32_t box_rows);

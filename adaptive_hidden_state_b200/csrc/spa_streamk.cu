@@ -3,47 +3,47 @@
 // The four GEMMs of a cached layer step (QKV, O-proj, gate/up, down) multiply
 // a large weight matrix by the few selected tokens (M <= 256): they are bound
 // by streaming the weights from HBM, so every SM has to stream its share of
-// them all the time.  The weights are cut into tiles of 128 output features
-// (the 128 TMEM lanes of one tcgen05.mma, M = 128) and k-blocks of 64 input
-// columns; the tile-major list of (tile, k-block) units is split evenly over
-// one CTA per SM (stream-K), so no SM idles whatever the tile count is.
+// them all the time.  The weights are cut into tiles of NACC x 128 output
+// features (the 128 TMEM lanes of one tcgen05.mma, M = 128, times NACC
+// accumulators sharing one token box) and k-blocks of 64 input columns; the
+// tile-major list of (tile, k-block) units is split evenly over one CTA per
+// SM (stream-K), so no SM idles whatever the tile count is.
 //
-// A CTA's range is a run of segments: the tail of one tile, whole tiles, the
-// head of another.  Roles (8 warps):
-//   warp 0      TMA producer: for every unit the weight box (128 x 64) and the
-//               token box (NT x 64) into a ring of stages, running straight
-//               across segment boundaries.  The weight boxes of the first
-//               stages are requested before griddepcontrol.wait (weights do
-//               not depend on earlier kernels).
+// tc_sk_kernel.  A CTA's range is a run of segments (the tail of one tile,
+// maybe whole tiles, the head of another).  Roles (8 warps):
+//   warp 0      TMA producer: for every unit the NACC weight boxes (128 x 64
+//               each) and the token box (NT x 64) into a ring of stages,
+//               straight across segment boundaries.  The weight boxes of the
+//               first stages are requested before griddepcontrol.wait
+//               (weights do not depend on earlier kernels).
 //   warp 1      one thread issues tcgen05.mma (D[f, t] += W[f, k] X[t, k]) into
-//               one of two TMEM accumulators (segment j uses j % 2), so the
-//               epilogue of a segment overlaps the main loop of the next.
-// A unit may also hold NACC = 2 consecutive 128-row tiles that share the
-// token box of the stage (half the token-tile traffic per weight byte); then
-// two accumulators per buffer, and one buffer when 4 * NT > 512 TMEM columns.
-//   warps 2-3   stage every token's (sequence, cache row), then idle.
-//   warps 4-7   epilogue: thread (quadrant q, lane) owns feature row
-//               f = 32 q + lane of the tile (its TMEM lane).
-// A tile split over several CTAs is fixed up without any CTA waiting for
-// another: each segment's CTA writes its fp32 partial tile [128][NT] to a
-// scratch slot and counts it in the tile's counter; the CTA that brings the
-// counter to the number of segments (or finds all other segments counted
-// before writing its own) sums every segment's partial in k-block order
-// (own partial straight from TMEM) and runs the fused epilogue, then resets
-// the counter.  The summation order is fixed by the partition, which depends
-// only on the weight shape and the SM count, so results are deterministic and
-// every output row depends only on its own token.
+//               the accumulators of buffer j % NBUF for segment j; with two
+//               buffers the epilogue of a segment overlaps the next main loop.
+//   warps 4-7   epilogue: thread (quadrant q, lane) reads TMEM lane f = 32 q +
+//               lane (feature f of the tile) and stores the segment's fp32
+//               partial sums into its own scratch slot, token-major
+//               [NT][NACC x 128], so a warp writes 128 contiguous bytes per
+//               token.
+// No CTA waits for another and none sums other CTAs' partials.
 //
-// Fused epilogues (from registers, one bf16 per thread and token; a warp
-// writes 32 consecutive features = 64 bytes of a row):
-//   EPI_QKV            RoPE on Q and K (the pair partner of feature f is
-//                      f ^ (head_dim / 2), exchanged through shared memory),
-//                      Q to the compact buffer, K and V into K^c, V^c rows I
-//   EPI_RESID          H1[t] = acc + H[b, I[t]]
+// sk_reduce_kernel<MODE>: one CTA per token row sums, for every feature, the
+// partials of the tile's segments in k-block order (the order is fixed by the
+// partition, which depends only on the weight shape and the grid: results are
+// deterministic, and each row depends only on its own token), then applies the
+// fused epilogue of the step:
+//   EPI_QKV            RoPE on Q and K (pairs f, f + head_dim/2 of a head), Q
+//                      to the compact buffer, K and V into K^c, V^c rows I
+//   EPI_RESID          H1[t] = acc + H[b, I[t]]; with x2 given also the FFN
+//                      RMSNorm of the row, x2 = RMSNorm(H1) (no separate norm
+//                      kernel)
 //   EPI_SWIGLU         tile = 64 gate rows (lanes 0-63) + the same 64 up rows
 //                      (lanes 64-127); A[t, f] = silu(gate) * up
 //   EPI_RESID_SCATTER  H^c[b, I[t]] = acc + H1[t] (+ compact copy, score zero)
 //   EPI_STORE          out[t, n] = acc
+// The reduce kernel is launched with programmatic dependent launch right
+// behind the GEMM; its CTAs are small enough to sit beside the GEMM's, and the
+// next GEMM's CTAs start prefetching their weights as soon as the GEMM's exit.
+#include <algorithm>
 #include <cstdio>
 
 #include "spa_device.cuh"
@@ -52,11 +52,13 @@
 namespace spa {
 
 constexpr int kSkThreads = 256;
-constexpr int kSkRing = 196 * 1024;     // bytes of the TMA ring
+constexpr int kSkRing = 200 * 1024;      // bytes of the TMA ring (leaves room for a reduce CTA beside it)
 constexpr int kSkMaxStages = 16;
 constexpr int kSkSmem = kSkRing + 1024;  // + alignment slack
-constexpr int kSkW = 128 * 128;          // one weight stage: 128 rows x 64 columns bf16
-constexpr int kSkXLd = 33;               // exchange tile row stride (floats)
+constexpr int kSkW = 128 * 128;          // one weight box: 128 rows x 64 columns bf16
+constexpr int kRedThreads = 128;
+constexpr int kRedMaxSeg = 16;    // segments per tile (the host keeps the grid within it)
+constexpr int kRedMaxTiles = 256;
 
 __device__ __forceinline__ float sk_silu(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
 
@@ -65,134 +67,27 @@ __host__ __device__ __forceinline__ int sk_start(int g, int G, int U) {
   return (int)(((long long)g * U) / G);
 }
 // The CTA whose range holds unit u.
-__device__ __forceinline__ int sk_owner(int u, int G, int U) {
+__host__ __device__ __forceinline__ int sk_owner(int u, int G, int U) {
   int g = (int)(((long long)u * G) / U);
   while (g + 1 < G && sk_start(g + 1, G, U) <= u) ++g;
   while (g > 0 && sk_start(g, G, U) > u) --g;
   return g;
 }
-// Scratch slot of CTA g's partial of tile t: slot 2g for the CTA's first
-// segment, 2g + 1 for its last (a CTA has at most two partial segments).
-__device__ __forceinline__ int sk_slot(int g, int t, int G, int U, int KB) {
-  return 2 * g + (sk_start(g, G, U) / KB == t ? 0 : 1);
-}
 
-// The weight boxes of unit (tile t, k-block kb) into sw (one 128-row stage).
-__device__ __forceinline__ void sk_load_w(const SkParams& p, int t, int kb, uint8_t* sw, uint64_t* bar) {
+// The weight box of 128-row tile vt, k-block kb into sw.
+__device__ __forceinline__ void sk_load_w(const SkParams& p, int vt, int kb, uint8_t* sw, uint64_t* bar) {
   const int kx = kb * 64;
   if (p.b_mode == B_GATEUP) {  // 64 gate rows, then the same 64 up rows
-    tma_load_2d(sw, &p.tmW[0], bar, kx, t * 64);
-    tma_load_2d(sw + kSkW / 2, &p.tmW[1], bar, kx, t * 64);
+    tma_load_2d(sw, &p.tmW[0], bar, kx, vt * 64);
+    tma_load_2d(sw + kSkW / 2, &p.tmW[1], bar, kx, vt * 64);
   } else if (p.b_mode == B_CONCAT3) {
-    const int g = t * 128;
+    const int g = vt * 128;
     tma_load_2d(sw, &p.tmW[g / p.b_rows_per_src], bar, kx, g % p.b_rows_per_src);
   } else {
-    tma_load_2d(sw, &p.tmW[0], bar, kx, t * 128);
+    tma_load_2d(sw, &p.tmW[0], bar, kx, vt * 128);
   }
 }
 
-// s_rows[t] = (sequence, cache row) of token t for every t < NT: (0, -1) past
-// the last token or for an index outside [0, N) (reported).
-__device__ void stage_rows_sk(const EpiParams& ep, int2* s_rows, int tid, int nthr) {
-  for (int t = tid; t < 256; t += nthr) {
-    int2 v = make_int2(0, -1);
-    if (t < ep.M) {
-      v.x = t / ep.tokens_per_seq;
-      v.y = ep.idx ? ep.idx[t] : (t % ep.tokens_per_seq);
-      if (v.y < 0 || v.y >= ep.N) {
-        report_error(ep.err, DEVERR_INDEX, 807);
-        v.y = -1;
-      }
-    }
-    s_rows[t] = v;
-  }
-}
-
-template <int MODE>
-__device__ __forceinline__ void sk_store_chunk(const SkParams& p, int t, int f, int c0, const float* acc,
-                                               const float* partner, const int2* s_rows) {
-  const EpiParams& ep = p.ep;
-  const int M = ep.M;
-  __nv_bfloat16* const outb = reinterpret_cast<__nv_bfloat16*>(ep.out);
-  if constexpr (MODE == EPI_STORE) {
-    const int n = t * 128 + f;
-    if (n >= ep.n_out) return;
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (c0 + j < M) outb[(size_t)(c0 + j) * ep.n_out + n] = __float2bfloat16_rn(acc[j]);
-  } else if constexpr (MODE == EPI_RESID) {
-    const int n = t * 128 + f;
-    if (n >= ep.n_out) return;
-    const __nv_bfloat16* res = reinterpret_cast<const __nv_bfloat16*>(ep.resid);
-    float h[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int2 br = s_rows[c0 + j];
-      h[j] = (c0 + j < M && br.y >= 0) ? __bfloat162float(res[((size_t)br.x * ep.N + br.y) * ep.d + n]) : 0.f;
-    }
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (c0 + j < M && s_rows[c0 + j].y >= 0)
-        outb[(size_t)(c0 + j) * ep.d + n] = __float2bfloat16_rn(acc[j] + h[j]);
-  } else if constexpr (MODE == EPI_RESID_SCATTER) {
-    const int n = t * 128 + f;
-    if (n >= ep.n_out) return;
-    const __nv_bfloat16* res = reinterpret_cast<const __nv_bfloat16*>(ep.resid);
-    __nv_bfloat16* rc = reinterpret_cast<__nv_bfloat16*>(ep.row_copy);
-    float h[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      h[j] = c0 + j < M ? __bfloat162float(res[(size_t)(c0 + j) * ep.d + n]) : 0.f;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int2 br = s_rows[c0 + j];
-      if (c0 + j >= M || br.y < 0) continue;
-      const __nv_bfloat16 v = __float2bfloat16_rn(acc[j] + h[j]);
-      outb[((size_t)br.x * ep.N + br.y) * ep.d + n] = v;
-      if (rc) rc[(size_t)(c0 + j) * ep.d + n] = v;
-      if (ep.score_zero && n == 0) ep.score_zero[(size_t)br.x * ep.N + br.y] = 0.f;
-    }
-  } else if constexpr (MODE == EPI_SWIGLU) {
-    if (f >= 64) return;  // the up rows only feed their gate partners
-    const int fo = t * 64 + f;
-    if (fo >= ep.n_out) return;
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (c0 + j < M) outb[(size_t)(c0 + j) * ep.n_out + fo] = __float2bfloat16_rn(sk_silu(acc[j]) * partner[j]);
-  } else if constexpr (MODE == EPI_QKV) {
-    const int n = t * 128 + f;
-    if (n >= ep.n_out) return;
-    const int part = n / ep.d, col = n % ep.d;
-    const int hd = ep.head_dim, hh = hd / 2;
-    const int jj = col % hd, i = jj % hh;
-    const bool first = jj < hh;
-    float cs[32], sn[32];
-    if (part < 2) {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int2 br = s_rows[c0 + j];
-        const bool ok = c0 + j < M && br.y >= 0;
-        cs[j] = ok ? ep.rope_cos[(size_t)br.y * hh + i] : 0.f;
-        sn[j] = ok ? ep.rope_sin[(size_t)br.y * hh + i] : 0.f;
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int2 br = s_rows[c0 + j];
-      if (c0 + j >= M || br.y < 0) continue;
-      float v = acc[j];
-      if (part < 2) {
-        // first half: x1 c - x2 s; second half: x2 c + x1 s (x1 = first-half value)
-        v = first ? acc[j] * cs[j] - partner[j] * sn[j] : acc[j] * cs[j] + partner[j] * sn[j];
-      }
-      const __nv_bfloat16 b = __float2bfloat16_rn(v);
-      if (part == 0) outb[(size_t)(c0 + j) * ep.d + col] = b;
-      else reinterpret_cast<__nv_bfloat16*>(part == 1 ? ep.k_cache : ep.v_cache)[((size_t)br.x * ep.N + br.y) * ep.d + col] = b;
-    }
-  }
-}
-
-template <int MODE>
 __global__ void __launch_bounds__(kSkThreads, 1) tc_sk_kernel(const __grid_constant__ SkParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -201,9 +96,7 @@ __global__ void __launch_bounds__(kSkThreads, 1) tc_sk_kernel(const __grid_const
   __shared__ __align__(8) uint64_t empty_bar[kSkMaxStages];
   __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
   __shared__ uint32_t tmem_slot;
-  __shared__ int abort_flag, prod_issued, mma_consumed, s_flag, s_ok;
-  __shared__ int2 s_rows[256];
-  __shared__ float xch[4][32 * kSkXLd];
+  __shared__ int abort_flag, prod_issued, mma_consumed, s_ok;
 
   griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -211,10 +104,9 @@ __global__ void __launch_bounds__(kSkThreads, 1) tc_sk_kernel(const __grid_const
   const int KB = p.KB, U = p.units, NT = p.NT;
   const int u0 = sk_start(g, G, U), u1 = sk_start(g + 1, G, U);
   const int n_units = u1 - u0;
-  const int NACC = p.nacc, NBUF = p.nbuf;
+  const int NACC = p.nacc, NBUF = p.nbuf, FEAT = NACC * 128;
   const int W_BYTES = NACC * kSkW;
-  const int X_BYTES = NT * 128;
-  const int STAGE_BYTES = W_BYTES + X_BYTES;  // multiple of 1024
+  const int STAGE_BYTES = W_BYTES + NT * 128;  // multiple of 1024
   int STAGES = kSkRing / STAGE_BYTES;
   if (STAGES > kSkMaxStages) STAGES = kSkMaxStages;
   int* err = p.ep.err;
@@ -302,27 +194,19 @@ __global__ void __launch_bounds__(kSkThreads, 1) tc_sk_kernel(const __grid_const
       mma_consumed = it;
       umma_commit(&mma_done);  // every MMA issued by this thread has completed
     }
-  } else if (warp < 4) {
-    griddep_wait();
-    stage_rows_sk(p.ep, s_rows, threadIdx.x - 64, 64);
-    named_bar_sync(1, 192);
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
+    // the scratch slots were read by the previous launch's reduce kernel
     griddep_wait();
-    named_bar_sync(1, 192);  // s_rows staged
     const int q = warp - 4, f = q * 32 + lane;
     const int et = threadIdx.x - 128;  // 0..127
     const uint32_t lane_base = tmem + ((uint32_t)(q * 32) << 16);
-    // the RoPE / SwiGLU partner of feature f
-    const int half = MODE == EPI_SWIGLU ? 64 : p.ep.head_dim / 2;
-    const int pf = f ^ half;
-    const int pq = pf >> 5, pl = pf & 31;
     const int M = p.ep.M;
+    const int mt = M < NT ? M : NT;
     int j = 0;
     for (int u = u0; u < u1; ++j) {
-      const int t = u / KB, kb0 = u % KB;
-      const int kb1 = kb0 + (u1 - u < KB - kb0 ? u1 - u : KB - kb0);
-      u += kb1 - kb0;
+      const int kb0 = u % KB;
+      u += (u1 - u < KB - kb0 ? u1 - u : KB - kb0);
       const int a = j % NBUF;
       const bool got = mbar_wait(&acc_full[a], (j / NBUF) & 1, &abort_flag, err, 804);
       __syncwarp();
@@ -333,91 +217,19 @@ __global__ void __launch_bounds__(kSkThreads, 1) tc_sk_kernel(const __grid_const
       named_bar_sync(2, 128);
       if (!s_ok) break;
       tc_fence_after();
-      const uint32_t buf_tmem = lane_base + (uint32_t)(a * NACC * NT);
-      // the tile's segments: CTAs g_first..g_last, own index own_s
-      const int g_first = sk_owner(t * KB, G, U), g_last = sk_owner(t * KB + KB - 1, G, U);
-      const int nseg = g_last - g_first + 1, own_s = g - g_first;
-      bool finisher = true;
-      if (nseg > 1) {
-        if (et == 0) {
-          int c;
-          asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(c) : "l"(p.count + t) : "memory");
-          s_flag = (c == nseg - 1) ? 1 : 0;  // every other segment is in: no need to publish ours
-        }
-        named_bar_sync(2, 128);
-        finisher = s_flag != 0;
-        named_bar_sync(2, 128);
-        if (!finisher) {
-          for (int sub = 0; sub < NACC; ++sub) {
-            float* dst = p.part + (((size_t)sk_slot(g, t, G, U, KB) * NACC + sub) * 128 + f) * NT;
-            const uint32_t acc_tmem = buf_tmem + (uint32_t)(sub * NT);
-            for (int c0 = 0; c0 < NT; c0 += 32) {
-              float v[32];
-              tmem_ld32(acc_tmem + (uint32_t)c0, v);
+      // segment j of this CTA -> scratch slot g * maxseg + j, [NT][FEAT] fp32
+      float* dst = p.part + ((size_t)g * p.maxseg + j) * (size_t)NT * FEAT + f;
+      for (int sub = 0; sub < NACC; ++sub) {
+        const uint32_t acc_tmem = lane_base + (uint32_t)((a * NACC + sub) * NT);
+        for (int c0 = 0; c0 < mt; c0 += 32) {
+          float v[32];
+          tmem_ld32(acc_tmem + (uint32_t)c0, v);
 #pragma unroll
-              for (int i = 0; i < 32; i += 4)
-                __stcg(reinterpret_cast<float4*>(dst + c0 + i), make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
-            }
-          }
-          __threadfence();
-          named_bar_sync(2, 128);
-          if (et == 0) s_flag = (atomicAdd(p.count + t, 1) == nseg - 1) ? 1 : 0;
-          named_bar_sync(2, 128);
-          finisher = s_flag != 0;
-          named_bar_sync(2, 128);
+          for (int i = 0; i < 32; ++i)
+            if (c0 + i < mt) __stcg(dst + (size_t)(c0 + i) * FEAT + sub * 128, v[i]);
         }
       }
-      if (finisher) {
-        __threadfence();
-        for (int sub = 0; sub < NACC; ++sub)
-        for (int c0 = 0; c0 < NT && c0 < M; c0 += 32) {
-          const uint32_t acc_tmem = buf_tmem + (uint32_t)(sub * NT);
-          const int vt = t * NACC + sub;  // 128-row tile of the weights
-          float acc[32];
-          tmem_ld32(acc_tmem + (uint32_t)c0, acc);  // own partial
-          if (nseg > 1) {
-            float sum[32];
-            for (int s = 0; s < nseg; ++s) {  // k-block order
-              float x[32];
-              if (s == own_s) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = acc[i];
-              } else {
-                const float4* src = reinterpret_cast<const float4*>(
-                    p.part + (((size_t)sk_slot(g_first + s, t, G, U, KB) * NACC + sub) * 128 + f) * NT + c0);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  const float4 w = __ldcg(src + i);
-                  x[4 * i] = w.x; x[4 * i + 1] = w.y; x[4 * i + 2] = w.z; x[4 * i + 3] = w.w;
-                }
-              }
-              if (s == 0) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) sum[i] = x[i];
-              } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) sum[i] += x[i];
-              }
-            }
-#pragma unroll
-            for (int i = 0; i < 32; ++i) acc[i] = sum[i];
-          }
-          float partner[32];
-          if constexpr (MODE == EPI_QKV || MODE == EPI_SWIGLU) {
-            float* mine = xch[q];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) mine[i * kSkXLd + lane] = acc[i];
-            named_bar_sync(3, 128);
-            const float* theirs = xch[pq];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) partner[i] = theirs[i * kSkXLd + pl];
-            named_bar_sync(3, 128);
-          }
-          sk_store_chunk<MODE>(p, vt, f, c0, acc, partner, s_rows);
-        }
-        if (nseg > 1 && et == 0) p.count[t] = 0;  // every segment has counted: ready for the next launch
-      }
-      // the accumulator buffer may be overwritten by segment j + 2
+      // the accumulator buffer may be overwritten by segment j + NBUF
       tc_fence_before();
       named_bar_sync(2, 128);
       if (et == 0) mbar_arrive_cta(&acc_empty[a]);
@@ -438,35 +250,189 @@ __global__ void __launch_bounds__(kSkThreads, 1) tc_sk_kernel(const __grid_const
   if (warp == 0) tmem_dealloc(tmem, (uint32_t)p.tmem_cols);
 }
 
-cudaError_t launch_tc_sk(int mode, const SkParams& p, int grid, cudaStream_t stream) {
-  const void* kern = nullptr;
+// ---------------------------------------------------------------------------
+// Reduce + fused epilogue: one CTA per token row.
+// ---------------------------------------------------------------------------
+
+// Sum of feature group f4 (4 features at 4 * f4 of 128-row tile vt) over the
+// tile's segments, in k-block order; all loads issued before the sum.
+__device__ __forceinline__ float4 sk_sum4(const SkReduceParams& r, const int* s_nseg,
+                                          const int (*s_slot)[kRedMaxSeg], int t, int vt, int f4) {
+  const int tu = vt / r.nacc, sub = vt % r.nacc;
+  const int n = s_nseg[tu];
+  const size_t off = (size_t)t * r.feat + sub * 128 + f4 * 4;
+  float4 v[kRedMaxSeg];
+#pragma unroll
+  for (int s = 0; s < kRedMaxSeg; ++s)
+    if (s < n) v[s] = __ldcg(reinterpret_cast<const float4*>(r.part + (size_t)s_slot[tu][s] * r.slot_floats + off));
+  float4 acc = v[0];
+#pragma unroll
+  for (int s = 1; s < kRedMaxSeg; ++s)
+    if (s < n) {
+      acc.x += v[s].x; acc.y += v[s].y; acc.z += v[s].z; acc.w += v[s].w;
+    }
+  return acc;
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kRedThreads) sk_reduce_kernel(const __grid_constant__ SkReduceParams r) {
+  __shared__ int s_nseg[kRedMaxTiles];
+  __shared__ int s_slot[kRedMaxTiles][kRedMaxSeg];
+  __shared__ float s_red[kRedThreads / 32];
+  griddep_launch_dependents();
+  const int t = blockIdx.x;
+  const EpiParams& ep = r.ep;
+  // the segments of every tile (the same integer arithmetic as the GEMM's partition)
+  for (int tu = threadIdx.x; tu < r.n_tiles; tu += kRedThreads) {
+    const int gf = sk_owner(tu * r.KB, r.G, r.U), gl = sk_owner(tu * r.KB + r.KB - 1, r.G, r.U);
+    s_nseg[tu] = gl - gf + 1;
+    for (int s = 0; s <= gl - gf && s < kRedMaxSeg; ++s) {
+      const int gg = gf + s;
+      s_slot[tu][s] = gg * r.maxseg + (tu - sk_start(gg, r.G, r.U) / r.KB);
+    }
+  }
+  __syncthreads();
+  griddep_wait();  // the GEMM's partials, and the rows earlier kernels wrote
+  if (t >= ep.M) return;
+  const int b = t / ep.tokens_per_seq;
+  const int row = ep.idx ? ep.idx[t] : (t % ep.tokens_per_seq);
+  if (row < 0 || row >= ep.N) {
+    if (threadIdx.x == 0) report_error(ep.err, DEVERR_INDEX, 808);
+    return;
+  }
+  const size_t crow = (size_t)b * ep.N + row;  // the token's cache row
+  __nv_bfloat16* const outb = reinterpret_cast<__nv_bfloat16*>(ep.out);
+  const int nv = r.n_tiles * r.nacc;          // 128-row tiles
+  if constexpr (MODE == EPI_QKV) {
+    // item = 4 rotary pairs (features f1..f1+3 and f1+hd/2..) of one head
+    const int hd = ep.head_dim, hh = hd / 2, per_head = hd / 8;
+#pragma unroll 1
+    for (int it = threadIdx.x; it < nv * 16; it += kRedThreads) {
+      const int vt = it / 16, jt = it % 16;
+      const int hl = jt / per_head, jj = jt % per_head;
+      const int f1 = hl * hd + 4 * jj;
+      const int n1 = vt * 128 + f1;
+      if (n1 >= ep.n_out) continue;
+      const float4 x1 = sk_sum4(r, s_nseg, s_slot, t, vt, f1 / 4);
+      const float4 x2 = sk_sum4(r, s_nseg, s_slot, t, vt, (f1 + hh) / 4);
+      const int part = n1 / ep.d, col1 = n1 % ep.d, col2 = col1 + hh;
+      float4 a = x1, bb = x2;
+      if (part < 2) {
+        const float4 c = *reinterpret_cast<const float4*>(ep.rope_cos + (size_t)row * hh + 4 * jj);
+        const float4 s_ = *reinterpret_cast<const float4*>(ep.rope_sin + (size_t)row * hh + 4 * jj);
+        a = make_float4(x1.x * c.x - x2.x * s_.x, x1.y * c.y - x2.y * s_.y, x1.z * c.z - x2.z * s_.z,
+                        x1.w * c.w - x2.w * s_.w);
+        bb = make_float4(x2.x * c.x + x1.x * s_.x, x2.y * c.y + x1.y * s_.y, x2.z * c.z + x1.z * s_.z,
+                         x2.w * c.w + x1.w * s_.w);
+      }
+      __nv_bfloat16* dst = part == 0 ? outb + (size_t)t * ep.d
+                                     : reinterpret_cast<__nv_bfloat16*>(part == 1 ? ep.k_cache : ep.v_cache) +
+                                           crow * ep.d;
+      store4(dst + col1, a);
+      store4(dst + col2, bb);
+    }
+  } else if constexpr (MODE == EPI_SWIGLU) {
+#pragma unroll 1
+    for (int it = threadIdx.x; it < nv * 16; it += kRedThreads) {
+      const int vt = it / 16, f4 = it % 16;
+      const int fo = vt * 64 + 4 * f4;
+      if (fo >= ep.n_out) continue;
+      const float4 gt = sk_sum4(r, s_nseg, s_slot, t, vt, f4);
+      const float4 up = sk_sum4(r, s_nseg, s_slot, t, vt, f4 + 16);
+      store4(outb + (size_t)t * ep.n_out + fo,
+             make_float4(sk_silu(gt.x) * up.x, sk_silu(gt.y) * up.y, sk_silu(gt.z) * up.z, sk_silu(gt.w) * up.w));
+    }
+  } else {
+    // STORE, RESID (+ the FFN RMSNorm), RESID_SCATTER: 4 consecutive features per item
+    const __nv_bfloat16* res = reinterpret_cast<const __nv_bfloat16*>(ep.resid);
+    __nv_bfloat16* rc = reinterpret_cast<__nv_bfloat16*>(ep.row_copy);
+    float ss = 0.f;
+#pragma unroll 1
+    for (int it = threadIdx.x; it < nv * 32; it += kRedThreads) {
+      const int vt = it / 32, f4 = it % 32;
+      const int n = vt * 128 + 4 * f4;
+      if (n >= ep.n_out) continue;
+      float4 v = sk_sum4(r, s_nseg, s_slot, t, vt, f4);
+      if constexpr (MODE == EPI_STORE) {
+        store4(outb + (size_t)t * ep.n_out + n, v);
+      } else if constexpr (MODE == EPI_RESID) {
+        const float4 h = load4(res + crow * ep.d + n);
+        v = make_float4(v.x + h.x, v.y + h.y, v.z + h.z, v.w + h.w);
+        store4(outb + (size_t)t * ep.d + n, v);
+        if (r.x2) {  // sum of squares of the stored (bf16-rounded) values
+          const float qx = __bfloat162float(__float2bfloat16_rn(v.x)), qy = __bfloat162float(__float2bfloat16_rn(v.y));
+          const float qz = __bfloat162float(__float2bfloat16_rn(v.z)), qw = __bfloat162float(__float2bfloat16_rn(v.w));
+          ss += qx * qx + qy * qy + qz * qz + qw * qw;
+        }
+      } else {  // EPI_RESID_SCATTER
+        const float4 h = load4(res + (size_t)t * ep.d + n);
+        v = make_float4(v.x + h.x, v.y + h.y, v.z + h.z, v.w + h.w);
+        store4(outb + crow * ep.d + n, v);
+        if (rc) store4(rc + (size_t)t * ep.d + n, v);
+        if (ep.score_zero && n == 0) ep.score_zero[crow] = 0.f;
+      }
+    }
+    if constexpr (MODE == EPI_RESID) {
+      if (r.x2) {
+        // x2 = RMSNorm(H1) * gamma over the whole row (block sum in a fixed order)
+        ss = warp_sum(ss);
+        if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = ss;
+        __syncthreads();
+        float tot = 0.f;
+#pragma unroll
+        for (int w = 0; w < kRedThreads / 32; ++w) tot += s_red[w];
+        const float inv = 1.0f / sqrtf(tot / (float)ep.d + r.eps);
+        const __nv_bfloat16* gam = reinterpret_cast<const __nv_bfloat16*>(r.gamma);
+        __nv_bfloat16* x2 = reinterpret_cast<__nv_bfloat16*>(r.x2);
+#pragma unroll 1
+        for (int it = threadIdx.x; it < nv * 32; it += kRedThreads) {
+          const int n = (it / 32) * 128 + 4 * (it % 32);  // the items this thread stored above
+          if (n >= ep.n_out) continue;
+          const float4 h = load4(outb + (size_t)t * ep.d + n);
+          const float4 gm = load4(gam + n);
+          store4(x2 + (size_t)t * ep.d + n,
+                 make_float4(h.x * inv * gm.x, h.y * inv * gm.y, h.z * inv * gm.z, h.w * inv * gm.w));
+        }
+      }
+    }
+  }
+}
+
+cudaError_t launch_tc_sk(int mode, const SkParams& p, int grid, const SkReduceParams& r, cudaStream_t stream) {
+  cudaError_t e = configure_kernel((const void*)tc_sk_kernel, kSkSmem, false);
+  if (e != cudaSuccess) return e;
+  e = launch_k(tc_sk_kernel, dim3(grid), dim3(kSkThreads), kSkSmem, stream, p);
+  if (e != cudaSuccess) return e;
+  const dim3 rg(p.ep.M), rb(kRedThreads);
   switch (mode) {
-    case EPI_STORE: kern = (const void*)tc_sk_kernel<EPI_STORE>; break;
-    case EPI_QKV: kern = (const void*)tc_sk_kernel<EPI_QKV>; break;
-    case EPI_RESID: kern = (const void*)tc_sk_kernel<EPI_RESID>; break;
-    case EPI_SWIGLU: kern = (const void*)tc_sk_kernel<EPI_SWIGLU>; break;
-    case EPI_RESID_SCATTER: kern = (const void*)tc_sk_kernel<EPI_RESID_SCATTER>; break;
+    case EPI_STORE: return launch_k(sk_reduce_kernel<EPI_STORE>, rg, rb, 0, stream, r);
+    case EPI_QKV: return launch_k(sk_reduce_kernel<EPI_QKV>, rg, rb, 0, stream, r);
+    case EPI_RESID: return launch_k(sk_reduce_kernel<EPI_RESID>, rg, rb, 0, stream, r);
+    case EPI_SWIGLU: return launch_k(sk_reduce_kernel<EPI_SWIGLU>, rg, rb, 0, stream, r);
+    case EPI_RESID_SCATTER: return launch_k(sk_reduce_kernel<EPI_RESID_SCATTER>, rg, rb, 0, stream, r);
     default: return cudaErrorInvalidValue;
   }
-  cudaError_t e = configure_kernel(kern, kSkSmem, false);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(kSkThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSkSmem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl_enabled() ? 1 : 0;
-  void* args[] = {const_cast<SkParams*>(&p)};
-  return cudaLaunchKernelExC(&cfg, kern, args);
 }
 
 int sk_stages(int nacc, int NT) {
   const int st = kSkRing / (nacc * kSkW + NT * 128);
   return st < kSkMaxStages ? st : kSkMaxStages;
 }
+
+void sk_partition_bounds(int n_tiles, int KB, int G, int* max_seg_per_cta, int* max_seg_per_tile) {
+  const int U = n_tiles * KB;
+  int mc = 0, mt = 0;
+  for (int g = 0; g < G; ++g) {
+    const int a = sk_start(g, G, U), b = sk_start(g + 1, G, U);
+    if (b > a) mc = std::max(mc, (b - 1) / KB - a / KB + 1);
+  }
+  for (int tu = 0; tu < n_tiles; ++tu)
+    mt = std::max(mt, sk_owner(tu * KB + KB - 1, G, U) - sk_owner(tu * KB, G, U) + 1);
+  *max_seg_per_cta = mc;
+  *max_seg_per_tile = mt;
+}
+
+int sk_reduce_max_seg() { return kRedMaxSeg; }
+int sk_reduce_max_tiles() { return kRedMaxTiles; }
 
 }  // namespace spa

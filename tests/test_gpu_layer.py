@@ -158,7 +158,7 @@ def test_bf16_stream_k_partitions(monkeypatch, nacc, grid, B, N, k):
     # takes one TMEM buffer when two tiles share a unit
     monkeypatch.setenv("SPA_SK_GRID", grid)
     monkeypatch.setenv("SPA_SK_NACC", nacc)
-    lp = LayerPair(spa, SMALL_BF16, seed=80 + k, dtype=spa.SPA_BF16, max_B=2, max_N=200, std=0.05)
+    lp = LayerPair(spa, SMALL_BF16, seed=80 + k, dtype=spa.SPA_BF16, max_B=2, max_N=300, std=0.05)
     H = synth.hidden_states(B, N, 256, seed=k + 3, bf16=True)
     cache, ocs = _run_fill(lp, H)
     H2, _ = synth.drift_rows(H, 0.2, 0.5, seed=k + 4, bf16=True)
