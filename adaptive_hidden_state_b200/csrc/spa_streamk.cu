@@ -56,8 +56,9 @@ constexpr int kSkRing = 200 * 1024;      // bytes of the TMA ring (leaves room f
 constexpr int kSkMaxStages = 16;
 constexpr int kSkSmem = kSkRing + 1024;  // + alignment slack
 constexpr int kSkW = 128 * 128;          // one weight box: 128 rows x 64 columns bf16
-constexpr int kRedThreads = 128;
-constexpr int kRedMaxSeg = 16;    // segments per tile (the host keeps the grid within it)
+constexpr int kRedThreads = 256;
+constexpr int kRedMaxSeg = 8;     // segments per tile (the host keeps the grid within it)
+constexpr int kRedJobs = 4;       // feature groups summed per thread at once (all their loads in flight)
 constexpr int kRedMaxTiles = 256;
 
 __device__ __forceinline__ float sk_silu(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
@@ -254,24 +255,37 @@ __global__ void __launch_bounds__(kSkThreads, 1) tc_sk_kernel(const __grid_const
 // Reduce + fused epilogue: one CTA per token row.
 // ---------------------------------------------------------------------------
 
-// Sum of feature group f4 (4 features at 4 * f4 of 128-row tile vt) over the
-// tile's segments, in k-block order; all loads issued before the sum.
-__device__ __forceinline__ float4 sk_sum4(const SkReduceParams& r, const int* s_nseg,
-                                          const int (*s_slot)[kRedMaxSeg], int t, int vt, int f4) {
-  const int tu = vt / r.nacc, sub = vt % r.nacc;
-  const int n = s_nseg[tu];
-  const size_t off = (size_t)t * r.feat + sub * 128 + f4 * 4;
-  float4 v[kRedMaxSeg];
+// Sums of kRedJobs feature groups (4 features at 4 * f4[j] of 128-row tile
+// vt[j]; skipped where ok[j] is false) over their tiles' segments, each in
+// k-block order.  Every load of the jobs is issued before any sum, so a
+// thread keeps up to kRedJobs * kRedMaxSeg 16-byte loads in flight.
+__device__ __forceinline__ void sk_sum_jobs(const SkReduceParams& r, const int* s_nseg,
+                                            const int (*s_slot)[kRedMaxSeg], int t, const int* vt,
+                                            const int* f4, const bool* ok, float4* out) {
+  float4 v[kRedJobs][kRedMaxSeg];
+  int n[kRedJobs];
 #pragma unroll
-  for (int s = 0; s < kRedMaxSeg; ++s)
-    if (s < n) v[s] = __ldcg(reinterpret_cast<const float4*>(r.part + (size_t)s_slot[tu][s] * r.slot_floats + off));
-  float4 acc = v[0];
+  for (int j = 0; j < kRedJobs; ++j) {
+    n[j] = 0;
+    if (!ok[j]) continue;
+    const int tu = vt[j] / r.nacc, sub = vt[j] % r.nacc;
+    n[j] = s_nseg[tu];
+    const size_t off = (size_t)t * r.feat + sub * 128 + f4[j] * 4;
 #pragma unroll
-  for (int s = 1; s < kRedMaxSeg; ++s)
-    if (s < n) {
-      acc.x += v[s].x; acc.y += v[s].y; acc.z += v[s].z; acc.w += v[s].w;
-    }
-  return acc;
+    for (int s = 0; s < kRedMaxSeg; ++s)
+      if (s < n[j]) v[j][s] = __ldcg(reinterpret_cast<const float4*>(r.part + (size_t)s_slot[tu][s] * r.slot_floats + off));
+  }
+#pragma unroll
+  for (int j = 0; j < kRedJobs; ++j) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (n[j] > 0) acc = v[j][0];
+#pragma unroll
+    for (int s = 1; s < kRedMaxSeg; ++s)
+      if (s < n[j]) {
+        acc.x += v[j][s].x; acc.y += v[j][s].y; acc.z += v[j][s].z; acc.w += v[j][s].w;
+      }
+    out[j] = acc;
+  }
 }
 
 template <int MODE>
@@ -303,73 +317,107 @@ __global__ void __launch_bounds__(kRedThreads) sk_reduce_kernel(const __grid_con
   const size_t crow = (size_t)b * ep.N + row;  // the token's cache row
   __nv_bfloat16* const outb = reinterpret_cast<__nv_bfloat16*>(ep.out);
   const int nv = r.n_tiles * r.nacc;          // 128-row tiles
-  if constexpr (MODE == EPI_QKV) {
-    // item = 4 rotary pairs (features f1..f1+3 and f1+hd/2..) of one head
+  int vt[kRedJobs], f4[kRedJobs];
+  bool ok[kRedJobs];
+  float4 sum[kRedJobs];
+  if constexpr (MODE == EPI_QKV || MODE == EPI_SWIGLU) {
+    // two groups per item: QKV 4 rotary pairs (features f1.. and f1 + hd/2..)
+    // of one head; SwiGLU 4 gate features and their 4 up features
+    constexpr int IPB = kRedJobs / 2;  // items per batch
     const int hd = ep.head_dim, hh = hd / 2, per_head = hd / 8;
+    const int n_items = nv * 16;
 #pragma unroll 1
-    for (int it = threadIdx.x; it < nv * 16; it += kRedThreads) {
-      const int vt = it / 16, jt = it % 16;
-      const int hl = jt / per_head, jj = jt % per_head;
-      const int f1 = hl * hd + 4 * jj;
-      const int n1 = vt * 128 + f1;
-      if (n1 >= ep.n_out) continue;
-      const float4 x1 = sk_sum4(r, s_nseg, s_slot, t, vt, f1 / 4);
-      const float4 x2 = sk_sum4(r, s_nseg, s_slot, t, vt, (f1 + hh) / 4);
-      const int part = n1 / ep.d, col1 = n1 % ep.d, col2 = col1 + hh;
-      float4 a = x1, bb = x2;
-      if (part < 2) {
-        const float4 c = *reinterpret_cast<const float4*>(ep.rope_cos + (size_t)row * hh + 4 * jj);
-        const float4 s_ = *reinterpret_cast<const float4*>(ep.rope_sin + (size_t)row * hh + 4 * jj);
-        a = make_float4(x1.x * c.x - x2.x * s_.x, x1.y * c.y - x2.y * s_.y, x1.z * c.z - x2.z * s_.z,
-                        x1.w * c.w - x2.w * s_.w);
-        bb = make_float4(x2.x * c.x + x1.x * s_.x, x2.y * c.y + x1.y * s_.y, x2.z * c.z + x1.z * s_.z,
-                         x2.w * c.w + x1.w * s_.w);
+    for (int base = threadIdx.x; base < n_items; base += IPB * kRedThreads) {
+      int it[IPB];
+#pragma unroll
+      for (int i = 0; i < IPB; ++i) {
+        it[i] = base + i * kRedThreads;
+        const int v_ = it[i] / 16, jt = it[i] % 16;
+        int fa, fb;
+        if constexpr (MODE == EPI_QKV) {
+          const int hl = jt / per_head, jj = jt % per_head;
+          fa = hl * hd + 4 * jj;
+          fb = fa + hh;
+        } else {
+          fa = 4 * jt;
+          fb = fa + 64;
+        }
+        const bool in = it[i] < n_items &&
+                        (MODE == EPI_QKV ? v_ * 128 + fa < ep.n_out : v_ * 64 + 4 * jt < ep.n_out);
+        vt[2 * i] = vt[2 * i + 1] = v_;
+        f4[2 * i] = fa / 4;
+        f4[2 * i + 1] = fb / 4;
+        ok[2 * i] = ok[2 * i + 1] = in;
       }
-      __nv_bfloat16* dst = part == 0 ? outb + (size_t)t * ep.d
-                                     : reinterpret_cast<__nv_bfloat16*>(part == 1 ? ep.k_cache : ep.v_cache) +
-                                           crow * ep.d;
-      store4(dst + col1, a);
-      store4(dst + col2, bb);
-    }
-  } else if constexpr (MODE == EPI_SWIGLU) {
-#pragma unroll 1
-    for (int it = threadIdx.x; it < nv * 16; it += kRedThreads) {
-      const int vt = it / 16, f4 = it % 16;
-      const int fo = vt * 64 + 4 * f4;
-      if (fo >= ep.n_out) continue;
-      const float4 gt = sk_sum4(r, s_nseg, s_slot, t, vt, f4);
-      const float4 up = sk_sum4(r, s_nseg, s_slot, t, vt, f4 + 16);
-      store4(outb + (size_t)t * ep.n_out + fo,
-             make_float4(sk_silu(gt.x) * up.x, sk_silu(gt.y) * up.y, sk_silu(gt.z) * up.z, sk_silu(gt.w) * up.w));
+      sk_sum_jobs(r, s_nseg, s_slot, t, vt, f4, ok, sum);
+#pragma unroll
+      for (int i = 0; i < IPB; ++i) {
+        if (!ok[2 * i]) continue;
+        const float4 x1 = sum[2 * i], x2 = sum[2 * i + 1];
+        if constexpr (MODE == EPI_QKV) {
+          const int n1 = vt[2 * i] * 128 + 4 * f4[2 * i];
+          const int part = n1 / ep.d, col1 = n1 % ep.d, col2 = col1 + hh;
+          const int jj = (col1 % hd) / 4;
+          float4 a = x1, bb = x2;
+          if (part < 2) {
+            const float4 c = *reinterpret_cast<const float4*>(ep.rope_cos + (size_t)row * hh + 4 * jj);
+            const float4 s_ = *reinterpret_cast<const float4*>(ep.rope_sin + (size_t)row * hh + 4 * jj);
+            a = make_float4(x1.x * c.x - x2.x * s_.x, x1.y * c.y - x2.y * s_.y, x1.z * c.z - x2.z * s_.z,
+                            x1.w * c.w - x2.w * s_.w);
+            bb = make_float4(x2.x * c.x + x1.x * s_.x, x2.y * c.y + x1.y * s_.y, x2.z * c.z + x1.z * s_.z,
+                             x2.w * c.w + x1.w * s_.w);
+          }
+          __nv_bfloat16* dst = part == 0 ? outb + (size_t)t * ep.d
+                                         : reinterpret_cast<__nv_bfloat16*>(part == 1 ? ep.k_cache : ep.v_cache) +
+                                               crow * ep.d;
+          store4(dst + col1, a);
+          store4(dst + col2, bb);
+        } else {
+          const int fo = vt[2 * i] * 64 + 4 * f4[2 * i];
+          store4(outb + (size_t)t * ep.n_out + fo,
+                 make_float4(sk_silu(x1.x) * x2.x, sk_silu(x1.y) * x2.y, sk_silu(x1.z) * x2.z, sk_silu(x1.w) * x2.w));
+        }
+      }
     }
   } else {
     // STORE, RESID (+ the FFN RMSNorm), RESID_SCATTER: 4 consecutive features per item
     const __nv_bfloat16* res = reinterpret_cast<const __nv_bfloat16*>(ep.resid);
     __nv_bfloat16* rc = reinterpret_cast<__nv_bfloat16*>(ep.row_copy);
+    const int n_items = nv * 32;
     float ss = 0.f;
 #pragma unroll 1
-    for (int it = threadIdx.x; it < nv * 32; it += kRedThreads) {
-      const int vt = it / 32, f4 = it % 32;
-      const int n = vt * 128 + 4 * f4;
-      if (n >= ep.n_out) continue;
-      float4 v = sk_sum4(r, s_nseg, s_slot, t, vt, f4);
-      if constexpr (MODE == EPI_STORE) {
-        store4(outb + (size_t)t * ep.n_out + n, v);
-      } else if constexpr (MODE == EPI_RESID) {
-        const float4 h = load4(res + crow * ep.d + n);
-        v = make_float4(v.x + h.x, v.y + h.y, v.z + h.z, v.w + h.w);
-        store4(outb + (size_t)t * ep.d + n, v);
-        if (r.x2) {  // sum of squares of the stored (bf16-rounded) values
-          const float qx = __bfloat162float(__float2bfloat16_rn(v.x)), qy = __bfloat162float(__float2bfloat16_rn(v.y));
-          const float qz = __bfloat162float(__float2bfloat16_rn(v.z)), qw = __bfloat162float(__float2bfloat16_rn(v.w));
-          ss += qx * qx + qy * qy + qz * qz + qw * qw;
+    for (int base = threadIdx.x; base < n_items; base += kRedJobs * kRedThreads) {
+#pragma unroll
+      for (int j = 0; j < kRedJobs; ++j) {
+        const int it = base + j * kRedThreads;
+        vt[j] = it / 32;
+        f4[j] = it % 32;
+        ok[j] = it < n_items && vt[j] * 128 + 4 * f4[j] < ep.n_out;
+      }
+      sk_sum_jobs(r, s_nseg, s_slot, t, vt, f4, ok, sum);
+#pragma unroll
+      for (int j = 0; j < kRedJobs; ++j) {
+        if (!ok[j]) continue;
+        const int n = vt[j] * 128 + 4 * f4[j];
+        float4 v = sum[j];
+        if constexpr (MODE == EPI_STORE) {
+          store4(outb + (size_t)t * ep.n_out + n, v);
+        } else if constexpr (MODE == EPI_RESID) {
+          const float4 h = load4(res + crow * ep.d + n);
+          v = make_float4(v.x + h.x, v.y + h.y, v.z + h.z, v.w + h.w);
+          store4(outb + (size_t)t * ep.d + n, v);
+          if (r.x2) {  // sum of squares of the stored (bf16-rounded) values
+            const float qx = __bfloat162float(__float2bfloat16_rn(v.x)), qy = __bfloat162float(__float2bfloat16_rn(v.y));
+            const float qz = __bfloat162float(__float2bfloat16_rn(v.z)), qw = __bfloat162float(__float2bfloat16_rn(v.w));
+            ss += qx * qx + qy * qy + qz * qz + qw * qw;
+          }
+        } else {  // EPI_RESID_SCATTER
+          const float4 h = load4(res + (size_t)t * ep.d + n);
+          v = make_float4(v.x + h.x, v.y + h.y, v.z + h.z, v.w + h.w);
+          store4(outb + crow * ep.d + n, v);
+          if (rc) store4(rc + (size_t)t * ep.d + n, v);
+          if (ep.score_zero && n == 0) ep.score_zero[crow] = 0.f;
         }
-      } else {  // EPI_RESID_SCATTER
-        const float4 h = load4(res + (size_t)t * ep.d + n);
-        v = make_float4(v.x + h.x, v.y + h.y, v.z + h.z, v.w + h.w);
-        store4(outb + crow * ep.d + n, v);
-        if (rc) store4(rc + (size_t)t * ep.d + n, v);
-        if (ep.score_zero && n == 0) ep.score_zero[crow] = 0.f;
       }
     }
     if constexpr (MODE == EPI_RESID) {
@@ -385,8 +433,8 @@ __global__ void __launch_bounds__(kRedThreads) sk_reduce_kernel(const __grid_con
         const __nv_bfloat16* gam = reinterpret_cast<const __nv_bfloat16*>(r.gamma);
         __nv_bfloat16* x2 = reinterpret_cast<__nv_bfloat16*>(r.x2);
 #pragma unroll 1
-        for (int it = threadIdx.x; it < nv * 32; it += kRedThreads) {
-          const int n = (it / 32) * 128 + 4 * (it % 32);  // the items this thread stored above
+        for (int it = threadIdx.x; it < n_items; it += kRedThreads) {
+          const int n = (it / 32) * 128 + 4 * (it % 32);  // items this thread stored above
           if (n >= ep.n_out) continue;
           const float4 h = load4(outb + (size_t)t * ep.d + n);
           const float4 gm = load4(gam + n);
