@@ -702,11 +702,11 @@ static int run_ws(int mode, bool gateup, TcWsParams& p, const void* X, int M, in
 // 128 output features (gate/up: 64 features, 64 gate + 64 up rows) times the
 // [M, K] bf16 token operand X, K / 64 k-blocks each, over one CTA per SM.
 static bool streamk_enabled() {
-  static const bool on = [] {
-    const char* e = std::getenv("SPA_STREAMK");
-    return !(e && e[0] == '0');
-  }();
-  return on;
+  // opt-in (SPA_STREAMK=1): measured slower than the cluster split-K kernel on
+  // the LLaDA-shaped layer, because the fp32 partials it writes and re-reads
+  // cost more than its even spread over the SMs gains
+  const char* e = std::getenv("SPA_STREAMK");
+  return e && e[0] == '1';
 }
 
 static int run_sk(int mode, SkParams& p, spa_workspace* ws, const void* X, int M, int K, int tiles128,

@@ -151,11 +151,12 @@ def test_bf16_wide_weight_tiles(monkeypatch, nacc, B, N, k):
 @pytest.mark.parametrize("grid", ["1", "5", "12", "24"])
 @pytest.mark.parametrize("B,N,k", [(1, 200, 96), (2, 160, 33), (1, 300, 200)])
 def test_bf16_stream_k_partitions(monkeypatch, nacc, grid, B, N, k):
-    # the stream-K weight-streaming GEMMs over 1, 5, 12 and 24 CTAs with one
+    # the opt-in stream-K weight-streaming GEMMs over 1, 5, 12 and 24 CTAs with one
     # or two 128-row tiles per unit: one CTA for everything, ranges that split
     # tiles unevenly, and one k-block per CTA (QKV and gate/up: 24 units of
     # one tile, 12 of two), so every tile is fixed up from 4 partials; k = 200
     # takes one TMEM buffer when two tiles share a unit
+    monkeypatch.setenv("SPA_STREAMK", "1")
     monkeypatch.setenv("SPA_SK_GRID", grid)
     monkeypatch.setenv("SPA_SK_NACC", nacc)
     lp = LayerPair(spa, SMALL_BF16, seed=80 + k, dtype=spa.SPA_BF16, max_B=2, max_N=300, std=0.05)
