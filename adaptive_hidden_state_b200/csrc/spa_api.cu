@@ -195,6 +195,9 @@ struct spa_workspace {
   int* err = nullptr;       // [2]
   float* sk_part = nullptr;  // stream-K GEMM: the segments' partial tiles (fp32)
   size_t sk_part_floats = 0;
+  float* ffn_part = nullptr;  // persistent FFN: the three phases' partial tiles (fp32)
+  size_t ffn_part_floats = 0;
+  int* ffn_sync = nullptr;    // persistent FFN: [8] phase counters
   float* rope_cos = nullptr;  // [max_N, hd/2]
   float* rope_sin = nullptr;
   CUtensorMap tmX, tmO, tmX2, tmA;
@@ -362,6 +365,74 @@ static size_t sk_scratch_floats(int sms, int d, int F) {
   return need;
 }
 
+// Plan of the persistent FFN for NT tokens per MMA on `sms` SMs: per phase
+// (O-proj, gate/up, down) the tile width, tiles, k-blocks, units, the
+// busiest CTA's segments and the total; one grid for all three phases.
+struct FfnPlan {
+  int nacc[3], n_tiles[3], KB[3], units[3], maxseg[3], seg_total[3], grid;
+  size_t part_floats[3];
+  bool ok;
+};
+
+static FfnPlan ffn_plan(int d, int F, int NT, int sms) {
+  FfnPlan pl;
+  std::memset(&pl, 0, sizeof(pl));
+  const int tiles128[3] = {d / 128, F / 64, d / 128}, K[3] = {d, d, F};
+  int min_units = 1 << 30;
+  for (int ph = 0; ph < 3; ++ph) {
+    // two 128-row gate/up tiles per unit while two TMEM buffers of both fit
+    pl.nacc[ph] = (ph == 1 && NT <= 128 && tiles128[ph] % 2 == 0) ? 2 : 1;
+    if (const char* env = std::getenv("SPA_FFN_NACC"))  // tuning override of the gate/up width
+      if (ph == 1 && env[0] == '1') pl.nacc[ph] = 1;
+    pl.n_tiles[ph] = tiles128[ph] / pl.nacc[ph];
+    pl.KB[ph] = K[ph] / 64;
+    pl.units[ph] = pl.n_tiles[ph] * pl.KB[ph];
+    min_units = std::min(min_units, pl.units[ph]);
+  }
+  pl.grid = std::max(1, std::min(sms, min_units / 4));
+  if (const char* env = std::getenv("SPA_FFN_GRID")) {  // tuning / test override, 1..SMs and <= units
+    const int v = std::atoi(env);
+    if (v >= 1 && v <= sms && v <= min_units) pl.grid = v;
+  }
+  pl.ok = true;
+  for (;;) {
+    bool fits = true;
+    for (int ph = 0; ph < 3; ++ph) {
+      int mc = 0, mt = 0;
+      sk_partition_bounds(pl.n_tiles[ph], pl.KB[ph], pl.grid, &mc, &mt);
+      if (mt > ffn_max_seg()) fits = false;
+      pl.maxseg[ph] = mc;
+    }
+    if (fits || pl.grid == 1) {
+      pl.ok = fits;
+      break;
+    }
+    --pl.grid;
+  }
+  for (int ph = 0; ph < 3; ++ph) {
+    if (pl.n_tiles[ph] > ffn_max_tiles()) pl.ok = false;
+    // every CTA's segments of the phase
+    const int U = pl.units[ph], KB = pl.KB[ph];
+    int tot = 0;
+    for (int g = 0; g < pl.grid; ++g) {
+      const int a = (int)(((long long)g * U) / pl.grid), b = (int)(((long long)(g + 1) * U) / pl.grid);
+      if (b > a) tot += (b - 1) / KB - a / KB + 1;
+    }
+    pl.seg_total[ph] = tot;
+    pl.part_floats[ph] = (size_t)pl.grid * pl.maxseg[ph] * NT * pl.nacc[ph] * 128;
+  }
+  return pl;
+}
+
+static size_t ffn_scratch_floats(int sms, int d, int F) {
+  size_t need = 0;
+  for (int NT = 32; NT <= 256; NT += 32) {
+    const FfnPlan pl = ffn_plan(d, F, NT, sms);
+    need = std::max(need, pl.part_floats[0] + pl.part_floats[1] + pl.part_floats[2]);
+  }
+  return need;
+}
+
 extern "C" void spa_workspace_free(spa_workspace* ws) {
   if (!ws) return;
   for (void* p : ws->allocs) cudaFree(p);
@@ -410,6 +481,9 @@ extern "C" int spa_workspace_create(const spa_layer_desc* desc, int max_B, int m
   if (desc->dtype == SPA_BF16) {
     ws->sk_part_floats = sk_scratch_floats(ws->num_sms, (int)d, (int)F);
     WS_ALLOC(sk_part, ws->sk_part_floats * 4)
+    ws->ffn_part_floats = ffn_scratch_floats(ws->num_sms, (int)d, (int)F);
+    WS_ALLOC(ffn_part, ws->ffn_part_floats * 4)
+    WS_ALLOC(ffn_sync, 8 * sizeof(int))
   }
   WS_ALLOC(rope_cos, (size_t)max_N * (desc->head_dim / 2) * 4)
   WS_ALLOC(rope_sin, (size_t)max_N * (desc->head_dim / 2) * 4)
@@ -431,7 +505,8 @@ extern "C" int spa_workspace_create(const spa_layer_desc* desc, int max_B, int m
   if (cudaMemcpy(ws->rope_cos, cs.data(), cs.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
       cudaMemcpy(ws->rope_sin, sn.data(), sn.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
       cudaMemset(ws->err, 0, 2 * sizeof(int)) != cudaSuccess ||
-      cudaMemset(ws->attn_sync, 0, (size_t)ws->attn_sync_len * sizeof(int)) != cudaSuccess) {
+      cudaMemset(ws->attn_sync, 0, (size_t)ws->attn_sync_len * sizeof(int)) != cudaSuccess ||
+      (ws->ffn_sync && cudaMemset(ws->ffn_sync, 0, 8 * sizeof(int)) != cudaSuccess)) {
     spa_workspace_free(ws);
     return fail(SPA_ERR_CUDA, "workspace initialisation copy failed");
   }
@@ -455,6 +530,7 @@ extern "C" int spa_workspace_status(spa_workspace* ws, void* stream) {
   SPA_CK(cudaMemset(ws->err, 0, sizeof(h)));
   // a kernel that gave up may have left split counters behind: start them afresh
   SPA_CK(cudaMemset(ws->attn_sync, 0, (size_t)ws->attn_sync_len * sizeof(int)));
+  if (ws->ffn_sync) SPA_CK(cudaMemset(ws->ffn_sync, 0, 8 * sizeof(int)));
   if (h[0] & DEVERR_TIMEOUT) return fail(SPA_ERR_TIMEOUT, "device wait timed out (site %d)", h[1]);
   return fail(SPA_ERR_DEVICE, "device check failed: bits 0x%x site %d", h[0], h[1]);
 }
@@ -914,6 +990,66 @@ static int run_attn_half(spa_layer* L, const void* H, const int32_t* idx, int tp
 // Phase 3 for the M = B * tps selected rows whose attention outputs are the
 // compact rows of Ob (tmOb: its tensor map, bf16): H1 = H[I] + O W_o^T,
 // x2 = RMSNorm(H1), A = SwiGLU, H^c[I] = H1 + A W_down^T.
+static bool ffn_persistent_enabled() {
+  const char* e = std::getenv("SPA_FFN");
+  return e && e[0] == '1';
+}
+
+// The persistent FFN half (M <= 256 bf16 tokens): one launch for the O-proj,
+// the FFN RMSNorm, gate/up + SwiGLU and down + H^c scatter.  Returns
+// SPA_ERR_UNSUPPORTED (nothing launched) when the shapes do not fit its plan.
+static int run_ffn_persistent(spa_layer* L, const void* H, const int32_t* idx, int tps, const spa_layer_cache* c,
+                              cudaStream_t s, const void* Ob, void* row_copy, float* score_zero) {
+  spa_workspace* ws = L->ws;
+  const spa_layer_desc& D = L->desc;
+  const int d = D.d, F = D.ffn, M = c->B * tps;
+  const int NT = ((M + 31) / 32) * 32;
+  const FfnPlan pl = ffn_plan(d, F, NT, ws->num_sms);
+  if (!pl.ok || pl.part_floats[0] + pl.part_floats[1] + pl.part_floats[2] > ws->ffn_part_floats)
+    return SPA_ERR_UNSUPPORTED;
+  FfnParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.tmWo = L->tm_wo;
+  p.tmWg = L->tm_wg64;
+  p.tmWu = L->tm_wu64;
+  p.tmWd = L->tm_wd;
+  if (encode_bf16_map_box(&p.tmX[0], Ob, (uint64_t)M, (uint64_t)d, (uint32_t)NT) ||
+      encode_bf16_map_box(&p.tmX[1], ws->X2, (uint64_t)M, (uint64_t)d, (uint32_t)NT) ||
+      encode_bf16_map_box(&p.tmX[2], ws->A, (uint64_t)M, (uint64_t)F, (uint32_t)NT))
+    return fail(SPA_ERR_CUDA, "tensor maps of the FFN token operands failed");
+  p.d = d; p.F = F; p.M = M; p.NT = NT; p.tps = tps; p.N = c->N; p.idx = idx;
+  p.H = (const __nv_bfloat16*)H;
+  p.gamma = (const __nv_bfloat16*)L->w.ffn_norm;
+  p.eps = D.rms_eps;
+  p.H1 = (__nv_bfloat16*)ws->H1;
+  p.X2 = (__nv_bfloat16*)ws->X2;
+  p.A = (__nv_bfloat16*)ws->A;
+  p.Hc = (__nv_bfloat16*)c->h_cache;
+  p.row_copy = (__nv_bfloat16*)row_copy;
+  p.score_zero = score_zero;
+  size_t off = 0;
+  for (int ph = 0; ph < 3; ++ph) {
+    p.KB[ph] = pl.KB[ph]; p.nacc[ph] = pl.nacc[ph]; p.n_tiles[ph] = pl.n_tiles[ph];
+    p.units[ph] = pl.units[ph]; p.maxseg[ph] = pl.maxseg[ph]; p.seg_total[ph] = pl.seg_total[ph];
+    p.part[ph] = ws->ffn_part + off;
+    off += pl.part_floats[ph];
+    p.max_nacc = std::max(p.max_nacc, pl.nacc[ph]);
+  }
+  p.acc_cols = p.max_nacc * NT;
+  int cols = 32;
+  while (cols < 2 * p.acc_cols) cols *= 2;
+  p.tmem_cols = cols;
+  p.sync = ws->ffn_sync;
+  p.err = ws->err;
+  const double es = 2.0, Md = (double)M * d;
+  const double wbytes = ((double)d * d + 3.0 * d * F) * es;
+  ProfScope ps(&ws->prof, SPA_PROF_FFN, wbytes + 6.0 * Md * es + 2.0 * (double)M * F * es,
+               2.0 * Md * d + 6.0 * Md * F, s);
+  const cudaError_t e = launch_ffn_persistent(p, pl.grid, s);
+  if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "persistent FFN launch: %s", cudaGetErrorString(e));
+  return SPA_OK;
+}
+
 static int run_ffn_half(spa_layer* L, const void* H, const int32_t* idx, int tps,
                         const spa_layer_cache* c, cudaStream_t s, const void* Ob, const CUtensorMap* tmOb,
                         void* row_copy, float* score_zero) {
@@ -924,6 +1060,10 @@ static int run_ffn_half(spa_layer* L, const void* H, const int32_t* idx, int tps
   const double es = bf ? 2.0 : 4.0, Md = (double)M * d;
   Profiler* prof = &ws->prof;
   cudaError_t e;
+  if (bf && M <= 256 && ffn_persistent_enabled()) {
+    const int st = run_ffn_persistent(L, H, idx, tps, c, s, Ob, row_copy, score_zero);
+    if (st != SPA_ERR_UNSUPPORTED) return st;  // otherwise the separate kernels below
+  }
   // H1 = H[I] + O W_o^T
   {
     EpiParams ep = base_epi(L, M, tps, N, idx);

@@ -2,6 +2,7 @@
 #pragma once
 #include <cstdint>
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 namespace spa {
@@ -114,6 +115,26 @@ struct SkReduceParams {
   EpiParams ep;
 };
 
+// Persistent FFN half of a cached layer step (spa_ffn.cu): O-proj (+ the FFN
+// RMSNorm), gate/up with SwiGLU and down with the H^c scatter in one launch;
+// phase p in 0..2, each split stream-K over the grid.
+struct alignas(64) FfnParams {
+  CUtensorMap tmWo, tmWg, tmWu, tmWd;  // W_o, W_down: 128-row boxes; W_gate, W_up: 64-row boxes
+  CUtensorMap tmX[3];  // token operands: O [M, d], X2 [M, d], A [M, F]; box 64 x NT
+  int d, F, M, NT, tps, N;
+  const int32_t* idx;  // [B * tps] cache rows of the tokens (null: t % tps)
+  const __nv_bfloat16* H;      // layer input [B, N, d] (residual of the O-proj)
+  const __nv_bfloat16* gamma;  // FFN RMSNorm gain [d]
+  float eps;
+  __nv_bfloat16 *H1, *X2, *A, *Hc, *row_copy;  // outputs (row_copy may be null)
+  float* score_zero;   // or null
+  int KB[3], nacc[3], n_tiles[3], units[3], maxseg[3], seg_total[3];
+  int max_nacc, acc_cols, tmem_cols;  // acc_cols = max nacc * NT; tmem_cols >= 2 * acc_cols
+  float* part[3];      // per-phase scratch slots (g * maxseg + j) = [NT][nacc * 128] fp32
+  int* sync;           // [8] segments counted, rows finished (per phase), CTAs done
+  int* err;
+};
+
 struct SimtGemmParams {
   const float* A;      // [M, K]
   const float* B[3];
@@ -133,6 +154,10 @@ cudaError_t launch_tc_gemm(int mode, int BN, const TcGemmParams& p, int m_tiles,
 cudaError_t launch_tc_ws(int mode, int nacc, const TcWsParams& p, int n_tiles, int splits,
                          cudaStream_t stream);
 int plan_ws_splits(int mode, int nacc, int n_tiles, int KB);
+// The persistent FFN kernel over `grid` CTAs (at most one per SM).
+cudaError_t launch_ffn_persistent(const FfnParams& p, int grid, cudaStream_t stream);
+int ffn_max_seg();    // segments per tile the reducers take
+int ffn_max_tiles();  // unit tiles per phase
 // Stream-K weight-streaming GEMM over `grid` CTAs (one per SM), then its
 // per-row reduce + epilogue kernel (M CTAs).
 cudaError_t launch_tc_sk(int mode, const SkParams& p, int grid, const SkReduceParams& r, cudaStream_t stream);

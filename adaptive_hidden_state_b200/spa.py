@@ -42,7 +42,7 @@ EXPORTS = [
 ]
 
 
-PROF_CLASSES = ["proxy", "topk", "norm", "qkv", "attn", "oproj", "gateup", "down", "lmhead", "misc"]
+PROF_CLASSES = ["proxy", "topk", "norm", "qkv", "attn", "oproj", "gateup", "down", "lmhead", "misc", "ffn"]
 
 
 def spa_launch_count() -> int:

@@ -41,8 +41,8 @@ CFG = dict(L=32, d=4096, n_heads=32, head_dim=128, ffn=12288, vocab=126464, B=1,
 WORKLOAD = ("LLaDA-8B-shaped 32-layer bf16 DLM decode step: B=1, N=1024 (256 prompt + 768 masked), "
             "r=128, piecewise-Gaussian rho(l) (rho_p=0.25, l_p=12, rho_1=rho_L=0.06), "
             "2 tokens unmasked per step")
-PROF_CLASSES = ["proxy", "topk", "norm", "qkv", "attn", "oproj", "gateup", "down", "lmhead", "misc"]
-LAYER_CLASSES = ["proxy", "topk", "norm", "qkv", "attn", "oproj", "gateup", "down"]
+PROF_CLASSES = ["proxy", "topk", "norm", "qkv", "attn", "oproj", "gateup", "down", "lmhead", "misc", "ffn"]
+LAYER_CLASSES = ["proxy", "topk", "norm", "qkv", "attn", "oproj", "gateup", "down", "ffn"]
 
 
 def parse_args():

@@ -140,6 +140,7 @@ enum {
   SPA_PROF_DOWN,      /* down GEMM + residual + H^c scatter */
   SPA_PROF_LMHEAD,    /* LM head GEMM + per-tile argmax */
   SPA_PROF_MISC,      /* embedding rows, final norm, argmax reduction */
+  SPA_PROF_FFN,       /* the persistent FFN half: O-proj + FFN norm + gate/up + down in one launch */
   SPA_PROF_CLASSES
 };
 int spa_profile_enable(spa_workspace *ws, int enable);

@@ -166,6 +166,24 @@ def test_bf16_stream_k_partitions(monkeypatch, nacc, grid, B, N, k):
     _step(lp, cache, ocs, H2, k)
 
 
+@pytest.mark.parametrize("grid", ["", "3", "8"])
+@pytest.mark.parametrize("B,N,k", [(1, 200, 96), (2, 160, 33), (1, 300, 200)])
+def test_bf16_persistent_ffn(monkeypatch, grid, B, N, k):
+    # the FFN half as one persistent launch (O-proj, FFN norm, gate/up, down
+    # streamed back to back, each phase split over the CTAs), over the
+    # planner's grid and over 3 and 8 CTAs (tiles fixed up from up to 4
+    # partials); k = 200 takes one 128-row gate/up tile per unit
+    monkeypatch.setenv("SPA_FFN", "1")
+    if grid:
+        monkeypatch.setenv("SPA_FFN_GRID", grid)
+    lp = LayerPair(spa, SMALL_BF16, seed=90 + k, dtype=spa.SPA_BF16, max_B=2, max_N=300, std=0.05)
+    H = synth.hidden_states(B, N, 256, seed=k + 5, bf16=True)
+    cache, ocs = _run_fill(lp, H)
+    H2, _ = synth.drift_rows(H, 0.2, 0.5, seed=k + 6, bf16=True)
+    _step(lp, cache, ocs, H2, k)
+    _step(lp, cache, ocs, H, k)   # a second launch: the counters were reset by the first
+
+
 @pytest.mark.parametrize("B,N,k", [(1, 2048, 200), (2, 1000, 62), (1, 1536, 129), (1, 3000, 200)])
 def test_bf16_split_key_attention(B, N, k):
     # long caches: the keys of each query tile are split over a cluster of 8,
@@ -270,6 +288,18 @@ def test_llada_fill_then_cached_step(llada):
     H2, rows = synth.drift_rows(H, 0.05, 0.3, seed=2, bf16=True)   # 26 drifted rows
     I, _ = _step(lp, cache, ocs, H2, 128)
     assert set(rows[0].tolist()) <= set(I[0].tolist())
+
+
+def test_llada_persistent_ffn_cached_steps(llada, monkeypatch):
+    # the persistent FFN launch at the LLaDA layer shape (148 CTAs), over two
+    # cached steps (the second one reuses the counters the first reset)
+    monkeypatch.setenv("SPA_FFN", "1")
+    lp, H = llada
+    cache, ocs = _run_fill(lp, H)
+    H2, rows = synth.drift_rows(H, 0.05, 0.3, seed=2, bf16=True)
+    I, _ = _step(lp, cache, ocs, H2, 128)
+    assert set(rows[0].tolist()) <= set(I[0].tolist())
+    _step(lp, cache, ocs, H, 200)
 
 
 def test_llada_graded_drift_exact_selection(llada):
