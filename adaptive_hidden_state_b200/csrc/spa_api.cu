@@ -198,6 +198,7 @@ struct spa_workspace {
   float* ffn_part = nullptr;  // persistent FFN: the three phases' partial tiles (fp32)
   size_t ffn_part_floats = 0;
   int* ffn_sync = nullptr;    // persistent FFN: [8] phase counters
+  float* ss_part = nullptr;   // folded FFN RMSNorm: per (token, 128-feature tile) sums of H1^2
   float* rope_cos = nullptr;  // [max_N, hd/2]
   float* rope_sin = nullptr;
   CUtensorMap tmX, tmO, tmX2, tmA;
@@ -484,6 +485,7 @@ extern "C" int spa_workspace_create(const spa_layer_desc* desc, int max_B, int m
     ws->ffn_part_floats = ffn_scratch_floats(ws->num_sms, (int)d, (int)F);
     WS_ALLOC(ffn_part, ws->ffn_part_floats * 4)
     WS_ALLOC(ffn_sync, 8 * sizeof(int))
+    WS_ALLOC(ss_part, std::min<size_t>(cap, 256) * ((d + 127) / 128) * 4)
   }
   WS_ALLOC(rope_cos, (size_t)max_N * (desc->head_dim / 2) * 4)
   WS_ALLOC(rope_sin, (size_t)max_N * (desc->head_dim / 2) * 4)
@@ -735,12 +737,16 @@ static int run_ws(int mode, bool gateup, TcWsParams& p, const void* X, int M, in
   if (M <= 0) return SPA_OK;
   if (M > 256) return fail(SPA_ERR_SHAPE, "weight-stationary GEMM takes at most 256 tokens");
   const int NT = ((M + 31) / 32) * 32;
-  // The layer GEMMs stream faster with one 128-row block per CTA (two for
-  // gate/up): smaller TMA ring stages, more of them in flight.  Only a GEMM
-  // with many more weight rows than the SMs can cover (the LM head) takes
-  // larger blocks, which need fewer TMA boxes per weight byte.
+  // Two 128-row blocks per CTA (gate/up: a W_gate and a W_up block) halve
+  // the token-tile traffic per weight byte: each CTA's TMA stream then moves
+  // 48 KB per stage for 32 KB of weights instead of 32 KB for 16 KB, which
+  // lets ~96 CTAs stream near the HBM rate.  A GEMM with fewer rows (O-proj,
+  // down: 32 blocks of 128) keeps one block per CTA so that its split-K
+  // clusters still cover the SMs.  Only a GEMM with many more weight rows
+  // than the SMs can cover (the LM head) takes four.
   const int min_nacc = gateup ? 2 : 1;
   int nacc = min_nacc;
+  if (!gateup && rows % 256 == 0 && rows / 128 >= 64 && 2 * NT <= 512) nacc = 2;
   if (rows / 128 > 4 * ws_num_sms_hint)
     for (int n = 4; n > min_nacc; n /= 2) {
       const int feat = gateup ? n / 2 * 128 : n * 128;
@@ -753,6 +759,7 @@ static int run_ws(int mode, bool gateup, TcWsParams& p, const void* X, int M, in
     const int v = std::atoi(env);
     if ((v == 1 || v == 2 || v == 4) && v >= min_nacc && v * NT <= 512) nacc = v;
   }
+  if (p.ep.x2 != nullptr) nacc = 1;  // the folded FFN norm sums a row's squares over 128-feature tiles
   const int feat = gateup ? nacc / 2 * 128 : nacc * 128;
   const int n_tiles = (rows + feat - 1) / feat;
   if (encode_bf16_map_box(&p.tmX, X, (uint64_t)M, (uint64_t)K, (uint32_t)NT))
@@ -1050,6 +1057,13 @@ static int run_ffn_persistent(spa_layer* L, const void* H, const int32_t* idx, i
   return SPA_OK;
 }
 
+// The FFN RMSNorm folded into the O-proj and gate/up epilogues of the
+// weight-stationary path (SPA_NORM_FOLD=0: a separate norm kernel instead).
+static bool norm_fold_enabled() {
+  const char* e = std::getenv("SPA_NORM_FOLD");
+  return !(e && e[0] == '0');
+}
+
 static int run_ffn_half(spa_layer* L, const void* H, const int32_t* idx, int tps,
                         const spa_layer_cache* c, cudaStream_t s, const void* Ob, const CUtensorMap* tmOb,
                         void* row_copy, float* score_zero) {
@@ -1082,8 +1096,15 @@ static int run_ffn_half(spa_layer* L, const void* H, const int32_t* idx, int tps
       TcWsParams p;
       std::memset(&p, 0, sizeof(p));
       p.tmW[0] = L->tm_wo; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
+      if (norm_fold_enabled()) {
+        // the FFN RMSNorm folded in: x2 = gamma * H1 and the rows' partial sums of squares
+        p.ep.gamma = L->w.ffn_norm;
+        p.ep.x2 = ws->X2;
+        p.ep.ss_part = ws->ss_part;
+        p.ep.ss_tiles = (d + 127) / 128;
+      }
       SPA_TRY(run_ws(EPI_RESID, false, p, Ob, M, d, d, s, prof,
-                     Work{SPA_PROF_OPROJ, (double)d * d * es + 3.0 * Md * es, 2.0 * Md * d}));
+                     Work{SPA_PROF_OPROJ, (double)d * d * es + 4.0 * Md * es + d * es, 2.0 * Md * d + 3.0 * Md}));
     } else if (bf) {
       TcGemmParams p;
       std::memset(&p, 0, sizeof(p));
@@ -1101,8 +1122,11 @@ static int run_ffn_half(spa_layer* L, const void* H, const int32_t* idx, int tps
                        Work{SPA_PROF_OPROJ, (double)d * d * es + 3.0 * Md * es, 2.0 * Md * d}));
     }
   }
-  // x2 = RMSNorm(H1) (the stream-K O-proj's reduce kernel wrote it already)
-  if (!(bf && M <= 256 && streamk_enabled())) {
+  // x2 = RMSNorm(H1) (the stream-K O-proj's reduce kernel wrote it already;
+  // the weight-stationary GEMMs fold it into their epilogues)
+  const bool ws_path = bf && M <= 256 && !streamk_enabled();
+  const bool fold = ws_path && norm_fold_enabled();
+  if (!(bf && M <= 256) || (ws_path && !fold)) {
     {
       ProfScope ps(prof, SPA_PROF_NORM, 2.0 * Md * es + d * es, 4.0 * Md, s);
       e = launch_rmsnorm_rows(D.dtype, ws->H1, 0, nullptr, tps, N, M, d, L->w.ffn_norm, D.rms_eps, ws->X2, ws->err, s);
@@ -1120,10 +1144,15 @@ static int run_ffn_half(spa_layer* L, const void* H, const int32_t* idx, int tps
       p.tmW[0] = L->tm_wg64; p.tmW[1] = L->tm_wu64; p.b_mode = B_GATEUP; p.b_rows_per_src = F; p.ep = ep;
       SPA_TRY(run_sk(EPI_SWIGLU, p, ws, ws->X2, M, d, F / 64, s, prof,
                      Work{SPA_PROF_GATEUP, 2.0 * F * d * es + Md * es + (double)M * F * es, 4.0 * Md * F}));
-    } else if (bf && M <= 256) {
+    } else if (ws_path) {
       TcWsParams p;
       std::memset(&p, 0, sizeof(p));
       p.tmW[0] = L->tm_wg; p.tmW[1] = L->tm_wu; p.b_mode = B_GATEUP; p.b_rows_per_src = F; p.ep = ep;
+      if (fold) {  // x2 holds gamma * H1: each token's 1 / rms(H1) scales its accumulators
+        p.ep.ss_part = ws->ss_part;
+        p.ep.ss_tiles = (d + 127) / 128;
+        p.ep.eps = D.rms_eps;
+      }
       SPA_TRY(run_ws(EPI_SWIGLU, true, p, ws->X2, M, d, F, s, prof,
                      Work{SPA_PROF_GATEUP, 2.0 * F * d * es + Md * es + (double)M * F * es, 4.0 * Md * F}));
     } else if (bf) {

@@ -49,7 +49,7 @@ constexpr int kFfSmem = kFfRing + kFfTableBytes + 1024;
 constexpr int kFfRed = 192;         // reducer threads
 constexpr int kFfJobs = 4;          // feature groups summed per reducer thread at once
 
-__device__ __forceinline__ float ff_silu(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
+__device__ __forceinline__ float ff_silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 __host__ __device__ __forceinline__ int ff_start(int g, int G, int U) { return (int)(((long long)g * U) / G); }
 __host__ __device__ __forceinline__ int ff_owner(int u, int G, int U) {

@@ -32,10 +32,12 @@ namespace spa {
 // ---------------------------------------------------------------------------
 constexpr int kUnroll = 8;
 
-// silu(g) = g / (1 + e^-g) with the fast exponential intrinsic and a
-// correctly rounded reciprocal: relative error ~1e-6, far below the bf16
-// rounding of the result.
-__device__ __forceinline__ float silu(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
+// silu(g) = g / (1 + e^-g) with the fast exponential and fast divide
+// intrinsics: relative error a few 1e-7, far below the bf16 rounding of the
+// result; for g below about -88, e^-g overflows and the quotient is -0, the
+// limit of silu.  (A correctly rounded reciprocal here cost ~4 us per gate/up
+// launch: its slow path serialises the epilogue's 64 silu per thread.)
+__device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 // s_rows[row] = (sequence b, cache row) of token t = gm0 + row; (0, -1) when
 // t >= M or the index is out of range (the latter is reported).
@@ -59,7 +61,7 @@ __device__ void stage_rows(const EpiParams& ep, int gm0, int row_begin, int row_
 template <int MODE, int BN, typename T>
 __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_end, int gm0,
                              int n_tile, const EpiParams& ep, const int2* s_rows, int tid,
-                             int nthr) {
+                             int nthr, const float* s_scale = nullptr) {
   const int nrows = row_end - row_begin;
   if (nrows <= 0) return;
 
@@ -108,6 +110,30 @@ __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_e
           }
         }
       }
+      if constexpr (MODE == EPI_RESID && BN == 128 && sizeof(T) == 2) {
+        // the FFN RMSNorm, folded: a warp holds one row's 128 features (32
+        // float4 items), so its sum of squares is a warp sum in a fixed order
+        if (ep.x2 != nullptr) {
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u) {
+            const int t = gm0 + row[u], gn = gn0 + c[u];
+            float ss = 0.f;
+            if (ok[u]) {
+              float4 q = v[u];
+              q.x += h[u].x; q.y += h[u].y; q.z += h[u].z; q.w += h[u].w;
+              // H1 as stored (bf16), times gamma
+              q.x = __bfloat162float(__float2bfloat16_rn(q.x)); q.y = __bfloat162float(__float2bfloat16_rn(q.y));
+              q.z = __bfloat162float(__float2bfloat16_rn(q.z)); q.w = __bfloat162float(__float2bfloat16_rn(q.w));
+              ss = q.x * q.x + q.y * q.y + q.z * q.z + q.w * q.w;
+              const float4 gm = load4(reinterpret_cast<const T*>(ep.gamma) + gn);
+              store4(reinterpret_cast<T*>(ep.x2) + (size_t)t * ep.d + gn,
+                     make_float4(q.x * gm.x, q.y * gm.y, q.z * gm.z, q.w * gm.w));
+            }
+            ss = warp_sum(ss);  // every lane of the warp runs the same items
+            if ((tid & 31) == 0 && ok[u]) ep.ss_part[(size_t)t * ep.ss_tiles + n_tile] = ss;
+          }
+        }
+      }
     }
   } else if constexpr (MODE == EPI_SWIGLU) {
     constexpr int HALF = BN / 2, C4 = HALF / 4;
@@ -116,8 +142,13 @@ __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_e
       const int row = row_begin + it / C4, c = (it % C4) * 4;
       const int t = gm0 + row, f = f0 + c;
       if (t >= ep.M || f >= ep.n_out) continue;
-      const float4 g = *reinterpret_cast<const float4*>(tile + row * ld + c);
-      const float4 u = *reinterpret_cast<const float4*>(tile + row * ld + HALF + c);
+      float4 g = *reinterpret_cast<const float4*>(tile + row * ld + c);
+      float4 u = *reinterpret_cast<const float4*>(tile + row * ld + HALF + c);
+      if (s_scale != nullptr) {  // the folded FFN RMSNorm of token t
+        const float sc = s_scale[row];
+        g.x *= sc; g.y *= sc; g.z *= sc; g.w *= sc;
+        u.x *= sc; u.y *= sc; u.z *= sc; u.w *= sc;
+      }
       const float4 a = make_float4(silu(g.x) * u.x, silu(g.y) * u.y, silu(g.z) * u.z, silu(g.w) * u.w);
       store4(reinterpret_cast<T*>(ep.out) + (size_t)t * ep.n_out + f, a);
     }
@@ -593,6 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ int2 s_rows[256];  // >= CHUNK
+  __shared__ float s_scale[MODE == EPI_SWIGLU ? 256 : 1];  // the folded FFN RMSNorm, per token
 
   griddep_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -684,6 +716,25 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
     // idle during the main loop: fetch the first chunk's row indices now
     griddep_wait();
     stage_rows(p.ep, 0, 0, min(CHUNK, NT), s_rows, threadIdx.x - 64, kThreads - 64);
+    if constexpr (MODE == EPI_SWIGLU) {
+      // and the per-token scale of the folded FFN RMSNorm: 1 / sqrt(mean(H1^2)
+      // + eps), the tiles' partial sums added in tile order
+      if (p.ep.ss_part != nullptr)
+        for (int t = threadIdx.x - 64; t < NT; t += kThreads - 64) {
+          float tot = 0.f;
+          if (t < p.ep.M) {
+            const float* sp = p.ep.ss_part + (size_t)t * p.ep.ss_tiles;
+            for (int j0 = 0; j0 < p.ep.ss_tiles; j0 += 8) {
+              float v[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) v[j] = j0 + j < p.ep.ss_tiles ? sp[j0 + j] : 0.f;
+#pragma unroll
+              for (int j = 0; j < 8; ++j) tot += v[j];
+            }
+          }
+          s_scale[t] = 1.0f / sqrtf(tot / (float)p.ep.d + p.ep.eps);
+        }
+    }
   }
   __syncwarp();
 
@@ -711,6 +762,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
           float g[32], u[32];
           tmem_ld32(row_base + (uint32_t)c, g);
           tmem_ld32(row_base + (uint32_t)(NT + c), u);
+          if (p.ep.ss_part != nullptr) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              g[j] *= s_scale[c + j];
+              u[j] *= s_scale[c + j];
+            }
+          }
           if (f < p.ep.n_out) {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
@@ -762,8 +820,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
         stage_rows(p.ep, c0, r0, r1, s_rows, threadIdx.x, kThreads);
         __syncthreads();
       }
-      run_epilogue<MODE, FEAT, __nv_bfloat16>(tile, LD, r0, r1, c0, n_tile, p.ep, s_rows,
-                                              threadIdx.x, kThreads);
+      run_epilogue<MODE, FEAT, __nv_bfloat16>(tile, LD, r0, r1, c0, n_tile, p.ep, s_rows, threadIdx.x, kThreads,
+                                              (MODE == EPI_SWIGLU && p.ep.ss_part) ? s_scale + c0 : nullptr);
     }
     __syncthreads();
   }

@@ -59,6 +59,16 @@ struct EpiParams {
   int32_t* amax_idx;
   float* amax_sum;     // ARGMAX: sum over the tile of exp(logit - tile max) [M, n_tiles], or null
   int n_tiles;
+  // The FFN RMSNorm folded into the GEMMs around it (weight-stationary path):
+  // RESID (128-feature tiles) also writes x2[t] = gamma * H1[t] (bf16) and
+  // ss_part[t * ss_tiles + tile] = the sum of H1[t]^2 over the tile's
+  // features; SWIGLU scales both accumulators of token t by 1 / sqrt(sum over
+  // tiles of ss_part[t] / d + eps) before silu(g) * u.  Null: not folded.
+  const void* gamma;
+  void* x2;
+  float* ss_part;
+  int ss_tiles;
+  float eps;
   int* err;            // device error word
 };
 

@@ -61,7 +61,7 @@ constexpr int kRedMaxSeg = 8;     // segments per tile (the host keeps the grid 
 constexpr int kRedJobs = 4;       // feature groups summed per thread at once (all their loads in flight)
 constexpr int kRedMaxTiles = 256;
 
-__device__ __forceinline__ float sk_silu(float g) { return g * __frcp_rn(1.0f + __expf(-g)); }
+__device__ __forceinline__ float sk_silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 // First unit of CTA g of G over U units.
 __host__ __device__ __forceinline__ int sk_start(int g, int G, int U) {
