@@ -715,13 +715,25 @@ struct Work {
   double bytes, flops;
 };
 
+// Tiled tcgen05 GEMM over M token rows.  With KB (the k-blocks of 64) given,
+// a layer GEMM of at least 512 rows takes 256-row tiles (twice the MMA work
+// per staged byte) and its split-K is re-planned for the halved tile count;
+// SPA_TC_BM=128 keeps 128-row tiles (tuning override).
 static int run_tc(int mode, int BN, TcGemmParams& p, int M, int n_tiles, int splits, cudaStream_t s,
-                  Profiler* prof, Work w) {
-  const int m_tiles = (M + 127) / 128;
+                  Profiler* prof, Work w, int KB = 0, int sms = 148) {
+  int BM = 128;
+  if (KB > 0 && BN == 256 && M >= 512 &&
+      (mode == EPI_STORE || mode == EPI_QKV || mode == EPI_RESID || mode == EPI_SWIGLU ||
+       mode == EPI_RESID_SCATTER)) {
+    const char* env = std::getenv("SPA_TC_BM");
+    if (!(env && std::atoi(env) == 128)) BM = 256;
+  }
+  const int m_tiles = (M + BM - 1) / BM;
   if (m_tiles == 0) return SPA_OK;
+  if (BM == 256) splits = choose_splits(n_tiles * m_tiles, KB, sms);
   ProfScope ps(prof, w.cls, w.bytes, w.flops, s);
   if (m_tiles > 65535 || n_tiles > 65535) return fail(SPA_ERR_SHAPE, "GEMM grid too large");
-  cudaError_t e = launch_tc_gemm(mode, BN, p, m_tiles, n_tiles, splits, s);
+  cudaError_t e = launch_tc_gemm(mode, BN, BM, p, m_tiles, n_tiles, splits, s);
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "tc GEMM launch (mode %d): %s", mode, cudaGetErrorString(e));
   return SPA_OK;
 }
@@ -972,7 +984,7 @@ static int run_attn_half(spa_layer* L, const void* H, const int32_t* idx, int tp
       p.K = d; p.b_mode = B_CONCAT3; p.b_rows_per_src = d; p.ep = ep;
       const int nt = 3 * d / 256, mt = (M + 127) / 128;
       SPA_TRY(run_tc(EPI_QKV, 256, p, M, nt, choose_splits(nt * mt, d / 64, ws->num_sms), s, prof,
-                     Work{SPA_PROF_QKV, 3.0 * d * d * es + Md * es + 3.0 * Md * es, 6.0 * Md * d}));
+                     Work{SPA_PROF_QKV, 3.0 * d * d * es + Md * es + 3.0 * Md * es, 6.0 * Md * d}, d / 64, ws->num_sms));
     } else {
       SimtGemmParams p;
       std::memset(&p, 0, sizeof(p));
@@ -1112,7 +1124,7 @@ static int run_ffn_half(spa_layer* L, const void* H, const int32_t* idx, int tps
       p.K = d; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
       const int nt = d / 256, mt = (M + 127) / 128;
       SPA_TRY(run_tc(EPI_RESID, 256, p, M, nt, choose_splits(nt * mt, d / 64, ws->num_sms), s, prof,
-                     Work{SPA_PROF_OPROJ, (double)d * d * es + 3.0 * Md * es, 2.0 * Md * d}));
+                     Work{SPA_PROF_OPROJ, (double)d * d * es + 3.0 * Md * es, 2.0 * Md * d}, d / 64, ws->num_sms));
     } else {
       SimtGemmParams p;
       std::memset(&p, 0, sizeof(p));
@@ -1162,7 +1174,7 @@ static int run_ffn_half(spa_layer* L, const void* H, const int32_t* idx, int tps
       p.K = d; p.b_mode = B_GATEUP; p.b_rows_per_src = F; p.ep = ep;
       const int nt = F / 128, mt = (M + 127) / 128;
       SPA_TRY(run_tc(EPI_SWIGLU, 256, p, M, nt, choose_splits(nt * mt, d / 64, ws->num_sms), s, prof,
-                     Work{SPA_PROF_GATEUP, 2.0 * F * d * es + Md * es + (double)M * F * es, 4.0 * Md * F}));
+                     Work{SPA_PROF_GATEUP, 2.0 * F * d * es + Md * es + (double)M * F * es, 4.0 * Md * F}, d / 64, ws->num_sms));
     } else {
       SimtGemmParams p;
       std::memset(&p, 0, sizeof(p));
@@ -1199,7 +1211,7 @@ static int run_ffn_half(spa_layer* L, const void* H, const int32_t* idx, int tps
       p.K = F; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
       const int nt = d / 256, mt = (M + 127) / 128;
       SPA_TRY(run_tc(EPI_RESID_SCATTER, 256, p, M, nt, choose_splits(nt * mt, F / 64, ws->num_sms), s, prof,
-                     Work{SPA_PROF_DOWN, (double)d * F * es + (double)M * F * es + 2.0 * Md * es, 2.0 * Md * F}));
+                     Work{SPA_PROF_DOWN, (double)d * F * es + (double)M * F * es + 2.0 * Md * es, 2.0 * Md * F}, F / 64, ws->num_sms));
     } else {
       SimtGemmParams p;
       std::memset(&p, 0, sizeof(p));

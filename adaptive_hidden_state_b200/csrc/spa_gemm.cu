@@ -376,17 +376,25 @@ __device__ __forceinline__ void b_source(const TcGemmParams& p, int n_tile, int 
 constexpr int kTcABytes = 128 * 128;  // 128 rows x 64 bf16
 constexpr int kThreads = 256;         // 8 warps: producer, MMA issuer, all 8 in the epilogue
 
-__host__ __device__ constexpr int tc_stages(int BN) { return BN == 256 ? 4 : 3; }
-__host__ __device__ constexpr int tc_smem_bytes(int BN) {
-  return tc_stages(BN) * (kTcABytes + BN * 128) + 1024;
+// BM = 256 (two 128-row A boxes and two TMEM accumulators of 128 x 256 per
+// CTA) doubles the MMA work per byte staged: a 64-column k-block moves 64 KB
+// through the ring for 2 x 128 x 256 x 64 MACs instead of 48 KB for half of
+// that, which lifts the TMA-fill-bound rate of a CTA (one per SM: it holds
+// tensor memory) by ~1.5x.  The epilogue runs the two 128-row halves in turn.
+__host__ __device__ constexpr int tc_stages(int BN, int BM = 128) { return BM == 256 ? 3 : BN == 256 ? 4 : 3; }
+__host__ __device__ constexpr int tc_smem_bytes(int BN, int BM = 128) {
+  return tc_stages(BN, BM) * ((BM / 128) * kTcABytes + BN * 128) + 1024;
 }
 
-template <int MODE, int BN>
+template <int MODE, int BN, int BM>
 __global__ void __launch_bounds__(kThreads, BN == 128 ? 2 : 1) tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
-  constexpr int STAGES = tc_stages(BN);
+  constexpr int STAGES = tc_stages(BN, BM);
+  constexpr int NA = BM / 128;  // A boxes (and accumulators) per stage
+  constexpr int A_BYTES = NA * kTcABytes;
   constexpr int B_BYTES = BN * 128;
-  constexpr int STAGE_BYTES = kTcABytes + B_BYTES;
+  constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   constexpr int LD = BN + 4;
+  static_assert(BM == 128 || (BM == 256 && BN == 256), "256-row tiles take 256 columns");
   static_assert(128 * LD * 4 <= STAGES * STAGE_BYTES, "epilogue tile must fit the ring");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -418,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, BN == 128 ? 2 : 1) tc_gemm_kernel(co
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(&tmem_slot, BN);
+    tmem_alloc(&tmem_slot, NA * BN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -434,10 +442,11 @@ __global__ void __launch_bounds__(kThreads, BN == 128 ? 2 : 1) tc_gemm_kernel(co
       if (it >= STAGES && !mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1, &abort_flag, err, 201))
         break;
       uint8_t* sa = smem + s * STAGE_BYTES;
-      uint8_t* sb = sa + kTcABytes;
+      uint8_t* sb = sa + A_BYTES;
       mbar_arrive_expect_tx(&full_bar[s], STAGE_BYTES);
       const int kx = (kb0 + it) * 64;
-      tma_load_2d(sa, &p.tmA, &full_bar[s], kx, m_tile * 128);
+#pragma unroll
+      for (int a = 0; a < NA; ++a) tma_load_2d(sa + a * kTcABytes, &p.tmA, &full_bar[s], kx, m_tile * BM + a * 128);
 #pragma unroll
       for (int h = 0; h < BN / 128; ++h) {
         int src, row;
@@ -452,11 +461,14 @@ __global__ void __launch_bounds__(kThreads, BN == 128 ? 2 : 1) tc_gemm_kernel(co
       if (!mbar_wait(&full_bar[s], (it / STAGES) & 1, &abort_flag, err, 202)) break;
       tc_fence_after();
       const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
-      const uint64_t da = smem_desc_sw128(sa);
-      const uint64_t db = smem_desc_sw128(sa + kTcABytes);
+      const uint64_t db = smem_desc_sw128(sa + A_BYTES);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        umma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+      for (int a = 0; a < NA; ++a) {
+        const uint64_t da = smem_desc_sw128(sa + a * kTcABytes);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16(tmem + (uint32_t)(a * BN), da + 2 * kk, db + 2 * kk, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+      }
       umma_commit(&empty_bar[s]);
     }
     umma_commit(&accum_bar);
@@ -469,50 +481,56 @@ __global__ void __launch_bounds__(kThreads, BN == 128 ? 2 : 1) tc_gemm_kernel(co
   tc_fence_after();
 
   float* tile = reinterpret_cast<float*>(smem);
-  if (good) {
-    const int q = warp & 3, half = warp >> 2;
-    float* dst = tile + (q * 32 + lane) * LD;
 #pragma unroll 1
-    for (int c = 32 * half; c < BN; c += 64) {
-      float v[32];
-      if (nk > 0) {
-        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
-      } else {
+  for (int a = 0; a < NA; ++a) {
+    // the a-th 128-row half of the tile: accumulator -> shared memory, split-K
+    // reduction across the cluster, epilogue
+    if (a > 0) __syncthreads();  // the previous half's epilogue is done with the tile
+    if (good) {
+      const int q = warp & 3, half = warp >> 2;
+      float* dst = tile + (q * 32 + lane) * LD;
+#pragma unroll 1
+      for (int c = 32 * half; c < BN; c += 64) {
+        float v[32];
+        if (nk > 0) {
+          tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * BN + c), v);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = 0.f;
+          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(dst + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
       }
-#pragma unroll
-      for (int j = 0; j < 32; j += 4)
-        *reinterpret_cast<float4*>(dst + c + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
     }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, BN);
-
-  const int gm0 = m_tile * 128;
-  int r0 = 0, r1 = 128;
-  if (S > 1) {
-    cluster_sync();
-    const int q = (int)cluster_ctarank();
-    r0 = (q * 128) / S;
-    r1 = ((q + 1) * 128) / S;
-    if (good) cluster_reduce_rows<BN>(tile, LD, r0, r1, S, threadIdx.x, kThreads);
-    cluster_sync();
-  }
-  if (good) {
-    stage_rows(p.ep, gm0, r0, r1, s_rows, threadIdx.x, kThreads);
+    tc_fence_before();
     __syncthreads();
-    run_epilogue<MODE, BN, __nv_bfloat16>(tile, LD, r0, r1, gm0, n_tile, p.ep, s_rows, threadIdx.x,
-                                          kThreads);
+    if (a == NA - 1 && warp == 0) tmem_dealloc(tmem, NA * BN);
+
+    const int gm0 = m_tile * BM + a * 128;
+    int r0 = 0, r1 = 128;
+    if (S > 1) {
+      cluster_sync();
+      const int q = (int)cluster_ctarank();
+      r0 = (q * 128) / S;
+      r1 = ((q + 1) * 128) / S;
+      if (good) cluster_reduce_rows<BN>(tile, LD, r0, r1, S, threadIdx.x, kThreads);
+      cluster_sync();
+    }
+    if (good) {
+      stage_rows(p.ep, gm0, r0, r1, s_rows, threadIdx.x, kThreads);
+      __syncthreads();
+      run_epilogue<MODE, BN, __nv_bfloat16>(tile, LD, r0, r1, gm0, n_tile, p.ep, s_rows, threadIdx.x,
+                                            kThreads);
+    }
   }
 }
 
-template <int MODE, int BN>
+template <int MODE, int BN, int BM>
 static cudaError_t launch_tc_typed(const TcGemmParams& p, int m_tiles, int n_tiles, int splits,
                                    cudaStream_t stream) {
-  auto kern = tc_gemm_kernel<MODE, BN>;
-  const int smem = tc_smem_bytes(BN);
+  auto kern = tc_gemm_kernel<MODE, BN, BM>;
+  const int smem = tc_smem_bytes(BN, BM);
   cudaError_t ec = configure_kernel((const void*)kern, smem, true);
   if (ec != cudaSuccess) return ec;
   cudaLaunchConfig_t cfg = {};
@@ -532,10 +550,22 @@ static cudaError_t launch_tc_typed(const TcGemmParams& p, int m_tiles, int n_til
   return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
-cudaError_t launch_tc_gemm(int mode, int BN, const TcGemmParams& p, int m_tiles, int n_tiles,
+cudaError_t launch_tc_gemm(int mode, int BN, int BM, const TcGemmParams& p, int m_tiles, int n_tiles,
                            int splits, cudaStream_t stream) {
+  if (BM == 256) {
+#define SPA_TC_CASE(M_)                                                                               \
+  if (mode == M_ && BN == 256) return launch_tc_typed<M_, 256, 256>(p, m_tiles, n_tiles, splits, stream);
+    SPA_TC_CASE(EPI_STORE)
+    SPA_TC_CASE(EPI_QKV)
+    SPA_TC_CASE(EPI_RESID)
+    SPA_TC_CASE(EPI_SWIGLU)
+    SPA_TC_CASE(EPI_RESID_SCATTER)
+#undef SPA_TC_CASE
+    return cudaErrorInvalidValue;
+  }
+  if (BM != 128) return cudaErrorInvalidValue;
 #define SPA_TC_CASE(M_, BN_)                                           \
-  if (mode == M_ && BN == BN_) return launch_tc_typed<M_, BN_>(p, m_tiles, n_tiles, splits, stream);
+  if (mode == M_ && BN == BN_) return launch_tc_typed<M_, BN_, 128>(p, m_tiles, n_tiles, splits, stream);
   SPA_TC_CASE(EPI_STORE, 128)
   SPA_TC_CASE(EPI_STORE, 256)
   SPA_TC_CASE(EPI_QKV, 256)

@@ -157,7 +157,9 @@ struct SimtGemmParams {
 // tcgen05 GEMM: D[M, n] = A[M, K] . B[n, K]^T, BM = 128, BN = 128 or 256,
 // split-K across a thread-block cluster of `splits` CTAs with a fixed-order
 // reduction through distributed shared memory.
-cudaError_t launch_tc_gemm(int mode, int BN, const TcGemmParams& p, int m_tiles, int n_tiles,
+// Tiled tcgen05 GEMM: BM x BN tiles (BM = 128, or 256 with BN = 256 for the
+// layer GEMMs' epilogues), split-K across a cluster of `splits` CTAs.
+cudaError_t launch_tc_gemm(int mode, int BN, int BM, const TcGemmParams& p, int m_tiles, int n_tiles,
                            int splits, cudaStream_t stream);
 // Weight-stationary tcgen05 GEMM for M <= 256 tokens: 128 weight rows per
 // CTA (NACC = 2: gate and up rows) against all tokens; same epilogues.

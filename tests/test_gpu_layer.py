@@ -134,6 +134,23 @@ def test_bf16_small_layer_shapes(B, N, k):
     _step(lp, cache, ocs, H2, k)
 
 
+@pytest.mark.parametrize("bm", ["", "128"])
+@pytest.mark.parametrize("B,N,k", [(1, 600, 600), (2, 300, 300), (1, 1030, 520), (2, 520, 40)])
+def test_bf16_tiled_gemm_row_tiles(monkeypatch, bm, B, N, k):
+    # the tiled GEMMs of the rho = 1 fill and of cached steps with more than 256
+    # tokens: 256-row tiles (two TMEM accumulators, the epilogue in two halves)
+    # for M >= 512, including ragged last tiles (M = 600, 1030, 1040) and the
+    # split-K the planner picks for them, against 128-row tiles (SPA_TC_BM=128)
+    if bm:
+        monkeypatch.setenv("SPA_TC_BM", bm)
+    lp = LayerPair(spa, SMALL_BF16, seed=20 + N + k, dtype=spa.SPA_BF16, max_B=B, max_N=N, std=0.05)
+    H = synth.hidden_states(B, N, 256, seed=N + 3, bf16=True)
+    cache, ocs = _run_fill(lp, H)
+    _compare_cache(lp, cache, ocs, "fill")
+    H2, _ = synth.drift_rows(H, 0.2, 0.5, seed=N + 4, bf16=True)
+    _step(lp, cache, ocs, H2, k)
+
+
 @pytest.mark.parametrize("nacc", ["2", "4"])
 @pytest.mark.parametrize("B,N,k", [(1, 200, 96), (2, 160, 33)])
 def test_bf16_wide_weight_tiles(monkeypatch, nacc, B, N, k):
