@@ -8,6 +8,7 @@
 // attn_simt_kernel: one warp per (query, head), online softmax over chunks of
 // 32 keys (one key per lane), fp32 throughout.  Used for the fp32
 // configurations and for head sizes the tensor-core kernel does not cover.
+#include <cstdlib>
 #include <cstring>
 
 #include "spa_device.cuh"
@@ -620,8 +621,13 @@ cudaError_t launch_attention(int dtype, const void* Q, const void* Kc, const voi
     int splits = 1;
     if (allow_cluster) {
       // split the keys while every cluster of the grid is resident at once and
-      // each split keeps >= 2 key tiles
-      while (splits < 8 && n_kt >= splits * 4 && groups <= attn_max_clusters(splits * 2)) splits *= 2;
+      // each split keeps >= 1 key tile (one tile per CTA measured fastest at
+      // N = 512: 16.9 against 18.8 us with two)
+      while (splits < 8 && n_kt >= splits * 2 && groups <= attn_max_clusters(splits * 2)) splits *= 2;
+      if (const char* env = std::getenv("SPA_ATTN_SPLITS")) {  // tuning override: 1, 2, 4 or 8 key splits
+        const int v = std::atoi(env);
+        if ((v == 1 || v == 2 || v == 4 || v == 8) && v <= n_kt) splits = v;
+      }
     } else {
       // split the keys while the grid is small, each split keeps >= 2 key tiles
       while (splits < 8 && groups * splits * 2 <= 160 && n_kt >= splits * 4 &&

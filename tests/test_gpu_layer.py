@@ -203,10 +203,11 @@ def test_bf16_persistent_ffn(monkeypatch, grid, B, N, k):
 
 @pytest.mark.parametrize("B,N,k", [(1, 2048, 200), (2, 1000, 62), (1, 1536, 129), (1, 3000, 200)])
 def test_bf16_split_key_attention(B, N, k):
-    # long caches: the keys of each query tile are split over a cluster of 8,
-    # 4, 4 and 8 CTAs (2, 2, 3 and 3 key tiles each; N=1000 and N=3000 end in
-    # a partial key tile), with one or two query tiles, the second holding 72
-    # or 1 rows.  N=3000 also takes the unfused select (more than 2048 scores).
+    # long caches: the keys of each query tile are split over a cluster of 8
+    # CTAs (2, 1, 1-2 and 3 key tiles each; N=1000 and N=3000 end in a partial
+    # key tile), with one or two query tiles, the second holding 72 or 1 rows
+    # (the LLaDA-shaped layer tests take 4-way and 2-way clusters).  N=3000 also
+    # takes the unfused select (more than 2048 scores).
     lp = LayerPair(spa, SMALL_BF16, seed=50 + k, dtype=spa.SPA_BF16, max_B=B, max_N=N, std=0.05)
     H = synth.hidden_states(B, N, 256, seed=k + 7, bf16=True)
     cache, ocs = _run_fill(lp, H)
