@@ -151,6 +151,18 @@ def test_bf16_tiled_gemm_row_tiles(monkeypatch, bm, B, N, k):
     _step(lp, cache, ocs, H2, k)
 
 
+@pytest.mark.parametrize("B,N,k", [(1, 200, 96), (2, 300, 129)])
+def test_bf16_separate_ffn_norm(monkeypatch, B, N, k):
+    # the FFN RMSNorm as its own kernel (SPA_NORM_FOLD=0) instead of folded into
+    # the O-proj and gate/up epilogues of the weight-stationary path
+    monkeypatch.setenv("SPA_NORM_FOLD", "0")
+    lp = LayerPair(spa, SMALL_BF16, seed=60 + k, dtype=spa.SPA_BF16, max_B=2, max_N=300, std=0.05)
+    H = synth.hidden_states(B, N, 256, seed=k + 11, bf16=True)
+    cache, ocs = _run_fill(lp, H)
+    H2, _ = synth.drift_rows(H, 0.2, 0.5, seed=k + 12, bf16=True)
+    _step(lp, cache, ocs, H2, k)
+
+
 @pytest.mark.parametrize("nacc", ["2", "4"])
 @pytest.mark.parametrize("B,N,k", [(1, 200, 96), (2, 160, 33)])
 def test_bf16_wide_weight_tiles(monkeypatch, nacc, B, N, k):
