@@ -151,7 +151,7 @@ def test_bf16_tiled_gemm_row_tiles(monkeypatch, bm, B, N, k):
     _step(lp, cache, ocs, H2, k)
 
 
-@pytest.mark.parametrize("B,N,k", [(1, 200, 96), (2, 300, 129)])
+@pytest.mark.parametrize("B,N,k", [(1, 200, 96), (2, 300, 100)])
 def test_bf16_separate_ffn_norm(monkeypatch, B, N, k):
     # the FFN RMSNorm as its own kernel (SPA_NORM_FOLD=0) instead of folded into
     # the O-proj and gate/up epilogues of the weight-stationary path
