@@ -844,6 +844,16 @@ def main():
     barrier()
     v_ms = max_over_ranks(dist, world, v0.elapsed_time(v1), "cuda") / vk
     ws.check()
+    # its roofline: the algorithmic bytes and flops of one profiled rho = 1 step
+    ws.profile_enable(True)
+    ws.profile_read()
+    spa.spa_decode_step(model, pos_dev[1], None, u, 2, tok_out[1])
+    vprof = ws.profile_read()
+    ws.profile_enable(False)
+    ws.check()
+    v_b = sum(vprof[k][2] for k in PROF_CLASSES)
+    v_f = sum(vprof[k][3] for k in PROF_CLASSES)
+    v_roof_ms = max(v_b / (hbm * 1e9), v_f / (tf_sus * 1e12)) * 1e3
 
     # ---- the other workloads: single layer, batched long-context decode, sweep
     extra = {}
@@ -888,7 +898,9 @@ def main():
                 "step_roofline_ms": step_roof_ms,
                 "step_roofline_frac": step_roof_ms / ms_step,
                 "vanilla_rho1": {"tokens_per_s": world * B * u / (v_ms / 1e3), "ms_per_step": v_ms,
-                                 "speedup_spa_over_vanilla": v_ms / ms_step},
+                                 "speedup_spa_over_vanilla": v_ms / ms_step,
+                                 "step_roofline_ms": v_roof_ms, "step_roofline_frac": v_roof_ms / v_ms,
+                                 "bound": "tensor" if v_f / (tf_sus * 1e12) > v_b / (hbm * 1e9) else "hbm"},
                 "roofline": roof,
                 "profiled_region": {"ms_per_step": prof_ms_step,
                                     "note": "same steps launched directly with CUDA events "
