@@ -742,20 +742,24 @@ static int run_tc(int mode, int BN, TcGemmParams& p, int M, int n_tiles, int spl
 // token operand (row-major, 16-byte aligned); `rows` weight rows (for
 // gate/up: features, each with a W_gate and a W_up row).  Each CTA keeps NACC
 // accumulators of 128 rows so one token tile feeds up to 512 weight rows
-// (NACC * NT <= 512 TMEM columns); NACC is the largest that still leaves at
-// least 16 tiles to spread over the SMs.
-static int run_ws(int mode, bool gateup, TcWsParams& p, const void* X, int M, int K, int rows,
-                  cudaStream_t s, Profiler* prof, Work w) {
-  if (M <= 0) return SPA_OK;
-  if (M > 256) return fail(SPA_ERR_SHAPE, "weight-stationary GEMM takes at most 256 tokens");
-  const int NT = ((M + 31) / 32) * 32;
-  // Two 128-row blocks per CTA (gate/up: a W_gate and a W_up block) halve
-  // the token-tile traffic per weight byte: each CTA's TMA stream then moves
-  // 48 KB per stage for 32 KB of weights instead of 32 KB for 16 KB, which
-  // lets ~96 CTAs stream near the HBM rate.  A GEMM with fewer rows (O-proj,
-  // down: 32 blocks of 128) keeps one block per CTA so that its split-K
-  // clusters still cover the SMs.  Only a GEMM with many more weight rows
-  // than the SMs can cover (the LM head) takes four.
+// (NACC * NT <= 512 TMEM columns).
+//
+// ws_shape is its plan: NT tokens per MMA, NACC, the column tiles and the
+// split-K cluster size.  Two 128-row blocks per CTA (gate/up: a W_gate and a
+// W_up block) halve the token-tile traffic per weight byte: each CTA's TMA
+// stream then moves 48 KB per stage for 32 KB of weights instead of 32 KB for
+// 16 KB, which lets ~96 CTAs stream near the HBM rate.  A GEMM with fewer rows
+// (O-proj, down: 32 blocks of 128) keeps one block per CTA so that its split-K
+// clusters still cover the SMs.  Only a GEMM with many more weight rows than
+// the SMs can cover (the LM head) takes four.  `fold`: the folded FFN norm
+// sums a row's squares over 128-feature tiles, so one block.
+struct WsShape {
+  int NT, nacc, n_tiles, splits;
+};
+static WsShape ws_shape(int mode, bool gateup, bool fold, int M, int K, int rows) {
+  WsShape sh;
+  sh.NT = ((M + 31) / 32) * 32;
+  const int NT = sh.NT;
   const int min_nacc = gateup ? 2 : 1;
   int nacc = min_nacc;
   if (!gateup && rows % 256 == 0 && rows / 128 >= 64 && 2 * NT <= 512) nacc = 2;
@@ -771,9 +775,24 @@ static int run_ws(int mode, bool gateup, TcWsParams& p, const void* X, int M, in
     const int v = std::atoi(env);
     if ((v == 1 || v == 2 || v == 4) && v >= min_nacc && v * NT <= 512) nacc = v;
   }
-  if (p.ep.x2 != nullptr) nacc = 1;  // the folded FFN norm sums a row's squares over 128-feature tiles
+  if (fold) nacc = 1;
   const int feat = gateup ? nacc / 2 * 128 : nacc * 128;
-  const int n_tiles = (rows + feat - 1) / feat;
+  sh.nacc = nacc;
+  sh.n_tiles = (rows + feat - 1) / feat;
+  sh.splits = plan_ws_splits(mode, nacc, sh.n_tiles, K / 64);
+  if (const char* env = std::getenv("SPA_WS_SPLITS")) {  // tuning override, 1..8
+    const int v = std::atoi(env);
+    if (v >= 1 && v <= 8 && K / 64 >= v) sh.splits = v;
+  }
+  return sh;
+}
+
+static int run_ws(int mode, bool gateup, TcWsParams& p, const void* X, int M, int K, int rows,
+                  cudaStream_t s, Profiler* prof, Work w) {
+  if (M <= 0) return SPA_OK;
+  if (M > 256) return fail(SPA_ERR_SHAPE, "weight-stationary GEMM takes at most 256 tokens");
+  const WsShape sh = ws_shape(mode, gateup, p.ep.x2 != nullptr, M, K, rows);
+  const int NT = sh.NT, nacc = sh.nacc, n_tiles = sh.n_tiles;
   if (encode_bf16_map_box(&p.tmX, X, (uint64_t)M, (uint64_t)K, (uint32_t)NT))
     return fail(SPA_ERR_CUDA, "tensor map for the token operand failed");
   int cols = 32;
@@ -782,13 +801,8 @@ static int run_ws(int mode, bool gateup, TcWsParams& p, const void* X, int M, in
   p.tmem_cols = cols;
   p.K = K;
   if (mode == EPI_ARGMAX) p.ep.n_tiles = n_tiles;
-  int splits = plan_ws_splits(mode, nacc, n_tiles, K / 64);
-  if (const char* env = std::getenv("SPA_WS_SPLITS")) {  // tuning override, 1..8
-    const int v = std::atoi(env);
-    if (v >= 1 && v <= 8 && K / 64 >= v) splits = v;
-  }
   ProfScope ps(prof, w.cls, w.bytes, w.flops, s);
-  cudaError_t e = launch_tc_ws(mode, nacc, p, n_tiles, splits, s);
+  cudaError_t e = launch_tc_ws(mode, nacc, p, n_tiles, sh.splits, s);
   if (e != cudaSuccess) return fail(SPA_ERR_CUDA, "weight-stationary GEMM launch (mode %d): %s", mode, cudaGetErrorString(e));
   return SPA_OK;
 }

@@ -150,6 +150,13 @@ __device__ __forceinline__ void named_bar_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+// Orders this thread's generic-proxy global accesses with async-proxy (TMA)
+// accesses: after writing rows that another CTA's TMA will read (before the
+// release), and after the acquire before issuing such reads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Wait until the global int *flag equals `expect` (acquire: what the writer
 // stored before releasing the flag is visible afterwards).  Gives up after
 // limit_ns and records the error.  Returns true when the flag was seen.

@@ -608,6 +608,19 @@ __host__ __device__ inline int ws_stages(int nacc, int NT) {
   return st < kWsMaxStages ? st : kWsMaxStages;
 }
 
+// A CTA that gave up (a bounded wait ran out) must not release its shared and
+// tensor memory while its copies or tensor-core operations are in flight:
+// thread 0 waits (bounded, ignoring the abort) for the accumulator commit and
+// for every requested stage the MMA did not consume; then all threads proceed.
+__device__ __forceinline__ void ws_drain_on_abort(int abort, uint64_t* accum_bar, uint64_t* full_bar, int stages,
+                                                  int consumed, int issued, int* err) {
+  if (abort && threadIdx.x == 0) {
+    mbar_drain_bounded(accum_bar, 0, err, 215);
+    for (int it = consumed; it < issued; ++it) mbar_drain_bounded(&full_bar[it % stages], (it / stages) & 1, err, 216);
+  }
+  __syncthreads();
+}
+
 // The NACC weight boxes (128 rows x 64 columns each) of one k-block of
 // column tile n_tile: GATEUP -> the first NACC/2 from W_gate, the rest the
 // same rows of W_up; otherwise 128 consecutive rows per accumulator.
@@ -653,6 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
   __shared__ __align__(8) uint64_t accum_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  __shared__ int s_issued, s_consumed;  // stages whose boxes were requested / consumed by the MMA
   __shared__ int2 s_rows[256];  // >= CHUNK
   __shared__ float s_scale[MODE == EPI_SWIGLU ? 256 : 1];  // the folded FFN RMSNorm, per token
 
@@ -679,6 +693,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
     }
     mbar_init(&accum_bar, 1);
     abort_flag = 0;
+    s_issued = 0;
+    s_consumed = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -690,12 +706,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
 
+  // The weights do not depend on earlier kernels: the weight boxes of the
+  // first stages are requested before griddepcontrol.wait, so they stream
+  // while the previous kernel finishes; the token tiles follow the wait.
+  const int pre = nk < STAGES ? nk : STAGES;
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&p.tmX);
-    // The weights do not depend on earlier kernels: the weight boxes of the
-    // first stages are requested before griddepcontrol.wait, so they stream
-    // while the previous kernel finishes; the token tiles follow the wait.
-    const int pre = nk < STAGES ? nk : STAGES;
+    s_issued = pre;
     for (int it = 0; it < pre; ++it) {
       uint8_t* sw = smem + it * STAGE_BYTES;
       mbar_arrive_expect_tx(&full_bar[it], (uint32_t)STAGE_BYTES);
@@ -704,6 +721,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
       const int kx = (kb0 + kit) * 64;
       ws_load_weights<NACC>(p, n_tile, sw, &full_bar[it], kx);
     }
+  }
+  if (warp == 0 && lane == 0) {
     griddep_wait();
     for (int it = 0; it < pre; ++it) {
       int kit = it + rot;
@@ -722,12 +741,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
       const int kx = (kb0 + kit) * 64;
       ws_load_weights<NACC>(p, n_tile, sw, &full_bar[s], kx);
       tma_load_2d(sx, &p.tmX, &full_bar[s], kx, 0);
+      s_issued = it + 1;
     }
   } else if (warp == 1 && lane == 0) {
     const uint32_t idesc = idesc_bf16_f32(128, NT);
     for (int it = 0; it < nk; ++it) {
       const int s = it % STAGES;
       if (!mbar_wait(&full_bar[s], (it / STAGES) & 1, &abort_flag, err, 212)) break;
+      s_consumed = it + 1;
       tc_fence_after();
       const uint32_t sw = smem_u32(smem + s * STAGE_BYTES);
       const uint64_t dx = smem_desc_sw128(sw + W_BYTES);
@@ -808,6 +829,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
       }
       tc_fence_before();
       __syncthreads();
+      ws_drain_on_abort(abort_flag, &accum_bar, full_bar, STAGES, s_consumed, s_issued, err);
       tc_fence_after();
       if (warp == 0) tmem_dealloc(tmem, (uint32_t)p.tmem_cols);
       return;
@@ -855,6 +877,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
     }
     __syncthreads();
   }
+  ws_drain_on_abort(abort_flag, &accum_bar, full_bar, STAGES, s_consumed, s_issued, err);
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, (uint32_t)p.tmem_cols);
 }

@@ -227,7 +227,9 @@ def test_bf16_split_key_attention(B, N, k):
     _step(lp, cache, ocs, H2, k)
 
 
-@pytest.mark.parametrize("bf16,B,N,k", [(False, 2, 64, 16), (True, 2, 1000, 62), (True, 1, 300, 257)])
+@pytest.mark.parametrize("bf16,B,N,k", [(False, 2, 64, 16), (True, 2, 1000, 62), (True, 1, 300, 257),
+                                        (True, 1, 2048, 200), (True, 2, 512, 128), (True, 1, 64, 64),
+                                        (True, 2, 300, 1)])
 def test_layer_step_equals_select_then_partial_block(bf16, B, N, k):
     # spa_layer_step selects, gathers and normalises in one launch; its
     # results must be bit-identical to spa_proxy_select + spa_partial_block
