@@ -240,6 +240,7 @@ struct spa_model {
   bool inc = false;           // incremental proxy enabled
   bool inc_valid = false;     // ahat_all / score_all / chg_rows describe the current state
   int graph_inc = 0;          // the captured step: 0 plain, 1 proxy state refreshed, 2 incremental
+  int graph_kernels = 0;      // kernel nodes of the captured step
   float* ahat_all = nullptr;  // [L, B, N, r]
   float* score_all = nullptr; // [L, B, N]
   void* chg_rows = nullptr;   // [B*N, d] compact changed rows (layer input of the next proxy)
@@ -1691,6 +1692,18 @@ extern "C" int spa_decode_graph_capture(spa_model* m, const int32_t* pos, const 
     return st;
   }
   if (ec != cudaSuccess) return fail(SPA_ERR_CUDA, "stream capture failed: %s", cudaGetErrorString(ec));
+  // count the kernel nodes the step recorded
+  int kernels = 0;
+  size_t n_nodes = 0;
+  if (cudaGraphGetNodes(g, nullptr, &n_nodes) == cudaSuccess && n_nodes > 0) {
+    std::vector<cudaGraphNode_t> nodes(n_nodes);
+    if (cudaGraphGetNodes(g, nodes.data(), &n_nodes) == cudaSuccess)
+      for (size_t i = 0; i < n_nodes; ++i) {
+        cudaGraphNodeType t;
+        if (cudaGraphNodeGetType(nodes[i], &t) == cudaSuccess && t == cudaGraphNodeTypeKernel) ++kernels;
+      }
+  }
+  cudaGetLastError();
   cudaGraphExec_t ex = nullptr;
   const cudaError_t ei = cudaGraphInstantiate(&ex, g, 0);
   cudaGraphDestroy(g);
@@ -1699,7 +1712,13 @@ extern "C" int spa_decode_graph_capture(spa_model* m, const int32_t* pos, const 
   m->graph = ex;
   m->graph_u = u;
   m->graph_inc = variant;
+  m->graph_kernels = kernels;
   return SPA_OK;
+}
+
+extern "C" int spa_decode_graph_kernel_nodes(const spa_model* m) {
+  if (!m) return -1;
+  return m->graph ? m->graph_kernels : 0;
 }
 
 extern "C" int spa_decode_graph_launch(spa_model* m, void* stream) {

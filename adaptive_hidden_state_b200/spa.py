@@ -36,7 +36,7 @@ EXPORTS = [
     "spa_layer_step_attn_identifier",
     "spa_model_create", "spa_model_free", "spa_model_layer_k", "spa_model_index_set", "spa_model_embed",
     "spa_decode_step", "spa_decode_layers", "spa_decode_confidence", "spa_model_write_tokens",
-    "spa_decode_graph_capture", "spa_decode_graph_launch",
+    "spa_decode_graph_capture", "spa_decode_graph_launch", "spa_decode_graph_kernel_nodes",
     "spa_model_set_incremental_proxy", "spa_debug_fail_alloc_after", "spa_debug_bounded_wait",
     "spa_attention_noalloc", "spa_attention_noalloc_status",
 ]
@@ -127,6 +127,7 @@ _sig("spa_decode_confidence", c_int, c_void_p, c_void_p, c_int, c_void_p, c_void
 _sig("spa_model_write_tokens", c_int, c_void_p, c_void_p, c_void_p, c_int, c_void_p)
 _sig("spa_decode_graph_capture", c_int, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p)
 _sig("spa_decode_graph_launch", c_int, c_void_p, c_void_p)
+_sig("spa_decode_graph_kernel_nodes", c_int, c_void_p)
 _sig("spa_attention_noalloc", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_int,
      c_int, c_int, c_void_p)
 _sig("spa_attention_noalloc_status", c_int, c_void_p)
@@ -388,6 +389,10 @@ def spa_decode_graph_capture(model: Model, pos, tok_in, u: int, tok_out, stream=
 
 def spa_decode_graph_launch(model: Model, stream=None):
     _check(lib.spa_decode_graph_launch(model.handle, _stream(stream)), "spa_decode_graph_launch")
+
+
+def spa_decode_graph_kernel_nodes(model: Model) -> int:
+    return lib.spa_decode_graph_kernel_nodes(model.handle)
 
 
 def spa_attention_noalloc(Q, k_cache, v_cache, O, B: int, k: int, N: int, n_heads: int,

@@ -731,9 +731,8 @@ def main():
 
     # capture one cached step into a CUDA graph (fixed pos/tok buffers)
     rewind()
-    n_cap0 = spa.spa_launch_count()
     spa.spa_decode_graph_capture(model, pos_buf, None, u, tok_buf)
-    launches_per_step = spa.spa_launch_count() - n_cap0
+    launches_per_step = spa.spa_decode_graph_kernel_nodes(model)  # the captured step's kernel nodes
     ws.check()
 
     # ---- timed region: K cached decode steps (graph replays), inputs resident in HBM
@@ -768,7 +767,6 @@ def main():
     rewind()
     ws.profile_enable(True)
     ws.profile_read()
-    n0 = spa.spa_launch_count()
     p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     p0.record(stream)
     for t in range(1 + args.warmup, total_steps):

@@ -285,6 +285,10 @@ int spa_model_write_tokens(spa_model *model, const int32_t *pos, const int32_t *
 int spa_decode_graph_capture(spa_model *model, const int32_t *pos, const int32_t *tok_in, int u,
                              int32_t *tok_out, void *stream);
 int spa_decode_graph_launch(spa_model *model, void *stream);
+/* Number of kernel nodes in the captured step's graph (the library kernels
+ * one launch of it runs); 0 when nothing has been captured, -1 for a null
+ * model. */
+int spa_decode_graph_kernel_nodes(const spa_model *model);
 
 /* Incremental proxy (enable = 1; 0 restores the plain path).  Phase 1 of
  * Algorithm 1 ([NOTES] 方法详解 > 整体框架; [GIST] Methodology 1) scores every

@@ -195,7 +195,13 @@ def test_bf16_decode_loop_and_graph_replay(inc):
         pos0 = torch.from_numpy(job.positions[0].astype(np.int32)).cuda()
         f0 = torch.from_numpy(job.forced[0].astype(np.int32)).cuda()
         spa.spa_decode_step(model, pos0, f0, u, 1, tout_buf)
+        n0 = spa.spa_launch_count()
         spa.spa_decode_graph_capture(model, pos_buf, tin_buf, u, tout_buf)
+        # the step's kernels, counted by the library and found in the graph: per layer
+        # proxy, select, QKV, attention, O-proj (+ folded FFN norm), gate/up, down; then
+        # the written tokens' embeddings, the final norm, the LM head and its argmax
+        nodes = spa.spa_decode_graph_kernel_nodes(model)
+        assert nodes == spa.spa_launch_count() - n0 == 7 * 2 + 4
         for t in range(1, steps):
             pos_buf.copy_(torch.from_numpy(job.positions[t].astype(np.int32)).cuda())
             tin_buf.copy_(torch.from_numpy(job.forced[t].astype(np.int32)).cuda())
