@@ -154,56 +154,54 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& t
 // Shared memory of block_select.
 template <int NT>
 struct SelectSmem {
-  unsigned cnt[2][NT / 32][3];
+  unsigned cnt[2][NT / 32];  // per round (double-buffered), per warp: three packed key counts
   int warp_tot[33];
 };
 
 // list[0..k) (and idx_out, when not null) <- the selected indices, ascending.
-template <int NT>
-__device__ void block_select(const float* s, int N, int k, int32_t* list, int32_t* idx_out,
-                             SelectSmem<NT>& sm, int* err) {
+// MAXE (2, 4 or 8) bounds the keys a thread holds (E = ceil(N / NT) <= MAXE);
+// block_select below picks the smallest that fits, so a round compares only
+// the keys there can be.  A round's three counts per thread (<= 8 each) and
+// per warp (<= 256) are packed 10 bits apart into one word, so one warp
+// reduction and one shared word per warp carry all three.
+template <int NT, int MAXE>
+__device__ void block_select_e(const float* s, int N, int k, int32_t* list, int32_t* idx_out,
+                               SelectSmem<NT>& sm, int* err) {
   constexpr int NW = NT / 32;
+  static_assert(MAXE <= kSelMaxPerThread && MAXE * 32 < 1024, "packed counts must not carry");
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int E = (N + NT - 1) / NT;
   const int i0 = tid * E;
-  uint32_t key[kSelMaxPerThread];
+  uint32_t key[MAXE];
 #pragma unroll
-  for (int j = 0; j < kSelMaxPerThread; ++j)
+  for (int j = 0; j < MAXE; ++j)
     key[j] = (j < E && i0 + j < N) ? score_key(s[i0 + j]) : 0u;  // 0 is below every candidate
   uint32_t t = 0;
 #pragma unroll 1
   for (int r = 0; r < 16; ++r) {
     const int shift = 30 - 2 * r;  // bits (31, 30), (29, 28), ..., (1, 0)
     const uint32_t c1 = t | (1u << shift), c2 = t | (2u << shift), c3 = t | (3u << shift);
-    unsigned n1 = 0, n2 = 0, n3 = 0;
+    unsigned packed = 0;
 #pragma unroll
-    for (int j = 0; j < kSelMaxPerThread; ++j) {
-      n1 += key[j] >= c1 ? 1u : 0u;
-      n2 += key[j] >= c2 ? 1u : 0u;
-      n3 += key[j] >= c3 ? 1u : 0u;
-    }
-    n1 = __reduce_add_sync(0xffffffffu, n1);
-    n2 = __reduce_add_sync(0xffffffffu, n2);
-    n3 = __reduce_add_sync(0xffffffffu, n3);
-    if (lane == 0) {
-      sm.cnt[r & 1][wid][0] = n1;
-      sm.cnt[r & 1][wid][1] = n2;
-      sm.cnt[r & 1][wid][2] = n3;
-    }
+    for (int j = 0; j < MAXE; ++j)
+      packed += (key[j] >= c1 ? 1u : 0u) + (key[j] >= c2 ? 1u << 10 : 0u) + (key[j] >= c3 ? 1u << 20 : 0u);
+    packed = __reduce_add_sync(0xffffffffu, packed);
+    if (lane == 0) sm.cnt[r & 1][wid] = packed;
     __syncthreads();  // double-buffered counts: one barrier per round
     unsigned s1 = 0, s2 = 0, s3 = 0;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
-      s1 += sm.cnt[r & 1][w][0];
-      s2 += sm.cnt[r & 1][w][1];
-      s3 += sm.cnt[r & 1][w][2];
+      const unsigned v = sm.cnt[r & 1][w];
+      s1 += v & 1023u;
+      s2 += (v >> 10) & 1023u;
+      s3 += v >> 20;
     }
     const unsigned kk = (unsigned)k;
     t = s3 >= kk ? c3 : s2 >= kk ? c2 : s1 >= kk ? c1 : t;
   }
   int n_gt = 0, n_eq = 0;
 #pragma unroll
-  for (int j = 0; j < kSelMaxPerThread; ++j) {
+  for (int j = 0; j < MAXE; ++j) {
     const bool v = j < E && i0 + j < N;
     n_gt += (v && key[j] > t) ? 1 : 0;
     n_eq += (v && key[j] == t) ? 1 : 0;
@@ -214,7 +212,7 @@ __device__ void block_select(const float* s, int N, int k, int32_t* list, int32_
   if (tid == 0 && (tot >> 16) + min(tot & 0xffff, need) != k) report_error(err, DEVERR_SHAPE, 401);
   int gb = pre >> 16, eb = pre & 0xffff;
 #pragma unroll
-  for (int j = 0; j < kSelMaxPerThread; ++j) {
+  for (int j = 0; j < MAXE; ++j) {
     if (!(j < E && i0 + j < N)) continue;
     int slot = -1;
     if (key[j] > t) {
@@ -231,5 +229,13 @@ __device__ void block_select(const float* s, int N, int k, int32_t* list, int32_
   }
 }
 
+template <int NT>
+__device__ void block_select(const float* s, int N, int k, int32_t* list, int32_t* idx_out,
+                             SelectSmem<NT>& sm, int* err) {
+  const int E = (N + NT - 1) / NT;  // block-uniform
+  if (E <= 2) block_select_e<NT, 2>(s, N, k, list, idx_out, sm, err);
+  else if (E <= 4) block_select_e<NT, 4>(s, N, k, list, idx_out, sm, err);
+  else block_select_e<NT, 8>(s, N, k, list, idx_out, sm, err);
+}
 
 }  // namespace spa
