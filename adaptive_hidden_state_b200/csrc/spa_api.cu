@@ -199,6 +199,9 @@ struct spa_workspace {
   size_t ffn_part_floats = 0;
   int* ffn_sync = nullptr;    // persistent FFN: [8] phase counters
   float* ss_part = nullptr;   // folded FFN RMSNorm: per (token, 128-feature tile) sums of H1^2
+  float* gs_part = nullptr;   // weight-stationary split-K through global memory: the splits' partial tiles
+  size_t gs_part_floats = 0;
+  int* gs_counter = nullptr;  // [2 * kWsCounters] its per-tile arrival and departure counts
   float* rope_cos = nullptr;  // [max_N, hd/2]
   float* rope_sin = nullptr;
   CUtensorMap tmX, tmO, tmX2, tmA;
@@ -487,6 +490,10 @@ extern "C" int spa_workspace_create(const spa_layer_desc* desc, int max_B, int m
     WS_ALLOC(ffn_part, ws->ffn_part_floats * 4)
     WS_ALLOC(ffn_sync, 8 * sizeof(int))
     WS_ALLOC(ss_part, std::min<size_t>(cap, 256) * ((d + 127) / 128) * 4)
+    // one partial tile of at most 512 accumulator columns x 128 rows per SM
+    ws->gs_part_floats = (size_t)ws->num_sms * 512 * 128;
+    WS_ALLOC(gs_part, ws->gs_part_floats * 4)
+    WS_ALLOC(gs_counter, 2 * kWsCounters * sizeof(int))
   }
   WS_ALLOC(rope_cos, (size_t)max_N * (desc->head_dim / 2) * 4)
   WS_ALLOC(rope_sin, (size_t)max_N * (desc->head_dim / 2) * 4)
@@ -509,7 +516,8 @@ extern "C" int spa_workspace_create(const spa_layer_desc* desc, int max_B, int m
       cudaMemcpy(ws->rope_sin, sn.data(), sn.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
       cudaMemset(ws->err, 0, 2 * sizeof(int)) != cudaSuccess ||
       cudaMemset(ws->attn_sync, 0, (size_t)ws->attn_sync_len * sizeof(int)) != cudaSuccess ||
-      (ws->ffn_sync && cudaMemset(ws->ffn_sync, 0, 8 * sizeof(int)) != cudaSuccess)) {
+      (ws->ffn_sync && cudaMemset(ws->ffn_sync, 0, 8 * sizeof(int)) != cudaSuccess) ||
+      (ws->gs_counter && cudaMemset(ws->gs_counter, 0, 2 * kWsCounters * sizeof(int)) != cudaSuccess)) {
     spa_workspace_free(ws);
     return fail(SPA_ERR_CUDA, "workspace initialisation copy failed");
   }
@@ -534,6 +542,7 @@ extern "C" int spa_workspace_status(spa_workspace* ws, void* stream) {
   // a kernel that gave up may have left split counters behind: start them afresh
   SPA_CK(cudaMemset(ws->attn_sync, 0, (size_t)ws->attn_sync_len * sizeof(int)));
   if (ws->ffn_sync) SPA_CK(cudaMemset(ws->ffn_sync, 0, 8 * sizeof(int)));
+  if (ws->gs_counter) SPA_CK(cudaMemset(ws->gs_counter, 0, 2 * kWsCounters * sizeof(int)));
   if (h[0] & DEVERR_TIMEOUT) return fail(SPA_ERR_TIMEOUT, "device wait timed out (site %d)", h[1]);
   return fail(SPA_ERR_DEVICE, "device check failed: bits 0x%x site %d", h[0], h[1]);
 }
@@ -756,8 +765,10 @@ static int run_tc(int mode, int BN, TcGemmParams& p, int M, int n_tiles, int spl
 // sums a row's squares over 128-feature tiles, so one block.
 struct WsShape {
   int NT, nacc, n_tiles, splits;
+  bool global;  // the splits are separate CTAs that reduce through global memory
 };
-static WsShape ws_shape(int mode, bool gateup, bool fold, int M, int K, int rows) {
+// g_floats: the global split-K scratch (0: none).
+static WsShape ws_shape(int mode, bool gateup, bool fold, int M, int K, int rows, size_t g_floats = 0) {
   WsShape sh;
   sh.NT = ((M + 31) / 32) * 32;
   const int NT = sh.NT;
@@ -781,19 +792,42 @@ static WsShape ws_shape(int mode, bool gateup, bool fold, int M, int K, int rows
   sh.nacc = nacc;
   sh.n_tiles = (rows + feat - 1) / feat;
   sh.splits = plan_ws_splits(mode, nacc, sh.n_tiles, K / 64);
-  if (const char* env = std::getenv("SPA_WS_SPLITS")) {  // tuning override, 1..8
+  sh.global = false;
+  // a split-K through global memory where it covers more SMs than the
+  // clusters can (QKV: 48 two-block tiles x 3 splits = 144 CTAs, where only 45
+  // clusters of 3 fit).  Tuning override SPA_WS_GLOBAL: 0 keeps the clusters;
+  // 2..8 takes that many global splits when the grid is resident at once.
+  const char* genv = std::getenv("SPA_WS_GLOBAL");
+  const int gforce = genv ? std::atoi(genv) : -1;
+  if (g_floats > 0 && sh.n_tiles <= kWsCounters && gforce != 0) {
+    const size_t per = (size_t)sh.n_tiles * NT * nacc * 128;
+    const int g_max = (int)std::min<size_t>(8, g_floats / per);
+    int sg = plan_ws_global_splits(mode, nacc, sh.n_tiles, K / 64, g_max);
+    if (gforce >= 2 && gforce <= g_max && K / 64 >= gforce && ws_resident_ctas(mode, nacc) >= sh.n_tiles * gforce)
+      sg = gforce;
+    if (sg > 1) {
+      sh.splits = sg;
+      sh.global = true;
+    }
+  }
+  if (const char* env = std::getenv("SPA_WS_SPLITS")) {  // tuning override, 1..8 (clusters)
     const int v = std::atoi(env);
-    if (v >= 1 && v <= 8 && K / 64 >= v) sh.splits = v;
+    if (v >= 1 && v <= 8 && K / 64 >= v) {
+      sh.splits = v;
+      sh.global = false;
+    }
   }
   return sh;
 }
 
-static int run_ws(int mode, bool gateup, TcWsParams& p, const void* X, int M, int K, int rows,
-                  cudaStream_t s, Profiler* prof, Work w) {
+static int run_ws(int mode, bool gateup, TcWsParams& p, spa_workspace* ws, const void* X, int M, int K,
+                  int rows, cudaStream_t s, Profiler* prof, Work w) {
   if (M <= 0) return SPA_OK;
   if (M > 256) return fail(SPA_ERR_SHAPE, "weight-stationary GEMM takes at most 256 tokens");
-  const WsShape sh = ws_shape(mode, gateup, p.ep.x2 != nullptr, M, K, rows);
+  const WsShape sh = ws_shape(mode, gateup, p.ep.x2 != nullptr, M, K, rows, ws->gs_part ? ws->gs_part_floats : 0);
   const int NT = sh.NT, nacc = sh.nacc, n_tiles = sh.n_tiles;
+  p.part = sh.global ? ws->gs_part : nullptr;
+  p.counter = sh.global ? ws->gs_counter : nullptr;
   if (encode_bf16_map_box(&p.tmX, X, (uint64_t)M, (uint64_t)K, (uint32_t)NT))
     return fail(SPA_ERR_CUDA, "tensor map for the token operand failed");
   int cols = 32;
@@ -989,7 +1023,7 @@ static int run_attn_half(spa_layer* L, const void* H, const int32_t* idx, int tp
       std::memset(&p, 0, sizeof(p));
       p.tmW[0] = L->tm_wq; p.tmW[1] = L->tm_wk; p.tmW[2] = L->tm_wv;
       p.b_mode = B_CONCAT3; p.b_rows_per_src = d; p.ep = ep;
-      SPA_TRY(run_ws(EPI_QKV, false, p, ws->X, M, d, 3 * d, s, prof,
+      SPA_TRY(run_ws(EPI_QKV, false, p, ws, ws->X, M, d, 3 * d, s, prof,
                      Work{SPA_PROF_QKV, 3.0 * d * d * es + Md * es + 3.0 * Md * es, 6.0 * Md * d}));
     } else if (bf) {
       TcGemmParams p;
@@ -1130,7 +1164,7 @@ static int run_ffn_half(spa_layer* L, const void* H, const int32_t* idx, int tps
         p.ep.ss_part = ws->ss_part;
         p.ep.ss_tiles = (d + 127) / 128;
       }
-      SPA_TRY(run_ws(EPI_RESID, false, p, Ob, M, d, d, s, prof,
+      SPA_TRY(run_ws(EPI_RESID, false, p, ws, Ob, M, d, d, s, prof,
                      Work{SPA_PROF_OPROJ, (double)d * d * es + 4.0 * Md * es + d * es, 2.0 * Md * d + 3.0 * Md}));
     } else if (bf) {
       TcGemmParams p;
@@ -1180,7 +1214,7 @@ static int run_ffn_half(spa_layer* L, const void* H, const int32_t* idx, int tps
         p.ep.ss_tiles = (d + 127) / 128;
         p.ep.eps = D.rms_eps;
       }
-      SPA_TRY(run_ws(EPI_SWIGLU, true, p, ws->X2, M, d, F, s, prof,
+      SPA_TRY(run_ws(EPI_SWIGLU, true, p, ws, ws->X2, M, d, F, s, prof,
                      Work{SPA_PROF_GATEUP, 2.0 * F * d * es + Md * es + (double)M * F * es, 4.0 * Md * F}));
     } else if (bf) {
       TcGemmParams p;
@@ -1217,7 +1251,7 @@ static int run_ffn_half(spa_layer* L, const void* H, const int32_t* idx, int tps
       TcWsParams p;
       std::memset(&p, 0, sizeof(p));
       p.tmW[0] = L->tm_wd; p.b_mode = B_SINGLE; p.b_rows_per_src = d; p.ep = ep;
-      SPA_TRY(run_ws(EPI_RESID_SCATTER, false, p, ws->A, M, F, d, s, prof,
+      SPA_TRY(run_ws(EPI_RESID_SCATTER, false, p, ws, ws->A, M, F, d, s, prof,
                      Work{SPA_PROF_DOWN, (double)d * F * es + (double)M * F * es + 2.0 * Md * es, 2.0 * Md * F}));
     } else if (bf) {
       TcGemmParams p;
@@ -1592,7 +1626,7 @@ static int lm_head_impl(spa_model* m, const int32_t* pos, int u, int32_t* tok_ou
     TcWsParams p;
     std::memset(&p, 0, sizeof(p));
     p.tmW[0] = m->tm_lm; p.b_mode = B_SINGLE; p.b_rows_per_src = m->desc.vocab; p.ep = ep;
-    SPA_TRY(run_ws(EPI_ARGMAX, false, p, ws->X, M, d, m->desc.vocab, s, &ws->prof, wl));
+    SPA_TRY(run_ws(EPI_ARGMAX, false, p, ws, ws->X, M, d, m->desc.vocab, s, &ws->prof, wl));
     tiles = p.ep.n_tiles;
   } else if (D.dtype == SPA_BF16) {
     tiles = (m->desc.vocab + 255) / 256;

@@ -608,6 +608,37 @@ __host__ __device__ inline int ws_stages(int nacc, int NT) {
   return st < kWsMaxStages ? st : kWsMaxStages;
 }
 
+// tile[row][0..FEAT) <- sum over splits q = 0..S-1 (in that order) of the
+// partial rows c0 + row, row < nt, from base + q * slot ([NT][FEAT] fp32
+// each): U items of QMAX loads in flight per thread (S <= QMAX).
+template <int U, int QMAX, int FEAT>
+__device__ __forceinline__ void ws_sum_splits(const float* base, size_t slot, int S, int c0, int nt, float* tile,
+                                              int ld, int tid, int nthr) {
+  constexpr int C4 = FEAT / 4;
+  const int total = nt * C4;
+  for (int it0 = tid; it0 < total; it0 += U * nthr) {
+    float4 v[U][QMAX];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int it = it0 + u * nthr;
+      const size_t off = (size_t)(c0 + it / C4) * FEAT + (it % C4) * 4;
+#pragma unroll
+      for (int q = 0; q < QMAX; ++q)
+        if (q < S && it < total) v[u][q] = __ldcg(reinterpret_cast<const float4*>(base + q * slot + off));
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int it = it0 + u * nthr;
+      if (it >= total) continue;
+      float4 acc = v[u][0];
+#pragma unroll
+      for (int q = 1; q < QMAX; ++q)
+        if (q < S) { acc.x += v[u][q].x; acc.y += v[u][q].y; acc.z += v[u][q].z; acc.w += v[u][q].w; }
+      *reinterpret_cast<float4*>(tile + (it / C4) * ld + (it % C4) * 4) = acc;
+    }
+  }
+}
+
 // A CTA that gave up (a bounded wait ran out) must not release its shared and
 // tensor memory while its copies or tensor-core operations are in flight:
 // thread 0 waits (bounded, ignoring the abort) for the accumulator commit and
@@ -667,6 +698,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ int s_issued, s_consumed;  // stages whose boxes were requested / consumed by the MMA
+  __shared__ int s_all_in;
   __shared__ int2 s_rows[256];  // >= CHUNK
   __shared__ float s_scale[MODE == EPI_SWIGLU ? 256 : 1];  // the folded FFN RMSNorm, per token
 
@@ -685,6 +717,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
   // same token tile at once (the sum order stays fixed per tile)
   const int rot = nk > 0 ? (n_tile * 5) % nk : 0;
   int* err = p.ep.err;
+  // token rows whose epilogue this CTA runs first: with split-K through
+  // global memory, split q takes rows [q*NT/S, (q+1)*NT/S); otherwise from 0
+  const bool g_split = p.part != nullptr && S > 1;
+  const int g_r0 = g_split ? (split * NT) / S : 0;
+  const int g_r1 = g_split ? ((split + 1) * NT) / S : NT;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -766,7 +803,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
   } else if (warp >= 2) {
     // idle during the main loop: fetch the first chunk's row indices now
     griddep_wait();
-    stage_rows(p.ep, 0, 0, min(CHUNK, NT), s_rows, threadIdx.x - 64, kThreads - 64);
+    stage_rows(p.ep, g_r0, 0, min(CHUNK, g_r1 - g_r0), s_rows, threadIdx.x - 64, kThreads - 64);
     if constexpr (MODE == EPI_SWIGLU) {
       // and the per-token scale of the folded FFN RMSNorm: 1 / sqrt(mean(H1^2)
       // + eps), the tiles' partial sums added in tile order
@@ -798,6 +835,83 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
   float* tile = reinterpret_cast<float*>(smem);
   const int M = p.ep.M;
   const int q4 = warp & 3, half = warp >> 2;
+  if (g_split) {
+    // ---- split-K through global memory: publish this split's partial tile,
+    // wait until every split of the tile has, then reduce this split's share
+    // of the token rows (summed in split order 0..S-1) and run its epilogue
+    {
+      const int f = q4 * 32 + lane;
+      float* mine = p.part + ((size_t)n_tile * S + split) * (size_t)NT * FEAT + f;
+#pragma unroll 1
+      for (int a = 0; a < NACC; ++a) {
+#pragma unroll 1
+        for (int c = 32 * half; c < NT; c += 64) {
+          float v[32];
+          if (good && nk > 0) {
+            tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + (uint32_t)(a * NT + c), v);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.f;
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) __stcg(mine + (size_t)(c + j) * FEAT + a * 128, v[j]);
+        }
+      }
+    }
+    tc_fence_before();
+    __threadfence();
+    __syncthreads();
+    int* arrive = p.counter + n_tile;
+    int* leave = p.counter + kWsCounters + n_tile;
+    if (threadIdx.x == 0) {
+      atomicAdd(arrive, 1);
+      // every split of the tile is resident (the host keeps the grid within
+      // one wave), so this wait ends unless a split gave up
+      s_all_in = flag_wait(arrive, S, err, 217) ? 1 : 0;
+      if (!s_all_in) abort_flag = 1;
+    }
+    __syncthreads();
+    const bool all_in = s_all_in != 0;
+    __threadfence();
+    const float* base = p.part + (size_t)n_tile * S * (size_t)NT * FEAT;
+    const size_t slot = (size_t)NT * FEAT;
+    for (int c0 = g_r0; c0 < g_r1; c0 += CHUNK) {
+      const int nt = min(CHUNK, g_r1 - c0);
+      if (all_in) {
+        if (S <= 4)
+          ws_sum_splits<4, 4, FEAT>(base, slot, S, c0, nt, tile, LD, threadIdx.x, kThreads);
+        else
+          ws_sum_splits<2, 8, FEAT>(base, slot, S, c0, nt, tile, LD, threadIdx.x, kThreads);
+      }
+      if (c0 > g_r0) stage_rows(p.ep, c0, 0, nt, s_rows, threadIdx.x, kThreads);  // first: staged above
+      __syncthreads();
+      // the partial rows just summed are dead: drop their L2 lines without a
+      // write-back (otherwise the next kernels pay for writing them to HBM);
+      // each 128-byte line of these rows is read by this CTA alone
+      if (all_in) {
+        constexpr int LINES = FEAT * 4 / 128;  // per row of one split's partial
+        for (int it = threadIdx.x; it < S * nt * LINES; it += kThreads) {
+          const int q = it / (nt * LINES), rl = it % (nt * LINES);
+          const float* line = base + q * slot + (size_t)(c0 + rl / LINES) * FEAT + (rl % LINES) * 32;
+          asm volatile("discard.global.L2 [%0], 128;" ::"l"(line) : "memory");
+        }
+      }
+      if (good && all_in && c0 < M)
+        run_epilogue<MODE, FEAT, __nv_bfloat16>(tile, LD, 0, nt, c0, n_tile, p.ep, s_rows, threadIdx.x, kThreads,
+                                                (MODE == EPI_SWIGLU && p.ep.ss_part) ? s_scale + c0 : nullptr);
+      __syncthreads();
+    }
+    if (threadIdx.x == 0 && atomicAdd(leave, 1) == S - 1) {
+      // the last split out: every split has passed its wait, so the counters
+      // can start afresh for the next launch
+      *arrive = 0;
+      *leave = 0;
+    }
+    ws_drain_on_abort(abort_flag, &accum_bar, full_bar, STAGES, s_consumed, s_issued, err);
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, (uint32_t)p.tmem_cols);
+    return;
+  }
   if constexpr (MODE == EPI_SWIGLU && NACC == 2) {
     if (S == 1) {
       // no reduction: thread (quadrant, lane) owns feature f, whose gate and
@@ -895,7 +1009,7 @@ static cudaError_t launch_ws_typed(const TcWsParams& p, int n_tiles, int splits,
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = splits;
+  attr[0].val.clusterDim.x = p.part ? 1 : splits;  // global split-K: separate CTAs
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -949,11 +1063,46 @@ static int ws_max_clusters(int splits) {
 
 cudaError_t launch_tc_ws(int mode, int nacc, const TcWsParams& p, int n_tiles, int splits,
                          cudaStream_t stream) {
+  if (p.part && (p.counter == nullptr || n_tiles > kWsCounters || splits > 8)) return cudaErrorInvalidValue;
 #define SPA_WS_CASE(M_, A_) \
   if (mode == M_ && nacc == A_) return launch_ws_typed<M_, A_>(p, n_tiles, splits, stream);
   SPA_WS_MODES(SPA_WS_CASE)
 #undef SPA_WS_CASE
   return cudaErrorInvalidValue;
+}
+
+int ws_resident_ctas(int mode, int nacc) {
+  int resident = 0;
+#define SPA_WS_FIT(M_, A_) \
+  if (mode == M_ && nacc == A_) resident = ws_max_clusters<M_, A_>(1);
+  SPA_WS_MODES(SPA_WS_FIT)
+#undef SPA_WS_FIT
+  return resident;
+}
+
+int plan_ws_global_splits(int mode, int nacc, int n_tiles, int KB, int g_max) {
+  const int resident = ws_resident_ctas(mode, nacc);
+  // the cluster plan's estimate (see plan_ws_splits)
+  const int sc = plan_ws_splits(mode, nacc, n_tiles, KB);
+  int fit = 0;
+#define SPA_WS_FIT(M_, A_) \
+  if (mode == M_ && nacc == A_) fit = ws_max_clusters<M_, A_>(sc);
+  SPA_WS_MODES(SPA_WS_FIT)
+#undef SPA_WS_FIT
+  const double c_cost = fit > 0 ? ((n_tiles + fit - 1) / fit) * ((KB + sc - 1) / sc + 12.0) : 1e30;
+  int best = 0;
+  double best_cost = c_cost;
+  for (int s = 2; s <= 8 && s <= g_max; ++s) {
+    if (KB / s < 4 || n_tiles * s > resident) continue;
+    // one wave; each split also stores its partial tile and reduces its share
+    // of the rows from every split's (about six k-blocks' time)
+    const double cost = (KB + s - 1) / s + 12.0 + 6.0;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
 }
 
 // Split-K plan for the weight-stationary GEMM: estimated time ~ waves x

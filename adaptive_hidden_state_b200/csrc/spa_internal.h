@@ -89,8 +89,17 @@ struct alignas(64) TcWsParams {
   int tmem_cols;       // power of two >= NACC * NT
   int b_mode;
   int b_rows_per_src;
+  // Split-K across separate CTAs (no cluster; the whole grid resident at
+  // once): every split stores its fp32 partial tile [NT][NACC * 128] at part +
+  // ((tile * splits + split) * NT) * NACC * 128, counts itself in on
+  // counter[tile], waits (bounded) for the tile's other splits, then sums the
+  // splits in order 0..splits-1 for its share of the token rows and runs their
+  // epilogue; the last split out (counter[kWsCounters + tile]) resets both.
+  float* part;         // null: the splits of a tile form a cluster (DSMEM reduction)
+  int* counter;        // [2 * kWsCounters], zero between launches
   EpiParams ep;
 };
+constexpr int kWsCounters = 4096;  // tiles of a split-K through global memory
 
 // Stream-K weight-streaming GEMM (spa_streamk.cu): units (tile of nacc x 128
 // output features, 64-column k-block) split evenly over the grid's CTAs; each
@@ -164,8 +173,14 @@ cudaError_t launch_tc_gemm(int mode, int BN, int BM, const TcGemmParams& p, int 
 // Weight-stationary tcgen05 GEMM for M <= 256 tokens: 128 weight rows per
 // CTA (NACC = 2: gate and up rows) against all tokens; same epilogues.
 cudaError_t launch_tc_ws(int mode, int nacc, const TcWsParams& p, int n_tiles, int splits,
-                         cudaStream_t stream);
+                         cudaStream_t stream);  // p.part set: splits of separate CTAs (no cluster)
 int plan_ws_splits(int mode, int nacc, int n_tiles, int KB);
+// Split count for a split-K through global memory (0: none fits): the whole
+// grid resident at once, at most g_max splits (the scratch), and cheaper than
+// the cluster plan of plan_ws_splits by the same estimate.
+int plan_ws_global_splits(int mode, int nacc, int n_tiles, int KB, int g_max);
+// CTAs of this weight-stationary GEMM the current device holds at once.
+int ws_resident_ctas(int mode, int nacc);
 // The persistent FFN kernel over `grid` CTAs (at most one per SM).
 cudaError_t launch_ffn_persistent(const FfnParams& p, int grid, cudaStream_t stream);
 int ffn_max_seg();    // segments per tile the reducers take

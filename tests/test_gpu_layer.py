@@ -176,6 +176,29 @@ def test_bf16_wide_weight_tiles(monkeypatch, nacc, B, N, k):
     _step(lp, cache, ocs, H2, k)
 
 
+MID_BF16 = synth.LayerShape(d=1024, n_heads=8, head_dim=128, ffn=1536, r=64)
+
+
+@pytest.mark.parametrize("glob", ["0", "2", "3", "5", "8", ""])
+@pytest.mark.parametrize("B,N,k", [(1, 200, 96), (2, 160, 33), (1, 300, 200)])
+def test_bf16_ws_global_split_k(monkeypatch, glob, B, N, k):
+    # the weight-stationary GEMMs with their k-blocks split over separate CTAs
+    # that reduce through global memory (each split publishes its fp32 partial
+    # tile, waits for the tile's other splits, and sums its share of the token
+    # rows in split order): 2, 3, 5 and 8 splits of every GEMM whose grid stays
+    # resident (QKV 24 tiles of 16 k-blocks, gate/up 12, O-proj and down 8 of 16
+    # and 24), the clusters only (0) and the planner's choice.  Two steps: the
+    # second finds the counters reset by the first.
+    if glob:
+        monkeypatch.setenv("SPA_WS_GLOBAL", glob)
+    lp = LayerPair(spa, MID_BF16, seed=70 + k, dtype=spa.SPA_BF16, max_B=2, max_N=300, std=0.03)
+    H = synth.hidden_states(B, N, MID_BF16.d, seed=k + 7, bf16=True)
+    cache, ocs = _run_fill(lp, H)
+    H2, _ = synth.drift_rows(H, 0.2, 0.5, seed=k + 8, bf16=True)
+    _step(lp, cache, ocs, H2, k)
+    _step(lp, cache, ocs, H, k)
+
+
 @pytest.mark.parametrize("nacc", ["1", "2"])
 @pytest.mark.parametrize("grid", ["1", "5", "12", "24"])
 @pytest.mark.parametrize("B,N,k", [(1, 200, 96), (2, 160, 33), (1, 300, 200)])
