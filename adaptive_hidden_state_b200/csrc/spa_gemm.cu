@@ -386,6 +386,19 @@ __host__ __device__ constexpr int tc_smem_bytes(int BN, int BM = 128) {
   return tc_stages(BN, BM) * ((BM / 128) * kTcABytes + BN * 128) + 1024;
 }
 
+// A CTA that gave up (a bounded wait ran out) must not release its shared and
+// tensor memory while its copies or tensor-core operations are in flight:
+// thread 0 waits (bounded, ignoring the abort) for the accumulator commit and
+// for every requested stage the MMA did not consume; then all threads proceed.
+__device__ __forceinline__ void ws_drain_on_abort(int abort, uint64_t* accum_bar, uint64_t* full_bar, int stages,
+                                                  int consumed, int issued, int* err) {
+  if (abort && threadIdx.x == 0) {
+    mbar_drain_bounded(accum_bar, 0, err, 215);
+    for (int it = consumed; it < issued; ++it) mbar_drain_bounded(&full_bar[it % stages], (it / stages) & 1, err, 216);
+  }
+  __syncthreads();
+}
+
 template <int MODE, int BN, int BM>
 __global__ void __launch_bounds__(kThreads, BN == 128 ? 2 : 1) tc_gemm_kernel(const __grid_constant__ TcGemmParams p) {
   constexpr int STAGES = tc_stages(BN, BM);
@@ -404,6 +417,7 @@ __global__ void __launch_bounds__(kThreads, BN == 128 ? 2 : 1) tc_gemm_kernel(co
   __shared__ __align__(8) uint64_t accum_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  __shared__ int s_issued, s_consumed;  // stages whose boxes were requested / consumed by the MMA
   __shared__ int2 s_rows[128];
 
   griddep_launch_dependents();
@@ -423,6 +437,8 @@ __global__ void __launch_bounds__(kThreads, BN == 128 ? 2 : 1) tc_gemm_kernel(co
     }
     mbar_init(&accum_bar, 1);
     abort_flag = 0;
+    s_issued = 0;
+    s_consumed = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -433,14 +449,39 @@ __global__ void __launch_bounds__(kThreads, BN == 128 ? 2 : 1) tc_gemm_kernel(co
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+
+  // The B operand is always a weight matrix, which no earlier kernel writes:
+  // the weight boxes of the first stages are requested before
+  // griddepcontrol.wait, so they stream while the previous kernel finishes;
+  // the token rows (A) follow the wait.
+  const int pre = nk < STAGES ? nk : STAGES;
+  if (warp == 0 && lane == 0) {
+    s_issued = pre;
+    for (int it = 0; it < pre; ++it) {
+      uint8_t* sb = smem + it * STAGE_BYTES + A_BYTES;
+      mbar_arrive_expect_tx(&full_bar[it], STAGE_BYTES);
+      const int kx = (kb0 + it) * 64;
+#pragma unroll
+      for (int h = 0; h < BN / 128; ++h) {
+        int src, row;
+        b_source<BN>(p, n_tile, h, src, row);
+        tma_load_2d(sb + h * 128 * 128, &p.tmB[src], &full_bar[it], kx, row);
+      }
+    }
+  }
   griddep_wait();  // the token rows and the epilogue operands come from earlier kernels
 
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&p.tmA);
-    for (int it = 0; it < nk; ++it) {
+    for (int it = 0; it < pre; ++it) {
+      uint8_t* sa = smem + it * STAGE_BYTES;
+      const int kx = (kb0 + it) * 64;
+#pragma unroll
+      for (int a = 0; a < NA; ++a) tma_load_2d(sa + a * kTcABytes, &p.tmA, &full_bar[it], kx, m_tile * BM + a * 128);
+    }
+    for (int it = pre; it < nk; ++it) {
       const int s = it % STAGES;
-      if (it >= STAGES && !mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1, &abort_flag, err, 201))
-        break;
+      if (!mbar_wait(&empty_bar[s], ((it / STAGES) - 1) & 1, &abort_flag, err, 201)) break;
       uint8_t* sa = smem + s * STAGE_BYTES;
       uint8_t* sb = sa + A_BYTES;
       mbar_arrive_expect_tx(&full_bar[s], STAGE_BYTES);
@@ -453,12 +494,14 @@ __global__ void __launch_bounds__(kThreads, BN == 128 ? 2 : 1) tc_gemm_kernel(co
         b_source<BN>(p, n_tile, h, src, row);
         tma_load_2d(sb + h * 128 * 128, &p.tmB[src], &full_bar[s], kx, row);
       }
+      s_issued = it + 1;
     }
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc = idesc_bf16_f32(128, BN);
     for (int it = 0; it < nk; ++it) {
       const int s = it % STAGES;
       if (!mbar_wait(&full_bar[s], (it / STAGES) & 1, &abort_flag, err, 202)) break;
+      s_consumed = it + 1;
       tc_fence_after();
       const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
       const uint64_t db = smem_desc_sw128(sa + A_BYTES);
@@ -486,7 +529,11 @@ __global__ void __launch_bounds__(kThreads, BN == 128 ? 2 : 1) tc_gemm_kernel(co
     // the a-th 128-row half of the tile: accumulator -> shared memory, split-K
     // reduction across the cluster, epilogue
     if (a > 0) __syncthreads();  // the previous half's epilogue is done with the tile
-    if (good) {
+    const int gm0 = m_tile * BM + a * 128;
+    // rows of this half that hold tokens: the rest are never read, so they are
+    // neither moved out of TMEM nor reduced
+    const int mv = min(128, max(0, p.ep.M - gm0));
+    if (good && (warp & 3) * 32 < mv) {
       const int q = warp & 3, half = warp >> 2;
       float* dst = tile + (q * 32 + lane) * LD;
 #pragma unroll 1
@@ -505,15 +552,18 @@ __global__ void __launch_bounds__(kThreads, BN == 128 ? 2 : 1) tc_gemm_kernel(co
     }
     tc_fence_before();
     __syncthreads();
-    if (a == NA - 1 && warp == 0) tmem_dealloc(tmem, NA * BN);
+    if (a == NA - 1) {
+      ws_drain_on_abort(abort_flag, &accum_bar, full_bar, STAGES, s_consumed, s_issued, err);
+      tc_fence_after();
+      if (warp == 0) tmem_dealloc(tmem, NA * BN);
+    }
 
-    const int gm0 = m_tile * BM + a * 128;
     int r0 = 0, r1 = 128;
     if (S > 1) {
       cluster_sync();
       const int q = (int)cluster_ctarank();
-      r0 = (q * 128) / S;
-      r1 = ((q + 1) * 128) / S;
+      r0 = (q * mv) / S;
+      r1 = ((q + 1) * mv) / S;
       if (good) cluster_reduce_rows<BN>(tile, LD, r0, r1, S, threadIdx.x, kThreads);
       cluster_sync();
     }
@@ -637,19 +687,6 @@ __device__ __forceinline__ void ws_sum_splits(const float* base, size_t slot, in
       *reinterpret_cast<float4*>(tile + (it / C4) * ld + (it % C4) * 4) = acc;
     }
   }
-}
-
-// A CTA that gave up (a bounded wait ran out) must not release its shared and
-// tensor memory while its copies or tensor-core operations are in flight:
-// thread 0 waits (bounded, ignoring the abort) for the accumulator commit and
-// for every requested stage the MMA did not consume; then all threads proceed.
-__device__ __forceinline__ void ws_drain_on_abort(int abort, uint64_t* accum_bar, uint64_t* full_bar, int stages,
-                                                  int consumed, int issued, int* err) {
-  if (abort && threadIdx.x == 0) {
-    mbar_drain_bounded(accum_bar, 0, err, 215);
-    for (int it = consumed; it < issued; ++it) mbar_drain_bounded(&full_bar[it % stages], (it / stages) & 1, err, 216);
-  }
-  __syncthreads();
 }
 
 // The NACC weight boxes (128 rows x 64 columns each) of one k-block of
@@ -914,13 +951,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
   }
   if constexpr (MODE == EPI_SWIGLU && NACC == 2) {
     if (S == 1) {
-      // no reduction: thread (quadrant, lane) owns feature f, whose gate and
-      // up accumulators sit in the same TMEM lane; silu(g) * u goes straight
-      // from registers to A, 32 tokens per TMEM load (64-byte rows of 32
-      // features per warp store), with no shared-memory pass
+      // no reduction: thread (quadrant, lane) owns feature q4*32 + lane, whose
+      // gate and up accumulators sit in the same TMEM lane; silu(g) * u is
+      // rounded to bf16 into a [token][128-feature] tile in the (idle) ring,
+      // which then leaves as 16-byte row chunks (two 256-byte row slabs per
+      // warp store instead of 64-byte pieces)
+      __nv_bfloat16* T = reinterpret_cast<__nv_bfloat16*>(smem);
       if (good && nk > 0) {
-        const int f = n_tile * 128 + q4 * 32 + lane;
-        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.ep.out);
         const uint32_t row_base = tmem + ((uint32_t)(q4 * 32) << 16);
 #pragma unroll 1
         for (int c = 32 * half; c < NT; c += 64) {
@@ -934,10 +971,22 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
               u[j] *= s_scale[c + j];
             }
           }
-          if (f < p.ep.n_out) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (c + j < M) out[(size_t)(c + j) * p.ep.n_out + f] = __float2bfloat16_rn(silu(g[j]) * u[j]);
+          for (int j = 0; j < 32; ++j) T[(c + j) * 128 + q4 * 32 + lane] = __float2bfloat16_rn(silu(g[j]) * u[j]);
+        }
+      }
+      __syncthreads();
+      if (good && nk > 0) {
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.ep.out);
+        const int n_out = p.ep.n_out;
+        for (int it = threadIdx.x; it < M * 16; it += kThreads) {
+          const int t = it >> 4, f0 = n_tile * 128 + (it & 15) * 8;
+          const __nv_bfloat16* src = T + t * 128 + (it & 15) * 8;
+          __nv_bfloat16* dst = out + (size_t)t * n_out + f0;
+          if ((n_out & 7) == 0 && f0 + 8 <= n_out) {
+            *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+          } else {
+            for (int e = 0; e < 8 && f0 + e < n_out; ++e) dst[e] = src[e];
           }
         }
       }
