@@ -58,6 +58,51 @@ __device__ void stage_rows(const EpiParams& ep, int gm0, int row_begin, int row_
   }
 }
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// While the main loop streams the weights, pull into L2 the global operands
+// that the epilogue of rows gm0 .. gm0 + nrows - 1 will read: the residual
+// rows' slice of this column tile (EPI_RESID: H[b, I_t]), the rotary table
+// rows of the tokens' positions (EPI_QKV, Q and K tiles) and the cached proxy
+// rows (EPI_PROXY).  One prefetch per 128-byte line; a hint, so no result
+// depends on it.
+template <int MODE, int FEAT, typename T>
+__device__ void prefetch_epilogue_rows(const EpiParams& ep, int gm0, int nrows, int n_tile, int tid,
+                                       int nthr) {
+  if constexpr (MODE == EPI_RESID || MODE == EPI_QKV || MODE == EPI_PROXY) {
+    for (int row = tid; row < nrows; row += nthr) {
+      const int t = gm0 + row;
+      if (t >= ep.M) break;
+      const int b = t / ep.tokens_per_seq;
+      const int pos = ep.idx ? ep.idx[t] : t % ep.tokens_per_seq;
+      if (pos < 0 || pos >= ep.N) continue;
+      const size_t cr = (size_t)b * ep.N + pos;
+      if constexpr (MODE == EPI_RESID) {
+        const char* src = reinterpret_cast<const char*>(reinterpret_cast<const T*>(ep.resid) + cr * ep.d +
+                                                        (size_t)n_tile * FEAT);
+        for (int o = 0; o < FEAT * (int)sizeof(T); o += 128) prefetch_l2(src + o);
+      } else if constexpr (MODE == EPI_QKV) {
+        if ((size_t)n_tile * FEAT < 2 * (size_t)ep.d) {
+          const int hh = ep.head_dim / 2;
+          const char* c = reinterpret_cast<const char*>(ep.rope_cos + (size_t)pos * hh);
+          const char* sn = reinterpret_cast<const char*>(ep.rope_sin + (size_t)pos * hh);
+          for (int o = 0; o < hh * 4; o += 128) {
+            prefetch_l2(c + o);
+            prefetch_l2(sn + o);
+          }
+        }
+      } else {
+        if (!ep.proxy_fill) {
+          const char* pc = reinterpret_cast<const char*>(ep.p_cache + cr * ep.n_out);
+          for (int o = 0; o < ep.n_out * 4; o += 128) prefetch_l2(pc + o);
+        }
+      }
+    }
+  }
+}
+
 template <int MODE, int BN, typename T>
 __device__ void run_epilogue(const float* tile, int ld, int row_begin, int row_end, int gm0,
                              int n_tile, const EpiParams& ep, const int2* s_rows, int tid,
@@ -515,6 +560,11 @@ __global__ void __launch_bounds__(kThreads, BN == 128 ? 2 : 1) tc_gemm_kernel(co
       umma_commit(&empty_bar[s]);
     }
     umma_commit(&accum_bar);
+  } else if (warp >= 2) {
+    // idle during the main loop: the epilogue's operands into L2
+    for (int a = 0; a < NA; ++a)
+      prefetch_epilogue_rows<MODE, BN, __nv_bfloat16>(p.ep, m_tile * BM + a * 128, 128, n_tile, threadIdx.x - 64,
+                                                      kThreads - 64);
   }
   __syncwarp();
 
@@ -660,10 +710,11 @@ __host__ __device__ inline int ws_stages(int nacc, int NT) {
 
 // tile[row][0..FEAT) <- sum over splits q = 0..S-1 (in that order) of the
 // partial rows c0 + row, row < nt, from base + q * slot ([NT][FEAT] fp32
-// each): U items of QMAX loads in flight per thread (S <= QMAX).
+// each), except split `own` (>= 0), whose partial rows are already in the
+// tile: U items of QMAX loads in flight per thread (S <= QMAX).
 template <int U, int QMAX, int FEAT>
-__device__ __forceinline__ void ws_sum_splits(const float* base, size_t slot, int S, int c0, int nt, float* tile,
-                                              int ld, int tid, int nthr) {
+__device__ __forceinline__ void ws_sum_splits(const float* base, size_t slot, int S, int own, int c0, int nt,
+                                              float* tile, int ld, int tid, int nthr) {
   constexpr int C4 = FEAT / 4;
   const int total = nt * C4;
   for (int it0 = tid; it0 < total; it0 += U * nthr) {
@@ -674,7 +725,9 @@ __device__ __forceinline__ void ws_sum_splits(const float* base, size_t slot, in
       const size_t off = (size_t)(c0 + it / C4) * FEAT + (it % C4) * 4;
 #pragma unroll
       for (int q = 0; q < QMAX; ++q)
-        if (q < S && it < total) v[u][q] = __ldcg(reinterpret_cast<const float4*>(base + q * slot + off));
+        if (q < S && it < total)
+          v[u][q] = q == own ? *reinterpret_cast<const float4*>(tile + (it / C4) * ld + (it % C4) * 4)
+                             : __ldcg(reinterpret_cast<const float4*>(base + q * slot + off));
     }
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -841,6 +894,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
     // idle during the main loop: fetch the first chunk's row indices now
     griddep_wait();
     stage_rows(p.ep, g_r0, 0, min(CHUNK, g_r1 - g_r0), s_rows, threadIdx.x - 64, kThreads - 64);
+    prefetch_epilogue_rows<MODE, FEAT, __nv_bfloat16>(p.ep, g_r0, min(CHUNK, g_r1 - g_r0), n_tile,
+                                                      threadIdx.x - 64, kThreads - 64);
     if constexpr (MODE == EPI_SWIGLU) {
       // and the per-token scale of the folded FFN RMSNorm: 1 / sqrt(mean(H1^2)
       // + eps), the tiles' partial sums added in tile order
@@ -876,6 +931,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
     // ---- split-K through global memory: publish this split's partial tile,
     // wait until every split of the tile has, then reduce this split's share
     // of the token rows (summed in split order 0..S-1) and run its epilogue
+    // this split's own share of the rows stays in shared memory (the tile,
+    // row c - g_r0) when it fits one epilogue chunk; only the other rows go out
+    const bool own_in_tile = g_r1 - g_r0 <= CHUNK;
     {
       const int f = q4 * 32 + lane;
       float* mine = p.part + ((size_t)n_tile * S + split) * (size_t)NT * FEAT + f;
@@ -891,7 +949,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
             for (int j = 0; j < 32; ++j) v[j] = 0.f;
           }
 #pragma unroll
-          for (int j = 0; j < 32; ++j) __stcg(mine + (size_t)(c + j) * FEAT + a * 128, v[j]);
+          for (int j = 0; j < 32; ++j) {
+            const int t = c + j;
+            if (own_in_tile && t >= g_r0 && t < g_r1) tile[(t - g_r0) * LD + a * 128 + f] = v[j];
+            else __stcg(mine + (size_t)t * FEAT + a * 128, v[j]);
+          }
         }
       }
     }
@@ -915,10 +977,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ws_kernel(const __grid_constan
     for (int c0 = g_r0; c0 < g_r1; c0 += CHUNK) {
       const int nt = min(CHUNK, g_r1 - c0);
       if (all_in) {
+        const int own = own_in_tile ? split : -1;
         if (S <= 4)
-          ws_sum_splits<4, 4, FEAT>(base, slot, S, c0, nt, tile, LD, threadIdx.x, kThreads);
+          ws_sum_splits<4, 4, FEAT>(base, slot, S, own, c0, nt, tile, LD, threadIdx.x, kThreads);
         else
-          ws_sum_splits<2, 8, FEAT>(base, slot, S, c0, nt, tile, LD, threadIdx.x, kThreads);
+          ws_sum_splits<2, 8, FEAT>(base, slot, S, own, c0, nt, tile, LD, threadIdx.x, kThreads);
       }
       if (c0 > g_r0) stage_rows(p.ep, c0, 0, nt, s_rows, threadIdx.x, kThreads);  // first: staged above
       __syncthreads();
